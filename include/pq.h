@@ -1,0 +1,181 @@
+/*
+ * pq.h — C ABI of libpq: online rotation + INT4 quantisation of bf16 activations and the
+ * W4A4 GEMM that consumes the codes, for NVIDIA B200 (sm_100a).
+ *
+ * Sources (pages, by title and section):
+ *   ParoQuant page — codearts.csdn.net article on independent rotation and channel scaling:
+ *       §2.2 (Algorithm A1, greedy disjoint channel pairs per 128-channel group; the three
+ *       properties listed under it), §2.3 (W^ = diag(alpha) W with alpha = exp(beta); 128
+ *       channels share the quantisation parameters), §3.2 (rotation, scaling and quantisation
+ *       fused in one kernel; only the angles are stored), §6.4 (cloud: tensor cores).
+ *   Hadamard page — "神经网络量化技术：Hadamard变换与格码本优化": §2.1 (Walsh–Hadamard matrix,
+ *       entries (-1)^popcount(i&j), 1/sqrt(n)), §4.2 (butterflies; H(AB) = (HA)B), §6.1 (block
+ *       Hadamard).
+ *   RRS page — "Rotated Runtime Smooth: 训练无关的激活平滑器，用于精确的 INT4 推理": main equation
+ *       (X_rot = XR, W_rot = R^-1 W, s_j = max|(X_rot)_j|, Quantize(X_rot diag(s)^-1),
+ *       Y = sum_j (X'_q)_j (W'_q)_j^T s_j), R = (1/sqrt(K))[s_ij], alpha = max|X|/(2^(N-1)-1),
+ *       the INT4 range -8..7, RTN rounding, Fig. 2(a) (Y = (XR)(R^-1 W^T) = XW^T) and Fig. 4
+ *       (scales applied to the interim block results inside the GEMM).
+ *
+ * Conventions
+ *   X  bf16 [T][D] row-major, row stride ldx elements (activations, one row per token).
+ *   W  bf16 [N][D] row-major (Y = X W^T).
+ *   g  group size; only g = 128 is supported.  G = D / g groups per row.
+ *   codes  uint8 [rows][D/2]: byte k holds element 2k in the low nibble and element 2k+1 in
+ *          the high nibble, both two's complement in -8..7.
+ *   scales float32 [rows][G]: per-group scale m/7, m = max |transformed value| in the group
+ *          (0 for an all-zero group, whose codes are 0).
+ *   Codes are q = round_half_even(y / scale) computed in float32 (|q| <= 7).
+ *
+ * Ownership and memory
+ *   Every tensor pointer is a DEVICE pointer owned by the caller, on the current device,
+ *   16-byte aligned.  The library allocates no user-visible buffer.  A plan owns a few small
+ *   device tables and a status word, allocated by pq_make_plan and freed by pq_destroy_plan;
+ *   it is immutable after creation and may be used from several streams at once.
+ *
+ * Errors
+ *   Every call returns pq_status and never throws, aborts or exits.  Arguments are validated
+ *   before anything is launched; a failed call launches nothing and pq_last_error() (thread
+ *   local) describes why.  Launches are asynchronous on the given stream (NULL = legacy default
+ *   stream); device-side faults surface at the caller's next synchronisation, and bounded-wait
+ *   timeouts inside the GEMM are reported by pq_check_status.
+ */
+#ifndef PQ_H_
+#define PQ_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pq_status {
+  PQ_OK = 0,
+  PQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, stride, alignment or plan */
+  PQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. g != 128) */
+  PQ_ERR_CUDA = 3,          /* a CUDA runtime call failed (message in pq_last_error) */
+  PQ_ERR_ALLOC = 4,         /* device allocation for a plan failed */
+  PQ_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up (see pq_check_status) */
+} pq_status;
+
+typedef enum pq_kind {
+  PQ_HADAMARD = 0,          /* block Walsh–Hadamard H_g / sqrt(g) per group */
+  PQ_GIVENS = 1,            /* K layers of disjoint Givens pairs per group, then exp(-beta) */
+  PQ_SMOOTH_HADAMARD = 2    /* runtime per-channel smoothing per 128-token block + Hadamard */
+} pq_kind;
+
+typedef enum pq_out_dtype {
+  PQ_OUT_F32 = 0,
+  PQ_OUT_BF16 = 1           /* round-to-nearest-even of the float32 result */
+} pq_out_dtype;
+
+/* pq_make_plan flags */
+#define PQ_FLAG_SMOOTH_AFTER_ROTATE 0x1u  /* PQ_SMOOTH_HADAMARD: rotate first, then smooth the
+                                             rotated channels (the RRS page's order).  Default:
+                                             smooth the input channels, then rotate. */
+
+/* Pair-slot marker for "no pair" in pair tables. */
+#define PQ_NO_PAIR 0xFFu
+
+typedef struct pq_plan pq_plan;
+
+/*
+ * pq_select_pairs — ParoQuant page §2.2, Algorithm A1, run once per group (host only, no GPU).
+ *   For each group independently: all pairs (i, j), 0 <= i < j < g, in lexicographic order,
+ *   Fisher–Yates shuffled (for i = n-1..1: swap a[i], a[r mod (i+1)], r = next SplitMix64
+ *   output; one SplitMix64 stream seeded with `seed` serves the groups in order 0..G-1).
+ *   Then K layers: scan the shuffled list, take a pair when both channels are still free in
+ *   this layer and the pair was not taken by an earlier layer; stop a layer at N pairs.
+ *   pairs_out: host uint8 [D/g][K][g/2][2], caller-owned; slots past a layer's last pair are
+ *   PQ_NO_PAIR.  Requires g = 128, D % g = 0, 1 <= K <= 64, 1 <= N <= g/2.
+ */
+pq_status pq_select_pairs(uint64_t seed, int D, int g, int K, int N, uint8_t* pairs_out);
+
+/*
+ * pq_make_plan — build the device tables for one transform.
+ *   kind    PQ_HADAMARD | PQ_GIVENS | PQ_SMOOTH_HADAMARD.
+ *   D, g    channels and group size (g must be 128, D % g == 0, D >= g).
+ *   K       Givens layers (1..64); ignored otherwise.
+ *   pairs   host uint8 [D/g][K][g/2][2] (Givens; NULL otherwise).  Within a layer of a group
+ *           the valid pairs (i < j < g) must be disjoint; PQ_NO_PAIR slots are skipped.
+ *   angles  host float32 [D/g][K][g/2] (Givens), radians.  Pair (i, j) with angle t maps the
+ *           column (x_i, x_j) to (cos t x_i - sin t x_j, sin t x_i + cos t x_j); layer 0 first.
+ *   beta    host float32 [D] or NULL (= 0): channel scale alpha = exp(beta) (ParoQuant page
+ *           §2.3).  Activations are multiplied by exp(-beta) after the rotations and weights by
+ *           exp(+beta), so that the product is unchanged before quantisation.
+ *   flags   PQ_FLAG_* bits.
+ *   cos/sin and exp(+-beta) are evaluated on the host in double precision and stored as float.
+ *   The plan is created on the current device.  *out is set only on success.
+ */
+pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int K, const uint8_t* pairs,
+                       const float* angles, const float* beta, uint32_t flags);
+
+/* pq_destroy_plan — frees the plan's device tables (synchronous).  NULL is a no-op. */
+void pq_destroy_plan(pq_plan* plan);
+
+/*
+ * pq_transform_quant — the online activation path, one fused kernel (ParoQuant page §3.2;
+ * RRS page main equation, first and fourth lines):
+ *   y = x M per row, M = H_g/sqrt(g) | R diag(exp(-beta)) | diag(1/s) H_g/sqrt(g) (smoothing
+ *   first; or H_g/sqrt(g) diag(1/s) with PQ_FLAG_SMOOTH_AFTER_ROTATE), then per group
+ *   scale = max|y|/7 and codes = round(y/scale), nibble-packed.
+ *   X          device bf16 [T][ldx] (first D columns used), ldx >= D, ldx % 8 == 0.
+ *   T          rows, T >= 1.
+ *   codes      device uint8 [T][D/2] (dense).
+ *   scales     device float32 [T][D/g] (dense).
+ *   smooth_out PQ_SMOOTH_HADAMARD only: device float32 [ceil(T/128)][D] receiving s, the max
+ *              |x| (or |rotated x|) of each channel over each 128-row block (0 -> 1); may be
+ *              NULL.  Must be NULL for the other kinds.
+ *   stream     cudaStream_t or NULL.
+ */
+pq_status pq_transform_quant(const pq_plan* plan, const void* X, int64_t T, int64_t ldx,
+                             uint8_t* codes, float* scales, float* smooth_out, void* stream);
+
+/*
+ * pq_pack_weights — the offline weight path: w -> w M^{-T} per row (RRS page: W_rot = R^-1 W;
+ * Hadamard page §4.2 H(AB) = (HA)B; OSTQuant page §3.2: the pair is merged into the weights),
+ * then the same per-group quantisation and packing as the activations.
+ *   Hadamard: same rotation.  Givens: same rotations, then exp(+beta).
+ *   Smooth+Hadamard: multiply channel j by smooth_w[j], then rotate (with
+ *   PQ_FLAG_SMOOTH_AFTER_ROTATE: rotate, then multiply by smooth_w); smooth_w NULL = ones.
+ *   W        device bf16 [N][D] dense.   N >= 1.
+ *   smooth_w device float32 [D] or NULL (PQ_SMOOTH_HADAMARD only; must be NULL otherwise).
+ *   codes_W  device uint8 [N][D/2];  scales_W device float32 [N][D/g].
+ */
+pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t N, const float* smooth_w,
+                          uint8_t* codes_W, float* scales_W, void* stream);
+
+/*
+ * pq_w4a4_gemm — Y[t][n] = sum_G scales_A[t][G] * scales_W[n][G] * d_G[t][n], with
+ * d_G = sum over the group's 128 channels of qa * qw computed exactly in int32 on the tensor
+ * cores (tcgen05 kind::i8, accumulator in tensor memory), and the per-group scaling applied to
+ * each group's interim result in float32, groups summed in ascending order (RRS page main
+ * equation, last line, and Fig. 4 step (3) with block size = group size).
+ *   codes_A [T][D/2], scales_A [T][D/g], codes_W [N][D/2], scales_W [N][D/g]: device, dense.
+ *   T >= 1, N >= 1 with N % 16 == 0, D % 128 == 0, g == 128.
+ *   Y device [T][N] float32 (PQ_OUT_F32) or bf16 (PQ_OUT_BF16, RNE of the float32 result).
+ *   Scales must be finite.  Every dot product fits int32 exactly (|d| <= 128*64).
+ */
+pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
+                       const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
+                       pq_out_dtype out_dtype, void* stream);
+
+/*
+ * pq_check_status — synchronises `stream`, then reads and clears the device status words
+ * (the plan's, if plan != NULL, and the GEMM's).  Returns PQ_ERR_TIMEOUT if a bounded
+ * device-side wait gave up since the last check (the affected output is incomplete),
+ * PQ_ERR_CUDA if the stream reports an error, PQ_OK otherwise.
+ */
+pq_status pq_check_status(const pq_plan* plan, void* stream);
+
+/* Static description of a status code. */
+const char* pq_status_string(pq_status status);
+
+/* Detail of the last failure on the calling thread ("" if none).  Valid until the next call. */
+const char* pq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PQ_H_ */

@@ -1,0 +1,74 @@
+// Internal declarations shared by the host code and the kernel launchers of libpq.
+#pragma once
+
+#include <cstdint>
+#include <cstdio>
+#include <string>
+
+#include <cuda_runtime.h>
+
+#include "../../include/pq.h"
+
+namespace pq {
+
+constexpr int kGroup = 128;            // the only supported group size
+constexpr int kSmoothBlock = 128;      // rows per runtime-smoothing block
+
+// One Givens pair of one layer of one group, as the kernels read it (16 bytes).
+struct GivensPair {
+  uint32_t ij;   // i | j << 16  (i < j < 128)
+  float c;       // cos(theta)
+  float s;       // sin(theta)
+  uint32_t pad;
+};
+
+}  // namespace pq
+
+// Device status word bits.
+#define PQ_DEV_TIMEOUT 0x1u
+
+struct pq_plan {
+  pq_kind kind;
+  int D;
+  int g;
+  int G;
+  int K;
+  uint32_t flags;
+  int device;
+  // Givens: pairs compacted per (group, layer): d_pairs[(gi*K + l)*64 + p], p < d_npairs[gi*K+l]
+  pq::GivensPair* d_pairs;
+  int* d_npairs;
+  int max_pairs;            // max over (group, layer) of the pair count
+  float* d_scale_act;       // [D] exp(-beta) or nullptr
+  float* d_scale_w;         // [D] exp(+beta) or nullptr
+  unsigned int* d_status;   // device status word (PQ_DEV_* bits)
+};
+
+namespace pq {
+
+// Thread-local last-error text.
+void set_error(const char* fmt, ...);
+void clear_error();
+
+// Returns PQ_ERR_CUDA (with the message recorded) when err != cudaSuccess.
+pq_status cuda_fail(cudaError_t err, const char* what);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Kernel launchers (transform.cu, gemm.cu).  Arguments are already validated.
+// y = ((x * pre) H) * post per row-group (pre/post per channel, either may be null).
+cudaError_t launch_hadamard_rows(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx,
+                                 const float* pre_scale, const float* post_scale,
+                                 uint8_t* codes, float* scales, cudaStream_t stream);
+cudaError_t launch_smooth_hadamard(const pq_plan* plan, const void* X, int64_t T, int64_t ldx,
+                                   uint8_t* codes, float* scales, float* smooth_out,
+                                   cudaStream_t stream);
+cudaError_t launch_givens(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx,
+                          const float* post_scale, uint8_t* codes, float* scales,
+                          cudaStream_t stream);
+pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
+                   const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
+                   pq_out_dtype out_dtype, cudaStream_t stream);
+pq_status gemm_read_and_clear_status(unsigned int* bits);
+
+}  // namespace pq

@@ -1,0 +1,375 @@
+// Host side of libpq: argument validation, greedy pair selection, plan tables, status.
+#include <cmath>
+#include <cstdarg>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "internal.h"
+
+namespace pq {
+
+static thread_local char g_last_error[512] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+}
+
+void clear_error() { g_last_error[0] = '\0'; }
+
+pq_status cuda_fail(cudaError_t err, const char* what) {
+  if (err == cudaSuccess) return PQ_OK;
+  set_error("%s: %s (%s)", what, cudaGetErrorString(err), cudaGetErrorName(err));
+  return PQ_ERR_CUDA;
+}
+
+// SplitMix64 (Steele, Lea & Flood, OOPSLA 2014), from its published definition.
+struct SplitMix64 {
+  uint64_t state;
+  explicit SplitMix64(uint64_t seed) : state(seed) {}
+  uint64_t next() {
+    state += 0x9E3779B97F4A7C15ull;
+    uint64_t z = state;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+  }
+};
+
+}  // namespace pq
+
+using namespace pq;
+
+extern "C" const char* pq_status_string(pq_status s) {
+  switch (s) {
+    case PQ_OK: return "PQ_OK";
+    case PQ_ERR_INVALID_ARG: return "PQ_ERR_INVALID_ARG";
+    case PQ_ERR_UNSUPPORTED: return "PQ_ERR_UNSUPPORTED";
+    case PQ_ERR_CUDA: return "PQ_ERR_CUDA";
+    case PQ_ERR_ALLOC: return "PQ_ERR_ALLOC";
+    case PQ_ERR_TIMEOUT: return "PQ_ERR_TIMEOUT";
+  }
+  return "PQ_ERR_UNKNOWN";
+}
+
+extern "C" const char* pq_last_error(void) { return g_last_error; }
+
+// ParoQuant page §2.2, Algorithm A1, per group (see pq.h for the exact shuffle).
+extern "C" pq_status pq_select_pairs(uint64_t seed, int D, int g, int K, int N,
+                                     uint8_t* pairs_out) {
+  clear_error();
+  if (!pairs_out) { set_error("pairs_out is NULL"); return PQ_ERR_INVALID_ARG; }
+  if (g != kGroup) { set_error("g=%d: only g=128 is supported", g); return PQ_ERR_UNSUPPORTED; }
+  if (D < g || D % g != 0) { set_error("D=%d must be a positive multiple of g", D); return PQ_ERR_INVALID_ARG; }
+  if (K < 1 || K > 64) { set_error("K=%d out of range 1..64", K); return PQ_ERR_INVALID_ARG; }
+  if (N < 1 || N > g / 2) { set_error("N=%d out of range 1..g/2", N); return PQ_ERR_INVALID_ARG; }
+  const int G = D / g, half = g / 2;
+  std::vector<uint16_t> cand;           // i << 8 | j
+  cand.reserve(g * (g - 1) / 2);
+  std::vector<uint8_t> avail(g * g), local(g * g);
+  SplitMix64 rng(seed);
+  std::memset(pairs_out, PQ_NO_PAIR, (size_t)G * K * half * 2);
+  for (int gi = 0; gi < G; ++gi) {
+    cand.clear();
+    for (int i = 0; i < g; ++i)
+      for (int j = i + 1; j < g; ++j) cand.push_back((uint16_t)(i << 8 | j));
+    for (size_t i = cand.size() - 1; i >= 1; --i) {
+      size_t k = (size_t)(rng.next() % (uint64_t)(i + 1));
+      uint16_t t = cand[i]; cand[i] = cand[k]; cand[k] = t;
+    }
+    for (int i = 0; i < g; ++i)
+      for (int j = 0; j < g; ++j) avail[i * g + j] = (i != j);
+    for (int l = 0; l < K; ++l) {
+      local = avail;
+      int n = 0;
+      uint8_t* dst = pairs_out + ((size_t)(gi * K + l) * half) * 2;
+      for (uint16_t c : cand) {
+        if (n >= N) break;
+        int i = c >> 8, j = c & 0xFF;
+        if (!local[i * g + j]) continue;
+        dst[2 * n] = (uint8_t)i;
+        dst[2 * n + 1] = (uint8_t)j;
+        ++n;
+        for (int k = 0; k < g; ++k) {
+          local[i * g + k] = local[k * g + i] = 0;
+          local[j * g + k] = local[k * g + j] = 0;
+        }
+        avail[i * g + j] = avail[j * g + i] = 0;
+      }
+    }
+  }
+  return PQ_OK;
+}
+
+static void free_plan_tables(pq_plan* p) {
+  if (!p) return;
+  if (p->d_pairs) cudaFree(p->d_pairs);
+  if (p->d_npairs) cudaFree(p->d_npairs);
+  if (p->d_scale_act) cudaFree(p->d_scale_act);
+  if (p->d_scale_w) cudaFree(p->d_scale_w);
+  if (p->d_status) cudaFree(p->d_status);
+}
+
+template <class T>
+static pq_status upload(T** dst, const T* src, size_t n, const char* what) {
+  cudaError_t e = cudaMalloc((void**)dst, n * sizeof(T));
+  if (e != cudaSuccess) {
+    *dst = nullptr;
+    set_error("cudaMalloc(%s, %zu bytes): %s", what, n * sizeof(T), cudaGetErrorString(e));
+    return PQ_ERR_ALLOC;
+  }
+  if (src) {
+    e = cudaMemcpy(*dst, src, n * sizeof(T), cudaMemcpyHostToDevice);
+  } else {
+    e = cudaMemset(*dst, 0, n * sizeof(T));
+  }
+  return cuda_fail(e, what);
+}
+
+extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int K,
+                                  const uint8_t* pairs, const float* angles, const float* beta,
+                                  uint32_t flags) {
+  clear_error();
+  if (!out) { set_error("out is NULL"); return PQ_ERR_INVALID_ARG; }
+  if (kind != PQ_HADAMARD && kind != PQ_GIVENS && kind != PQ_SMOOTH_HADAMARD) {
+    set_error("unknown kind %d", (int)kind);
+    return PQ_ERR_INVALID_ARG;
+  }
+  if (g != kGroup) { set_error("g=%d: only g=128 is supported", g); return PQ_ERR_UNSUPPORTED; }
+  if (D < g || D % g != 0) { set_error("D=%d must be a positive multiple of 128", D); return PQ_ERR_INVALID_ARG; }
+  if (flags & ~PQ_FLAG_SMOOTH_AFTER_ROTATE) { set_error("unknown flags 0x%x", flags); return PQ_ERR_INVALID_ARG; }
+  if ((flags & PQ_FLAG_SMOOTH_AFTER_ROTATE) && kind != PQ_SMOOTH_HADAMARD) {
+    set_error("PQ_FLAG_SMOOTH_AFTER_ROTATE needs PQ_SMOOTH_HADAMARD");
+    return PQ_ERR_INVALID_ARG;
+  }
+  const int G = D / g, half = g / 2;
+  std::vector<GivensPair> table;
+  std::vector<int> npairs;
+  int max_pairs = 0;
+  if (kind == PQ_GIVENS) {
+    if (K < 1 || K > 64) { set_error("K=%d out of range 1..64", K); return PQ_ERR_INVALID_ARG; }
+    if (!pairs || !angles) { set_error("Givens plan needs pairs and angles"); return PQ_ERR_INVALID_ARG; }
+    table.assign((size_t)G * K * half, GivensPair{0, 1.0f, 0.0f, 0});
+    npairs.assign((size_t)G * K, 0);
+    std::vector<uint8_t> seen(g);
+    for (int gi = 0; gi < G; ++gi) {
+      for (int l = 0; l < K; ++l) {
+        std::fill(seen.begin(), seen.end(), 0);
+        int n = 0;
+        for (int p = 0; p < half; ++p) {
+          size_t slot = (size_t)(gi * K + l) * half + p;
+          uint8_t i = pairs[2 * slot], j = pairs[2 * slot + 1];
+          if (i == PQ_NO_PAIR || j == PQ_NO_PAIR) continue;
+          if (!(i < j && j < g)) {
+            set_error("group %d layer %d slot %d: pair (%d,%d) must satisfy i<j<%d", gi, l, p, i, j, g);
+            return PQ_ERR_INVALID_ARG;
+          }
+          if (seen[i] || seen[j]) {
+            set_error("group %d layer %d: channel used twice (pairs must be disjoint)", gi, l);
+            return PQ_ERR_INVALID_ARG;
+          }
+          seen[i] = seen[j] = 1;
+          double th = (double)angles[slot];
+          if (!std::isfinite(th)) { set_error("non-finite angle at slot %zu", slot); return PQ_ERR_INVALID_ARG; }
+          GivensPair& e = table[(size_t)(gi * K + l) * half + n];
+          e.ij = (uint32_t)i | ((uint32_t)j << 16);
+          e.c = (float)std::cos(th);
+          e.s = (float)std::sin(th);
+          e.pad = 0;
+          ++n;
+        }
+        npairs[(size_t)gi * K + l] = n;
+        if (n > max_pairs) max_pairs = n;
+      }
+    }
+  } else {
+    K = 0;
+  }
+  std::vector<float> sa, sw;
+  if (kind == PQ_GIVENS && beta) {
+    sa.resize(D);
+    sw.resize(D);
+    for (int c = 0; c < D; ++c) {
+      double b = (double)beta[c];
+      if (!std::isfinite(b)) { set_error("non-finite beta[%d]", c); return PQ_ERR_INVALID_ARG; }
+      sa[c] = (float)std::exp(-b);
+      sw[c] = (float)std::exp(b);
+    }
+  }
+  pq_plan* p = new (std::nothrow) pq_plan();
+  if (!p) { set_error("host allocation failed"); return PQ_ERR_ALLOC; }
+  *p = pq_plan{};
+  p->kind = kind;
+  p->D = D;
+  p->g = g;
+  p->G = G;
+  p->K = K;
+  p->flags = flags;
+  p->max_pairs = max_pairs;
+  pq_status st = cuda_fail(cudaGetDevice(&p->device), "cudaGetDevice");
+  if (st == PQ_OK && kind == PQ_GIVENS) {
+    st = upload(&p->d_pairs, table.data(), table.size(), "givens pair table");
+    if (st == PQ_OK) st = upload(&p->d_npairs, npairs.data(), npairs.size(), "givens pair counts");
+  }
+  if (st == PQ_OK && !sa.empty()) {
+    st = upload(&p->d_scale_act, sa.data(), sa.size(), "exp(-beta)");
+    if (st == PQ_OK) st = upload(&p->d_scale_w, sw.data(), sw.size(), "exp(+beta)");
+  }
+  if (st == PQ_OK) st = upload<unsigned int>(&p->d_status, nullptr, 1, "status word");
+  if (st != PQ_OK) {
+    free_plan_tables(p);
+    delete p;
+    return st;
+  }
+  *out = p;
+  return PQ_OK;
+}
+
+extern "C" void pq_destroy_plan(pq_plan* plan) {
+  if (!plan) return;
+  free_plan_tables(plan);
+  delete plan;
+}
+
+static pq_status check_plan(const pq_plan* plan) {
+  if (!plan) { set_error("plan is NULL"); return PQ_ERR_INVALID_ARG; }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != plan->device) {
+    set_error("plan was created on device %d, current device is %d", plan->device, dev);
+    return PQ_ERR_INVALID_ARG;
+  }
+  return PQ_OK;
+}
+
+extern "C" pq_status pq_transform_quant(const pq_plan* plan, const void* X, int64_t T,
+                                        int64_t ldx, uint8_t* codes, float* scales,
+                                        float* smooth_out, void* stream) {
+  clear_error();
+  if (!plan) { set_error("plan is NULL"); return PQ_ERR_INVALID_ARG; }
+  if (!X || !codes || !scales) { set_error("X, codes and scales must be non-NULL"); return PQ_ERR_INVALID_ARG; }
+  if (T < 1) { set_error("T=%lld must be >= 1", (long long)T); return PQ_ERR_INVALID_ARG; }
+  if (ldx < plan->D || ldx % 8 != 0) {
+    set_error("ldx=%lld must be >= D=%d and a multiple of 8", (long long)ldx, plan->D);
+    return PQ_ERR_INVALID_ARG;
+  }
+  if (!aligned16(X) || !aligned16(codes) || !aligned16(scales) ||
+      (smooth_out && !aligned16(smooth_out))) {
+    set_error("device pointers must be 16-byte aligned");
+    return PQ_ERR_INVALID_ARG;
+  }
+  if (smooth_out && plan->kind != PQ_SMOOTH_HADAMARD) {
+    set_error("smooth_out must be NULL for this plan kind");
+    return PQ_ERR_INVALID_ARG;
+  }
+  if (T >= ((int64_t)1 << 31)) { set_error("T=%lld must be < 2^31", (long long)T); return PQ_ERR_INVALID_ARG; }
+  pq_status st = check_plan(plan);
+  if (st != PQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  switch (plan->kind) {
+    case PQ_HADAMARD:
+      e = launch_hadamard_rows(plan, X, T, ldx, nullptr, nullptr, codes, scales, s);
+      break;
+    case PQ_GIVENS:
+      e = launch_givens(plan, X, T, ldx, plan->d_scale_act, codes, scales, s);
+      break;
+    case PQ_SMOOTH_HADAMARD:
+      e = launch_smooth_hadamard(plan, X, T, ldx, codes, scales, smooth_out, s);
+      break;
+  }
+  return cuda_fail(e, "pq_transform_quant launch");
+}
+
+extern "C" pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t N,
+                                     const float* smooth_w, uint8_t* codes_W, float* scales_W,
+                                     void* stream) {
+  clear_error();
+  if (!plan) { set_error("plan is NULL"); return PQ_ERR_INVALID_ARG; }
+  if (!W || !codes_W || !scales_W) { set_error("W, codes_W and scales_W must be non-NULL"); return PQ_ERR_INVALID_ARG; }
+  if (N < 1 || N >= ((int64_t)1 << 31)) { set_error("N=%lld must be in [1, 2^31)", (long long)N); return PQ_ERR_INVALID_ARG; }
+  if (!aligned16(W) || !aligned16(codes_W) || !aligned16(scales_W) ||
+      (smooth_w && !aligned16(smooth_w))) {
+    set_error("device pointers must be 16-byte aligned");
+    return PQ_ERR_INVALID_ARG;
+  }
+  if (smooth_w && plan->kind != PQ_SMOOTH_HADAMARD) {
+    set_error("smooth_w must be NULL for this plan kind");
+    return PQ_ERR_INVALID_ARG;
+  }
+  pq_status st = check_plan(plan);
+  if (st != PQ_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  switch (plan->kind) {
+    case PQ_HADAMARD:
+      e = launch_hadamard_rows(plan, W, N, plan->D, nullptr, nullptr, codes_W, scales_W, s);
+      break;
+    case PQ_GIVENS:
+      e = launch_givens(plan, W, N, plan->D, plan->d_scale_w, codes_W, scales_W, s);
+      break;
+    case PQ_SMOOTH_HADAMARD:
+      if (plan->flags & PQ_FLAG_SMOOTH_AFTER_ROTATE)
+        e = launch_hadamard_rows(plan, W, N, plan->D, nullptr, smooth_w, codes_W, scales_W, s);
+      else
+        e = launch_hadamard_rows(plan, W, N, plan->D, smooth_w, nullptr, codes_W, scales_W, s);
+      break;
+  }
+  return cuda_fail(e, "pq_pack_weights launch");
+}
+
+extern "C" pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A,
+                                  const uint8_t* codes_W, const float* scales_W, int64_t T,
+                                  int64_t N, int64_t D, int g, void* Y, pq_out_dtype out_dtype,
+                                  void* stream) {
+  clear_error();
+  if (!codes_A || !scales_A || !codes_W || !scales_W || !Y) {
+    set_error("all tensor pointers must be non-NULL");
+    return PQ_ERR_INVALID_ARG;
+  }
+  if (g != kGroup) { set_error("g=%d: only g=128 is supported", g); return PQ_ERR_UNSUPPORTED; }
+  if (T < 1 || N < 1 || D < g) { set_error("T, N must be >= 1 and D >= 128"); return PQ_ERR_INVALID_ARG; }
+  if (D % g != 0) { set_error("D=%lld must be a multiple of 128", (long long)D); return PQ_ERR_INVALID_ARG; }
+  if (N % 16 != 0) { set_error("N=%lld must be a multiple of 16", (long long)N); return PQ_ERR_INVALID_ARG; }
+  if (out_dtype != PQ_OUT_F32 && out_dtype != PQ_OUT_BF16) { set_error("bad out_dtype"); return PQ_ERR_INVALID_ARG; }
+  if (T >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || D >= ((int64_t)1 << 24)) {
+    set_error("T, N must be < 2^31 and D < 2^24");
+    return PQ_ERR_INVALID_ARG;
+  }
+  if (!aligned16(codes_A) || !aligned16(scales_A) || !aligned16(codes_W) ||
+      !aligned16(scales_W) || !aligned16(Y)) {
+    set_error("device pointers must be 16-byte aligned");
+    return PQ_ERR_INVALID_ARG;
+  }
+  return gemm_run(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" pq_status pq_check_status(const pq_plan* plan, void* stream) {
+  clear_error();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  pq_status st = cuda_fail(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+  if (st != PQ_OK) return st;
+  unsigned int bits = 0;
+  if (plan && plan->d_status) {
+    unsigned int pb = 0;
+    st = cuda_fail(cudaMemcpy(&pb, plan->d_status, sizeof(pb), cudaMemcpyDeviceToHost), "read plan status");
+    if (st != PQ_OK) return st;
+    if (pb) {
+      st = cuda_fail(cudaMemset(plan->d_status, 0, sizeof(pb)), "clear plan status");
+      if (st != PQ_OK) return st;
+    }
+    bits |= pb;
+  }
+  unsigned int gb = 0;
+  st = gemm_read_and_clear_status(&gb);
+  if (st != PQ_OK) return st;
+  bits |= gb;
+  if (bits & PQ_DEV_TIMEOUT) {
+    set_error("a device-side bounded wait timed out (status bits 0x%x)", bits);
+    return PQ_ERR_TIMEOUT;
+  }
+  return PQ_OK;
+}

@@ -1,0 +1,402 @@
+// Fused rotate / scale / smooth + per-group INT4 quantisation kernels (sm_100a).
+//
+// ParoQuant page §3.2: rotation, scaling and quantisation are one kernel, so each element is
+// read once from HBM (bf16, 2 B) and written once (a nibble), plus one float scale per group.
+//
+// Block Hadamard (Hadamard page §2.1/§4.2/§6.1, RRS page R = (1/sqrt(K))[s_ij]): a 128-channel
+// group is held by 4 lanes, 32 consecutive channels each (four 16-byte loads per lane).  H_128
+// = H_4 (x) H_32 in Sylvester order: channel bits 0..4 are transformed in registers (5 radix-2
+// stages), bits 5..6 across the 4 lanes with two xor-shuffle stages.  The 1/sqrt(128) factor
+// never touches the data: the codes do not depend on a uniform factor, so it is folded into the
+// stored scale.
+//
+// Quantisation (RRS page: alpha = max|X| / 7, codes in -8..7, RTN): m = max|y| over the group
+// (two xor-shuffles), inv = 7/m, q = RNE(y * inv) by one FMA with 1.5 * 2^23, whose low 4 bits
+// are already the two's-complement nibble; nibbles are packed with byte permutes.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+
+namespace pq {
+namespace {
+
+constexpr float kRoundMagic = 12582912.0f;                   // 1.5 * 2^23
+constexpr float kInvSqrt128 = 0.088388347648318440550f;     // 1/sqrt(128), float-rounded
+constexpr float kScaleHadamard = 0.012626906806902634f;     // 1/(7*sqrt(128)), float-rounded
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+  uint4 r;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float* v) {
+  v[0] = __uint_as_float(w.x << 16);
+  v[1] = __uint_as_float(w.x & 0xFFFF0000u);
+  v[2] = __uint_as_float(w.y << 16);
+  v[3] = __uint_as_float(w.y & 0xFFFF0000u);
+  v[4] = __uint_as_float(w.z << 16);
+  v[5] = __uint_as_float(w.z & 0xFFFF0000u);
+  v[6] = __uint_as_float(w.w << 16);
+  v[7] = __uint_as_float(w.w & 0xFFFF0000u);
+}
+
+// Unnormalised Walsh-Hadamard transform of 32 register values (Sylvester order).
+__device__ __forceinline__ void fwht32(float (&v)[32]) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+    }
+  }
+}
+
+// The two remaining radix-2 stages across the 4 lanes (lane bits 0,1 = channel bits 5,6):
+// the lane holding the low half keeps a + b, the other keeps a - b.
+__device__ __forceinline__ void fwht_across4(float (&v)[32], int lane) {
+  const float s1 = (lane & 1) ? -1.0f : 1.0f;
+  const float s2 = (lane & 2) ? -1.0f : 1.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = fmaf(s1, v[i], __shfl_xor_sync(0xffffffffu, v[i], 1));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = fmaf(s2, v[i], __shfl_xor_sync(0xffffffffu, v[i], 2));
+}
+
+__device__ __forceinline__ float absmax32(const float (&v)[32]) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
+  return m;
+}
+
+__device__ __forceinline__ float group_max4(float m) {
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+  return m;
+}
+
+__device__ __forceinline__ float quant_inv(float m) { return m > 0.0f ? __fdiv_rn(7.0f, m) : 0.0f; }
+
+// 8 values -> 8 nibbles in one word: byte k = q[2k] | q[2k+1] << 4.
+__device__ __forceinline__ uint32_t quant_pack8(const float* v, float inv) {
+  uint32_t b[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) b[k] = __float_as_uint(fmaf(v[k], inv, kRoundMagic));
+  const uint32_t even = __byte_perm(__byte_perm(b[0], b[2], 0x0040), __byte_perm(b[4], b[6], 0x0040), 0x5410);
+  const uint32_t odd = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
+  return (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
+}
+
+__device__ __forceinline__ uint4 quant_pack32(const float (&v)[32], float inv) {
+  return make_uint4(quant_pack8(v, inv), quant_pack8(v + 8, inv), quant_pack8(v + 16, inv),
+                    quant_pack8(v + 24, inv));
+}
+
+__device__ __forceinline__ void load32(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* p = reinterpret_cast<const uint4*>(src);
+  const uint4 w0 = ld_stream(p), w1 = ld_stream(p + 1), w2 = ld_stream(p + 2), w3 = ld_stream(p + 3);
+  bf16x8_to_f32(w0, v);
+  bf16x8_to_f32(w1, v + 8);
+  bf16x8_to_f32(w2, v + 16);
+  bf16x8_to_f32(w3, v + 24);
+}
+
+__device__ __forceinline__ void scale32(float (&v)[32], const float* s) {
+  const float4* p = reinterpret_cast<const float4*>(s);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float4 f = __ldg(p + k);
+    v[4 * k] *= f.x;
+    v[4 * k + 1] *= f.y;
+    v[4 * k + 2] *= f.z;
+    v[4 * k + 3] *= f.w;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Flat stream of row-groups (row t, group gi), 8 per warp.  y = ((x * pre) H) * post.
+__global__ void __launch_bounds__(256) hadamard_rows_kernel(
+    const __nv_bfloat16* __restrict__ X, int64_t rows, int64_t ldx, int G,
+    const float* __restrict__ pre, const float* __restrict__ post, uint8_t* __restrict__ codes,
+    float* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int q = lane & 3;
+  const int64_t R = rows * (int64_t)G;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t halfD = (int64_t)G * 64;
+  for (int64_t base = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 8; base < R;
+       base += nwarps * 8) {
+    const int64_t r = base + (lane >> 2);
+    const bool valid = r < R;
+    const int64_t t = valid ? r / G : 0;
+    const int gi = valid ? (int)(r - t * G) : 0;
+    const int c0 = gi * 128 + q * 32;
+    float v[32];
+    if (valid) {
+      load32(X + t * ldx + c0, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+    }
+    if (pre) scale32(v, pre + c0);
+    fwht32(v);
+    fwht_across4(v, lane);
+    if (post) scale32(v, post + c0);
+    const float m = group_max4(absmax32(v));
+    const uint4 packed = quant_pack32(v, quant_inv(m));
+    if (valid) {
+      *reinterpret_cast<uint4*>(codes + t * halfD + gi * 64 + q * 16) = packed;
+      if (q == 0) scales[r] = m * kScaleHadamard;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Runtime smoothing + Hadamard on a 128-row x 128-channel tile (one CTA, 4 warps).  Lane
+// (warp w, slot = lane/4, q = lane%4) holds rows 32k + 8w + slot (k = 0..3), channels 32q..+31.
+// after_rotate = false: s = max|x| per channel over the tile's rows, y = (x / s) H.
+// after_rotate = true:  s = max|x H| per channel (rotated channels), y = (x H) / s.
+__global__ void __launch_bounds__(128) smooth_hadamard_kernel(
+    const __nv_bfloat16* __restrict__ X, int64_t T, int64_t ldx, int G, int after_rotate,
+    uint8_t* __restrict__ codes, float* __restrict__ scales, float* __restrict__ smooth_out) {
+  __shared__ __align__(16) float red[4][4][32];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, q = lane & 3, slot = lane >> 2;
+  const int64_t b = blockIdx.x;
+  const int gi = blockIdx.y;
+  const int c0 = gi * 128 + q * 32;
+  const int64_t D = (int64_t)G * 128;
+
+  uint4 x[4][4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int64_t t = b * 128 + 32 * k + 8 * w + slot;
+    if (t < T) {
+      const uint4* p = reinterpret_cast<const uint4*>(X + t * ldx + c0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) x[k][j] = ld_stream(p + j);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) x[k][j] = make_uint4(0, 0, 0, 0);
+    }
+  }
+
+  // Per-channel maximum over the tile -> s (32 channels per lane).
+  float s[32];
+  if (!after_rotate) {
+    // |bf16| compared as unsigned 16-bit integers (sign bit cleared): exact, no conversion.
+    uint32_t mw[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) mw[j] = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t* xw = reinterpret_cast<const uint32_t*>(&x[k][0]);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) mw[j] = __vmaxu2(mw[j], xw[j] & 0x7FFF7FFFu);
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      mw[j] = __vmaxu2(mw[j], __shfl_xor_sync(0xffffffffu, mw[j], 4));
+      mw[j] = __vmaxu2(mw[j], __shfl_xor_sync(0xffffffffu, mw[j], 8));
+      mw[j] = __vmaxu2(mw[j], __shfl_xor_sync(0xffffffffu, mw[j], 16));
+    }
+    if (slot == 0) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        red[w][q][2 * j] = __uint_as_float(mw[j] << 16);
+        red[w][q][2 * j + 1] = __uint_as_float(mw[j] & 0xFFFF0000u);
+      }
+    }
+  } else {
+    float cm[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) cm[i] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bf16x8_to_f32(x[k][j], v + 8 * j);
+      fwht32(v);
+      fwht_across4(v, lane);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) cm[i] = fmaxf(cm[i], fabsf(v[i]));
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      cm[i] = fmaxf(cm[i], __shfl_xor_sync(0xffffffffu, cm[i], 4));
+      cm[i] = fmaxf(cm[i], __shfl_xor_sync(0xffffffffu, cm[i], 8));
+      cm[i] = fmaxf(cm[i], __shfl_xor_sync(0xffffffffu, cm[i], 16));
+    }
+    if (slot == 0) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) red[w][q][i] = cm[i];
+    }
+  }
+  __syncthreads();
+  float rs[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float m = fmaxf(fmaxf(red[0][q][i], red[1][q][i]), fmaxf(red[2][q][i], red[3][q][i]));
+    // Reported s is for the normalised rotation; the kernel divides unnormalised values by the
+    // unnormalised maximum, which gives the same quotient.
+    s[i] = m > 0.0f ? (after_rotate ? m * kInvSqrt128 : m) : 1.0f;
+    rs[i] = m > 0.0f ? __frcp_rn(m) : 0.0f;
+  }
+  if (smooth_out && w == 0 && slot == 0) {
+    float4* dst = reinterpret_cast<float4*>(smooth_out + b * D + c0);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dst[j] = make_float4(s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3]);
+  }
+
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int64_t t = b * 128 + 32 * k + 8 * w + slot;
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bf16x8_to_f32(x[k][j], v + 8 * j);
+    if (!after_rotate) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= rs[i];
+    }
+    fwht32(v);
+    fwht_across4(v, lane);
+    if (after_rotate) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= rs[i];
+    }
+    const float m = group_max4(absmax32(v));
+    const uint4 packed = quant_pack32(v, quant_inv(m));
+    if (t < T) {
+      *reinterpret_cast<uint4*>(codes + t * (D / 2) + gi * 64 + q * 16) = packed;
+      // before the rotation the values are x/s (normalised range), after it (x H)/s_unnorm.
+      if (q == 0) scales[t * G + gi] = after_rotate ? __fdiv_rn(m, 7.0f) : m * kScaleHadamard;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Givens layers (ParoQuant page §2.2): one lane per row, the row's 128 channels of group gi
+// staged in shared memory as [channel][lane] (stride 33: conflict-free), the layer's pairs
+// read as warp-uniform broadcasts.  Then y *= post per channel, quantise, pack.
+constexpr int kGivensRows = 128;   // rows per CTA (4 warps x 32 lanes)
+
+__global__ void __launch_bounds__(128) givens_kernel(
+    const __nv_bfloat16* __restrict__ X, int64_t rows, int64_t ldx, int G, int K,
+    const GivensPair* __restrict__ pairs, const int* __restrict__ npairs,
+    const float* __restrict__ post, uint8_t* __restrict__ codes, float* __restrict__ scales) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  GivensPair* tbl = reinterpret_cast<GivensPair*>(smem_raw);
+  int* np = reinterpret_cast<int*>(tbl + K * 64);
+  float* tile = reinterpret_cast<float*>(np + ((K + 3) & ~3));
+  const int gi = blockIdx.y;
+  for (int i = threadIdx.x; i < K * 64; i += blockDim.x) tbl[i] = pairs[(size_t)gi * K * 64 + i];
+  for (int i = threadIdx.x; i < K; i += blockDim.x) np[i] = npairs[gi * K + i];
+  __syncthreads();
+
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* col = tile + w * (128 * 33) + lane;
+  const int64_t t = (int64_t)blockIdx.x * kGivensRows + w * 32 + lane;
+  if (t >= rows) return;
+  const uint4* src = reinterpret_cast<const uint4*>(X + t * ldx + gi * 128);
+#pragma unroll 4
+  for (int c16 = 0; c16 < 16; ++c16) {
+    float v[8];
+    bf16x8_to_f32(ld_stream(src + c16), v);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) col[(8 * c16 + k) * 33] = v[k];
+  }
+  for (int l = 0; l < K; ++l) {
+    const int n = np[l];
+    const GivensPair* e = tbl + l * 64;
+    for (int p = 0; p < n; ++p) {
+      const GivensPair pe = e[p];
+      const int i = pe.ij & 0xFFFF, j = pe.ij >> 16;
+      const float xi = col[i * 33], xj = col[j * 33];
+      col[i * 33] = fmaf(pe.c, xi, -pe.s * xj);
+      col[j * 33] = fmaf(pe.s, xi, pe.c * xj);
+    }
+  }
+  float m = 0.0f;
+  const float* ps = post ? post + gi * 128 : nullptr;
+  for (int c = 0; c < 128; ++c) {
+    float v = col[c * 33];
+    if (ps) {
+      v *= __ldg(ps + c);
+      col[c * 33] = v;
+    }
+    m = fmaxf(m, fabsf(v));
+  }
+  const float inv = quant_inv(m);
+  uint32_t words[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = col[(8 * k + j) * 33];
+    words[k] = quant_pack8(v, inv);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(codes + t * (int64_t)G * 64 + gi * 64);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) dst[k] = make_uint4(words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]);
+  scales[t * G + gi] = __fdiv_rn(m, 7.0f);
+}
+
+int sm_count() {
+  static int count[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!count[dev]) {
+    int c = 0;
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
+    count[dev] = c;
+  }
+  return count[dev];
+}
+
+}  // namespace
+
+cudaError_t launch_hadamard_rows(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx,
+                                 const float* pre_scale, const float* post_scale, uint8_t* codes,
+                                 float* scales, cudaStream_t stream) {
+  const int64_t R = rows * plan->G;
+  const int64_t tasks = (R + 7) / 8;                // one warp-iteration = 8 row-groups
+  const int64_t want = (tasks + 7) / 8;             // 8 warps per block
+  const int64_t cap = (int64_t)sm_count() * 6;      // a few resident blocks per SM, grid-stride
+  const int grid = (int)(want < cap ? want : cap);
+  hadamard_rows_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(X), rows,
+                                                 ldx, plan->G, pre_scale, post_scale, codes, scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_smooth_hadamard(const pq_plan* plan, const void* X, int64_t T, int64_t ldx,
+                                   uint8_t* codes, float* scales, float* smooth_out,
+                                   cudaStream_t stream) {
+  dim3 grid((unsigned)((T + kSmoothBlock - 1) / kSmoothBlock), (unsigned)plan->G);
+  smooth_hadamard_kernel<<<grid, 128, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(X), T, ldx, plan->G,
+      (plan->flags & PQ_FLAG_SMOOTH_AFTER_ROTATE) ? 1 : 0, codes, scales, smooth_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_givens(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx,
+                          const float* post_scale, uint8_t* codes, float* scales,
+                          cudaStream_t stream) {
+  const size_t smem = (size_t)plan->K * 64 * sizeof(GivensPair) + ((plan->K + 3) & ~3) * sizeof(int) +
+                      (size_t)4 * 128 * 33 * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(givens_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((rows + kGivensRows - 1) / kGivensRows), (unsigned)plan->G);
+  givens_kernel<<<grid, 128, smem, stream>>>(reinterpret_cast<const __nv_bfloat16*>(X), rows, ldx,
+                                             plan->G, plan->K, plan->d_pairs, plan->d_npairs,
+                                             post_scale, codes, scales);
+  return cudaGetLastError();
+}
+
+}  // namespace pq

@@ -1,0 +1,170 @@
+"""ctypes binding for libpq (``include/pq.h``): the same entry points, argument marshalling only.
+
+Tensors are passed as device pointers (``torch.Tensor.data_ptr()``) with the current CUDA
+stream unless one is given.  Every call checks the returned status and raises ``PQError``
+with the library's message.  Importing this module loads the library and raises if it has
+not been built (``python -m rotation_int4_w4a4_b200.build``): there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libpq.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libpq.so is not built ({_LIB_PATH}); run python -m rotation_int4_w4a4_b200.build")
+lib = ctypes.CDLL(_LIB_PATH)
+
+PQ_OK, PQ_ERR_INVALID_ARG, PQ_ERR_UNSUPPORTED, PQ_ERR_CUDA, PQ_ERR_ALLOC, PQ_ERR_TIMEOUT = range(6)
+PQ_HADAMARD, PQ_GIVENS, PQ_SMOOTH_HADAMARD = range(3)
+PQ_OUT_F32, PQ_OUT_BF16 = range(2)
+PQ_FLAG_SMOOTH_AFTER_ROTATE = 0x1
+PQ_NO_PAIR = 0xFF
+KINDS = {"hadamard": PQ_HADAMARD, "givens": PQ_GIVENS, "smooth_hadamard": PQ_SMOOTH_HADAMARD}
+
+# Every symbol the header declares.
+EXPORTS = ("pq_select_pairs", "pq_make_plan", "pq_destroy_plan", "pq_transform_quant",
+           "pq_pack_weights", "pq_w4a4_gemm", "pq_check_status", "pq_status_string",
+           "pq_last_error")
+
+_c = ctypes
+_vp, _i64, _u64, _i32, _u32 = _c.c_void_p, _c.c_int64, _c.c_uint64, _c.c_int, _c.c_uint32
+lib.pq_select_pairs.argtypes = [_u64, _i32, _i32, _i32, _i32, _vp]
+lib.pq_select_pairs.restype = _i32
+lib.pq_make_plan.argtypes = [_c.POINTER(_vp), _i32, _i32, _i32, _i32, _vp, _vp, _vp, _u32]
+lib.pq_make_plan.restype = _i32
+lib.pq_destroy_plan.argtypes = [_vp]
+lib.pq_destroy_plan.restype = None
+lib.pq_transform_quant.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]
+lib.pq_transform_quant.restype = _i32
+lib.pq_pack_weights.argtypes = [_vp, _vp, _i64, _vp, _vp, _vp, _vp]
+lib.pq_pack_weights.restype = _i32
+lib.pq_w4a4_gemm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _i32, _vp]
+lib.pq_w4a4_gemm.restype = _i32
+lib.pq_check_status.argtypes = [_vp, _vp]
+lib.pq_check_status.restype = _i32
+lib.pq_status_string.argtypes = [_i32]
+lib.pq_status_string.restype = _c.c_char_p
+lib.pq_last_error.argtypes = []
+lib.pq_last_error.restype = _c.c_char_p
+
+
+class PQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.pq_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {lib.pq_status_string(status).decode()}: {msg}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != PQ_OK:
+        raise PQError(status, where)
+
+
+def _ptr(x):
+    """Device pointer of a tensor (or None -> NULL)."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def pq_select_pairs(seed: int, D: int, g: int, K: int, N: int) -> np.ndarray:
+    """Host-side greedy pair selection -> uint8 [D/g, K, g/2, 2] (0xFF = no pair)."""
+    out = np.empty((D // g, K, g // 2, 2), dtype=np.uint8)
+    _check(lib.pq_select_pairs(seed, D, g, K, N, out.ctypes.data), "pq_select_pairs")
+    return out
+
+
+class Plan:
+    """Owns a ``pq_plan`` (device tables); freed by :meth:`close` or garbage collection."""
+
+    def __init__(self, kind, D: int, g: int = 128, K: int = 0, pairs=None, angles=None,
+                 beta=None, flags: int = 0):
+        kind = KINDS.get(kind, kind)
+        self.kind, self.D, self.g, self.K, self.flags = kind, D, g, K, flags
+        keep = []
+
+        def host(a, dt):
+            if a is None:
+                return None
+            a = np.ascontiguousarray(a, dtype=dt)
+            keep.append(a)
+            return a.ctypes.data
+
+        h = _vp()
+        _check(lib.pq_make_plan(_c.byref(h), kind, D, g, K, host(pairs, np.uint8),
+                                host(angles, np.float32), host(beta, np.float32), flags),
+               "pq_make_plan")
+        self._h = h
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib.pq_destroy_plan(self._h)
+            self._h = None
+
+    def __del__(self):  # pragma: no cover - interpreter teardown order
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def pq_make_plan(kind, D, g=128, K=0, pairs=None, angles=None, beta=None, flags=0) -> Plan:
+    return Plan(kind, D, g, K, pairs, angles, beta, flags)
+
+
+def pq_destroy_plan(plan: Plan) -> None:
+    plan.close()
+
+
+def pq_transform_quant(plan: Plan, X, codes, scales, smooth_out=None, T=None, ldx=None,
+                       stream=None) -> None:
+    """X bf16 [T, ldx] -> codes uint8 [T, D/2], scales float32 [T, D/g] (device tensors)."""
+    T = X.shape[0] if T is None else T
+    ldx = X.stride(0) if ldx is None else ldx
+    _check(lib.pq_transform_quant(plan.handle, _ptr(X), T, ldx, _ptr(codes), _ptr(scales),
+                                  _ptr(smooth_out), _stream(stream)), "pq_transform_quant")
+
+
+def pq_pack_weights(plan: Plan, W, codes_W, scales_W, smooth_w=None, N=None, stream=None) -> None:
+    """W bf16 [N, D] -> codes_W uint8 [N, D/2], scales_W float32 [N, D/g] (device tensors)."""
+    N = W.shape[0] if N is None else N
+    _check(lib.pq_pack_weights(plan.handle, _ptr(W), N, _ptr(smooth_w), _ptr(codes_W),
+                               _ptr(scales_W), _stream(stream)), "pq_pack_weights")
+
+
+def pq_w4a4_gemm(codes_A, scales_A, codes_W, scales_W, Y, T=None, N=None, D=None, g=128,
+                 out_dtype=None, stream=None) -> None:
+    """Y [T, N] = per-group scaled int4 x int4 product (device tensors)."""
+    T = codes_A.shape[0] if T is None else T
+    N = codes_W.shape[0] if N is None else N
+    D = codes_A.shape[1] * 2 if D is None else D
+    if out_dtype is None:
+        import torch
+        out_dtype = PQ_OUT_BF16 if Y.dtype == torch.bfloat16 else PQ_OUT_F32
+    _check(lib.pq_w4a4_gemm(_ptr(codes_A), _ptr(scales_A), _ptr(codes_W), _ptr(scales_W),
+                            T, N, D, g, _ptr(Y), out_dtype, _stream(stream)), "pq_w4a4_gemm")
+
+
+def pq_check_status(plan: Plan | None = None, stream=None) -> int:
+    """Synchronise and return the status code (raises PQError on failure)."""
+    st = lib.pq_check_status(plan.handle if plan is not None else None, _stream(stream))
+    _check(st, "pq_check_status")
+    return st

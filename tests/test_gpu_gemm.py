@@ -1,0 +1,107 @@
+"""GPU parity of the tcgen05 W4A4 GEMM against the CPU oracle on identical codes and scales.
+
+Acceptance: per-group integer dots bit-exact (D = 128, unit scales: Y is the dot itself);
+float32 Y within 1e-5 relative Frobenius error of the oracle; bf16 Y within one bf16 ulp of
+the round-to-nearest-even of the oracle's float32 result.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from rotation_int4_w4a4_b200 import inputs
+from tests.helpers import to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pq():
+    from rotation_int4_w4a4_b200 import pq as _pq
+    return _pq
+
+
+def run_gemm(pq, ca, sa, cw, sw, out="f32"):
+    import torch
+    T, N = ca.shape[0], cw.shape[0]
+    Y = torch.empty((T, N), dtype=torch.float32 if out == "f32" else torch.bfloat16, device="cuda")
+    pq.pq_w4a4_gemm(to_dev(ca), to_dev(sa), to_dev(cw), to_dev(sw), Y)
+    pq.pq_check_status()
+    return Y.float().cpu().numpy()
+
+
+def rel_fro(a, b):
+    return float(np.linalg.norm(a.astype(np.float64) - b) / max(np.linalg.norm(b), 1e-300))
+
+
+@pytest.mark.parametrize("T,N", [(1, 256), (128, 256), (130, 512), (257, 768), (64, 16)])
+def test_dots_bit_exact(pq, T, N):
+    """D = 128 (one group) and unit scales: Y[t][n] is the integer dot product itself."""
+    ca, _ = inputs.random_codes(101 + T, T, 128)
+    cw, _ = inputs.random_codes(202 + N, N, 128)
+    ones_a = np.ones((T, 1), np.float32)
+    ones_w = np.ones((N, 1), np.float32)
+    Y = run_gemm(pq, ca, ones_a, cw, ones_w)
+    d = oracle.group_dots(ca, cw, 128)[0]
+    assert np.array_equal(Y, d.astype(np.float32))
+
+
+def test_extreme_codes_bit_exact(pq):
+    # all -8 x all -8 gives the largest dot, 128 * 64 = 8192; mixed signs the most negative.
+    T, N = 128, 256
+    m8 = oracle.pack_nibbles(np.full((T, 128), -8, np.int8))
+    p7 = oracle.pack_nibbles(np.full((N, 128), 7, np.int8))
+    n8 = oracle.pack_nibbles(np.full((N, 128), -8, np.int8))
+    one_a, one_w = np.ones((T, 1), np.float32), np.ones((N, 1), np.float32)
+    assert np.all(run_gemm(pq, m8, one_a, n8, one_w) == 8192.0)
+    assert np.all(run_gemm(pq, m8, one_a, p7, one_w) == -7168.0)
+
+
+@pytest.mark.parametrize("T,N,D", [(3, 16, 256), (200, 272, 384), (128, 256, 1024), (333, 1024, 512)])
+def test_random_codes_f32(pq, T, N, D):
+    ca, sa = inputs.random_codes(7 + T, T, D)
+    cw, sw = inputs.random_codes(9 + N, N, D)
+    Y = run_gemm(pq, ca, sa, cw, sw)
+    ref = oracle.gemm(ca, sa, cw, sw)
+    assert rel_fro(Y, ref.y64) < 1e-5
+    assert rel_fro(Y, ref.y32) < 1e-5
+
+
+def test_random_codes_bf16(pq):
+    T, N, D = 150, 512, 512
+    ca, sa = inputs.random_codes(31, T, D)
+    cw, sw = inputs.random_codes(32, N, D)
+    Y = run_gemm(pq, ca, sa, cw, sw, out="bf16")
+    ref = oracle.bf16_round(oracle.gemm(ca, sa, cw, sw).y32)
+    # one bf16 ulp of the reference value
+    ulp = np.maximum(np.abs(ref), 2.0 ** -126) * 2.0 ** -7
+    assert np.all(np.abs(Y - ref) <= ulp)
+
+
+def test_oracle_codes_end_to_end_tiny(pq):
+    """The tiny Givens workload: the oracle's own activation and weight codes through the GPU GEMM."""
+    wl = inputs.workload("tiny")
+    pairs = oracle.select_pairs(wl.pair_seed, wl.D, wl.g, wl.K, 64)
+    plan = oracle.Plan("givens", wl.D, 128, wl.K, pairs, wl.angles, wl.beta)
+    a = oracle.transform_quant(wl.X, plan)
+    w = oracle.pack_weights(wl.W, plan)
+    Y = run_gemm(pq, a.codes, a.scales, w.codes, w.scales)
+    ref = oracle.gemm(a.codes, a.scales, w.codes, w.scales)
+    assert rel_fro(Y, ref.y64) < 1e-5
+
+
+@pytest.mark.parametrize("name", ["q_proj", "up_proj", "down_proj"])
+def test_full_size_sampled_rows(pq, name):
+    """The full workload shapes in the launch configuration the benchmark uses, checked on a
+    few sampled rows (first, middle, last tile) against the oracle."""
+    import torch
+    wl = inputs.workload(name, with_weights=False)
+    T, N, D = wl.T, wl.N, wl.D
+    ca, sa = inputs.random_codes(1000 + T, T, D)
+    cw, sw = inputs.random_codes(2000 + N, N, D)
+    Y = torch.empty((T, N), dtype=torch.float32, device="cuda")
+    pq.pq_w4a4_gemm(to_dev(ca), to_dev(sa), to_dev(cw), to_dev(sw), Y)
+    pq.pq_check_status()
+    rows = np.array([0, 1, 127, T // 2, T // 2 + 77, T - 1])
+    Ys = Y[torch.from_numpy(rows).cuda()].cpu().numpy()
+    ref = oracle.gemm(ca[rows], sa[rows], cw, sw)
+    assert rel_fro(Ys, ref.y64) < 1e-5

