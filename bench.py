@@ -63,7 +63,7 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: str):
         self.gpu = gpu_index
         self.lines: list[tuple[float, str]] = []
         self.proc = None
@@ -117,7 +117,7 @@ class ClockSampler:
 
 
 # -------------------------------------------------------------------- CPU oracle
-def oracle_sample(wl, x_rows=8, w_rows=128):
+def oracle_sample(wl, x_rows=128, w_rows=1024):
     """Time the oracle on a bounded sample and extrapolate to one full step (seconds)."""
     import numpy as np
     from threadpoolctl import threadpool_limits
@@ -224,8 +224,8 @@ def run_ours(args, wl, rank, world, local_rank):
     torch.cuda.synchronize()
     pq.pq_check_status(plan)
 
-    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[0])
-                          if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local_rank)
+    vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    clocks = ClockSampler(vis[local_rank] if local_rank < len(vis) else str(local_rank))
     clocks.start()
     t_roll = time.time()
     while time.time() - t_roll < 0.6:            # keep the GPU busy while sampling starts
