@@ -69,6 +69,13 @@ cudaError_t launch_givens(const pq_plan* plan, const void* X, int64_t rows, int6
 pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                    const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
                    pq_out_dtype out_dtype, cudaStream_t stream);
+// Bytes of int8 operand scratch the GEMM needs: (T + N) * D.
+size_t gemm_scratch_bytes(int64_t T, int64_t N, int64_t D);
+// Expansion + contraction launches on `stream` using caller-provided scratch.
+pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
+                      const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
+                      pq_out_dtype out_dtype, uint8_t* scratch, unsigned int* status,
+                      cudaStream_t stream);
 pq_status gemm_read_and_clear_status(unsigned int* bits);
 
 }  // namespace pq

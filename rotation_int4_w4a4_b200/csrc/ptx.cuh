@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads, tcgen05 (TMEM, UMMA).
-// Every wait is bounded (see BoundedWait); nothing here traps.
+// Every wait is bounded (mbar_wait_bounded); nothing here traps.
 #pragma once
 
 #include <cstdint>
@@ -42,6 +42,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same, but the thread may be suspended for up to `hint_ns` while the phase is incomplete
+// (it resumes when the phase completes), so a waiting warp does not consume issue slots.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -54,12 +68,10 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
                                                   volatile int* abort, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) return false;
-    }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -135,6 +147,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "memory");
 }
 
+// 32 lanes x 32 bit, 32 consecutive columns.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Store the same 32-bit value into 16 consecutive columns of the warp's 32 lanes.
@@ -142,6 +168,22 @@ __device__ __forceinline__ void tmem_st16_fill(uint32_t taddr, uint32_t v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
+
+// Store the same 32-bit value into 4 consecutive columns of the warp's 32 lanes (needs only 4
+// live copies of the value).
+__device__ __forceinline__ void tmem_st4_fill(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %1, %1, %1};" ::"r"(taddr), "r"(v) : "memory");
+}
+
+// Store the same 32-bit value into 32 consecutive columns of the warp's 32 lanes.
+__device__ __forceinline__ void tmem_st32_fill(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {"
+      "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+      "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
       "r"(v)
       : "memory");
 }
@@ -167,6 +209,81 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
 // 10..12 = 1), both K-major, N >> 3 in bits 17..22, M >> 4 in bits 24..28.
 __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
   return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// -------------------------------------------------------------- cp.async (4-byte, zero-fill)
+// Copies 4 bytes global -> shared; with src_bytes = 0 nothing is read and zeros are written.
+__device__ __forceinline__ void cp_async4(void* dst_smem, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared::cta.global [%0], [%1], 4, %2;" ::"r"(smem_addr(dst_smem)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
+// The mbarrier receives one arrival when all of this thread's earlier cp.async copies have
+// landed (the arrival counts toward the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// ------------------------------------------------------------------ packed float32 pairs
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t u2_pack(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// Four columns k of one accumulator row, two f32x2 FMAs per column pair:
+//   u_k = fma(bits(r_k), sw, csw)   with csw = -(1.5*2^23)*sw exact  ->  u_k = fl(d_k * sw)
+//   a_k = fma(u_k, s_k, a_k)
+// r_k are raw TMEM words holding 1.5*2^23 + d_k (an exact float); sw2/csw2 hold the row's
+// scale pair, s = (s0, s1, s2, s3) the four column scales.
+__device__ __forceinline__ void epi_fma4(float& a0, float& a1, float& a2, float& a3, float4 s, uint64_t sw2,
+                                         uint64_t csw2, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm("{\n\t.reg .b64 s01, s23, q01, q23, c01, c23;\n\t"
+      "mov.b64 q01, {%8, %9};\n\t"
+      "mov.b64 q23, {%10, %11};\n\t"
+      "fma.rn.f32x2 q01, q01, %12, %13;\n\t"
+      "fma.rn.f32x2 q23, q23, %12, %13;\n\t"
+      "mov.b64 s01, {%4, %5};\n\t"
+      "mov.b64 s23, {%6, %7};\n\t"
+      "mov.b64 c01, {%0, %1};\n\t"
+      "mov.b64 c23, {%2, %3};\n\t"
+      "fma.rn.f32x2 c01, q01, s01, c01;\n\t"
+      "fma.rn.f32x2 c23, q23, s23, c23;\n\t"
+      "mov.b64 {%0, %1}, c01;\n\t"
+      "mov.b64 {%2, %3}, c23;\n\t}"
+      : "+f"(a0), "+f"(a1), "+f"(a2), "+f"(a3)
+      : "f"(s.x), "f"(s.y), "f"(s.z), "f"(s.w), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "l"(sw2), "l"(csw2));
 }
 
 // -------------------------------------------------------------------- register budget

@@ -16,6 +16,7 @@
 #include <cuda_bf16.h>
 
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace pq {
 namespace {
@@ -43,30 +44,45 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float* v) {
   v[7] = __uint_as_float(w.w & 0xFFFF0000u);
 }
 
-// Unnormalised Walsh-Hadamard transform of 32 register values (Sylvester order).
+// Unnormalised Walsh-Hadamard transform of 32 register values (Sylvester order).  The first
+// stage pairs neighbours; the other four run on packed float pairs (two butterflies per
+// add.f32x2 / sub.f32x2, bit-identical to the scalar form).
 __device__ __forceinline__ void fwht32(float (&v)[32]) {
 #pragma unroll
-  for (int h = 1; h < 32; h <<= 1) {
+  for (int i = 0; i < 32; i += 2) {
+    const float a = v[i], b = v[i + 1];
+    v[i] = a + b;
+    v[i + 1] = a - b;
+  }
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+  for (int h = 2; h < 32; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
       if ((i & h) == 0) {
-        const float a = v[i], b = v[i + h];
-        v[i] = a + b;
-        v[i + h] = a - b;
+        const uint64_t P = ptx::f2_pack(v[i], v[i + 1]), Q = ptx::f2_pack(v[i + h], v[i + h + 1]);
+        ptx::f2_unpack(ptx::f2_add(P, Q), v[i], v[i + 1]);
+        ptx::f2_unpack(ptx::f2_sub(P, Q), v[i + h], v[i + h + 1]);
       }
     }
   }
 }
 
 // The two remaining radix-2 stages across the 4 lanes (lane bits 0,1 = channel bits 5,6):
-// the lane holding the low half keeps a + b, the other keeps a - b.
+// the lane holding the low half keeps a + b, the other keeps a - b (as +-v + partner).
 __device__ __forceinline__ void fwht_across4(float (&v)[32], int lane) {
   const float s1 = (lane & 1) ? -1.0f : 1.0f;
   const float s2 = (lane & 2) ? -1.0f : 1.0f;
+  const uint64_t S1 = ptx::f2_pack(s1, s1), S2 = ptx::f2_pack(s2, s2);
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = fmaf(s1, v[i], __shfl_xor_sync(0xffffffffu, v[i], 1));
+  for (int i = 0; i < 32; i += 2) {
+    const float p0 = __shfl_xor_sync(0xffffffffu, v[i], 1), p1 = __shfl_xor_sync(0xffffffffu, v[i + 1], 1);
+    ptx::f2_unpack(ptx::f2_fma(S1, ptx::f2_pack(v[i], v[i + 1]), ptx::f2_pack(p0, p1)), v[i], v[i + 1]);
+  }
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = fmaf(s2, v[i], __shfl_xor_sync(0xffffffffu, v[i], 2));
+  for (int i = 0; i < 32; i += 2) {
+    const float p0 = __shfl_xor_sync(0xffffffffu, v[i], 2), p1 = __shfl_xor_sync(0xffffffffu, v[i + 1], 2);
+    ptx::f2_unpack(ptx::f2_fma(S2, ptx::f2_pack(v[i], v[i + 1]), ptx::f2_pack(p0, p1)), v[i], v[i + 1]);
+  }
 }
 
 __device__ __forceinline__ float absmax32(const float (&v)[32]) {
@@ -82,13 +98,19 @@ __device__ __forceinline__ float group_max4(float m) {
   return m;
 }
 
-__device__ __forceinline__ float quant_inv(float m) { return m > 0.0f ? __fdiv_rn(7.0f, m) : 0.0f; }
+__device__ __forceinline__ float quant_inv(float m) { return m > 0.0f ? 7.0f * __frcp_rn(m) : 0.0f; }
 
 // 8 values -> 8 nibbles in one word: byte k = q[2k] | q[2k+1] << 4.
 __device__ __forceinline__ uint32_t quant_pack8(const float* v, float inv) {
   uint32_t b[8];
+  const uint64_t I2 = ptx::f2_pack(inv, inv), M2 = ptx::f2_pack(kRoundMagic, kRoundMagic);
 #pragma unroll
-  for (int k = 0; k < 8; ++k) b[k] = __float_as_uint(fmaf(v[k], inv, kRoundMagic));
+  for (int k = 0; k < 8; k += 2) {
+    float lo, hi;
+    ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(v[k], v[k + 1]), I2, M2), lo, hi);
+    b[k] = __float_as_uint(lo);
+    b[k + 1] = __float_as_uint(hi);
+  }
   const uint32_t even = __byte_perm(__byte_perm(b[0], b[2], 0x0040), __byte_perm(b[4], b[6], 0x0040), 0x5410);
   const uint32_t odd = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
   return (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
@@ -121,7 +143,9 @@ __device__ __forceinline__ void scale32(float (&v)[32], const float* s) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Flat stream of row-groups (row t, group gi), 8 per warp.  y = ((x * pre) H) * post.
+// Flat stream of row-groups (row t, group gi), 8 per warp-task, tasks strided over the grid.
+// y = ((x * pre) H) * post.  The next task's four 16-byte loads are issued before the current
+// task is transformed, so each warp keeps 2 KB in flight while it computes.
 __global__ void __launch_bounds__(256) hadamard_rows_kernel(
     const __nv_bfloat16* __restrict__ X, int64_t rows, int64_t ldx, int G,
     const float* __restrict__ pre, const float* __restrict__ post, uint8_t* __restrict__ codes,
@@ -129,32 +153,58 @@ __global__ void __launch_bounds__(256) hadamard_rows_kernel(
   const int lane = threadIdx.x & 31;
   const int q = lane & 3;
   const int64_t R = rows * (int64_t)G;
+  const int64_t ntasks = (R + 7) / 8;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (task >= ntasks) return;
   const int64_t halfD = (int64_t)G * 64;
-  for (int64_t base = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 8; base < R;
-       base += nwarps * 8) {
-    const int64_t r = base + (lane >> 2);
-    const bool valid = r < R;
-    const int64_t t = valid ? r / G : 0;
-    const int gi = valid ? (int)(r - t * G) : 0;
-    const int c0 = gi * 128 + q * 32;
-    float v[32];
-    if (valid) {
-      load32(X + t * ldx + c0, v);
+  // This lane's row-group r = 8 task + lane/4, kept as (t, gi) and advanced incrementally.
+  const int64_t stride = nwarps * 8;
+  const int64_t st_t = stride / G;
+  const int st_g = (int)(stride - st_t * G);
+  int64_t r = task * 8 + (lane >> 2);
+  int64_t t = r / G;
+  int gi = (int)(r - t * G);
+  uint4 cur[4], nxt[4];
+  auto load = [&](int64_t rr, int64_t tt, int gg, uint4 (&dst)[4]) {
+    if (rr < R) {
+      const uint4* p = reinterpret_cast<const uint4*>(X + tt * ldx + gg * 128 + q * 32);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dst[j] = ld_stream(p + j);
     } else {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+      for (int j = 0; j < 4; ++j) dst[j] = make_uint4(0, 0, 0, 0);
     }
+  };
+  load(r, t, gi, cur);
+  for (;;) {
+    const int64_t ntask = task + nwarps;
+    int64_t nr = r + stride, nt = t + st_t;
+    int ng = gi + st_g;
+    if (ng >= G) { ng -= G; ++nt; }
+    const bool more = ntask < ntasks;                  // warp-uniform
+    if (more) load(nr, nt, ng, nxt);
+    const int c0 = gi * 128 + q * 32;
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) bf16x8_to_f32(cur[j], v + 8 * j);
     if (pre) scale32(v, pre + c0);
     fwht32(v);
     fwht_across4(v, lane);
     if (post) scale32(v, post + c0);
     const float m = group_max4(absmax32(v));
     const uint4 packed = quant_pack32(v, quant_inv(m));
-    if (valid) {
+    if (r < R) {
       *reinterpret_cast<uint4*>(codes + t * halfD + gi * 64 + q * 16) = packed;
       if (q == 0) scales[r] = m * kScaleHadamard;
     }
+    if (!more) break;
+    task = ntask;
+    r = nr;
+    t = nt;
+    gi = ng;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
   }
 }
 
@@ -366,9 +416,15 @@ cudaError_t launch_hadamard_rows(const pq_plan* plan, const void* X, int64_t row
                                  const float* pre_scale, const float* post_scale, uint8_t* codes,
                                  float* scales, cudaStream_t stream) {
   const int64_t R = rows * plan->G;
-  const int64_t tasks = (R + 7) / 8;                // one warp-iteration = 8 row-groups
+  const int64_t tasks = (R + 7) / 8;                // one warp-task = 8 row-groups
   const int64_t want = (tasks + 7) / 8;             // 8 warps per block
-  const int64_t cap = (int64_t)sm_count() * 6;      // a few resident blocks per SM, grid-stride
+  static int per_sm = 0;
+  if (!per_sm) {
+    int b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, hadamard_rows_kernel, 256, 0) != cudaSuccess || b < 1) b = 2;
+    per_sm = b;
+  }
+  const int64_t cap = (int64_t)sm_count() * per_sm;  // one resident wave, tasks strided over it
   const int grid = (int)(want < cap ? want : cap);
   hadamard_rows_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(X), rows,
                                                  ldx, plan->G, pre_scale, post_scale, codes, scales);
