@@ -169,6 +169,27 @@ def config_of(wl, l2):
             "out": "float32", "l2": l2, "parallelism": "replicas (one independent workload per GPU)"}
 
 
+def max_over_ranks(x, world, device):
+    """Max of a per-rank float over all ranks (the process group's backend: NCCL on the GPU
+    arm, gloo in the CPU tests).  Every rank must call it, in the same order."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world, tokens_per_rank_step, steps, total_ms):
+    """Whole-job tokens/s: every rank processes its own workload (weak scaling); the slowest
+    rank's device time bounds the job."""
+    return world * tokens_per_rank_step * steps / (total_ms * 1e-3)
+
+
+# Kernels one step launches: transform_quant, pack_weights, int4 -> int8 expansion, GEMM.
+LAUNCHES_PER_STEP = 4
+
+
 # ------------------------------------------------------------------------ GPU arm
 def run_ours(args, wl, rank, world, local_rank):
     import numpy as np
@@ -254,20 +275,14 @@ def run_ours(args, wl, rank, world, local_rank):
 
     per = [[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in ev]     # ms
     step_ms = [sum(p) for p in per]
-    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
-    total_ms = float(total_ms.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     tq_ms = statistics.mean(p[0] for p in per)
     pw_ms = statistics.mean(p[1] for p in per)
     gm_ms = statistics.mean(p[2] for p in per)
 
     # ---------------------------------------------------------------- end to end
     e2e_ms, h2d, d2h = e2e_run(args, wl, pq, plan, dev, stream, flush, sm, smooth_w)
-    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
     if rank != 0:
         return
@@ -295,7 +310,7 @@ def run_ours(args, wl, rank, world, local_rank):
         roof = {"bound": "hbm", "achieved": comps[dominant]["GB_s"], "peak": hbm, "unit": "GB/s",
                 "frac": comps[dominant]["GB_s"] / hbm, "traffic": traffic, "kernel": dominant,
                 "peak_source": f"{peak_src} copy bandwidth"}
-    value = world * wl.T * args.steps / (total_ms * 1e-3)
+    value = job_value(world, wl.T, args.steps, total_ms)
     cpu = None
     if world == 1:
         full, spent, sample = oracle_sample(wl)
@@ -307,9 +322,9 @@ def run_ours(args, wl, rank, world, local_rank):
             "data": "synthetic (seeded SplitMix64 generator)",
             "config": config_of(wl, "flushed between steps (256 MiB write, then 256 MiB read)"),
             "components": comps, "roofline": roof, "cpu_baseline": cpu,
-            "e2e": {"value": world * wl.T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": job_value(world, wl.T, 1, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": 3 * args.steps, "clocks": ck, "wall_s_timed_region": w1 - w0}
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": ck, "wall_s_timed_region": w1 - w0}
     print(json.dumps(line), flush=True)
 
 
