@@ -160,6 +160,31 @@ pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A, const uint
                        const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
                        pq_out_dtype out_dtype, void* stream);
 
+/* Bytes of the fixed device-array scratch behind pq_w4a4_gemm_noalloc (32 MiB). */
+#define PQ_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/*
+ * pq_w4a4_gemm_noalloc — the same operation, arguments, layouts and results as pq_w4a4_gemm,
+ * for callers that cannot let a library allocate device memory (for example an engine that has
+ * reserved nearly all of it for its own caches, or a loop that needs a fixed footprint).  None
+ * of the pages has a counterpart: it only changes where the GEMM's temporary int8 operands live.
+ *   Scratch: a fixed device array of PQ_NOALLOC_SCRATCH_BYTES inside the library, one per
+ *   device, reserved when the CUDA module holding it is loaded (at the latest by the first
+ *   call on that device).  No call allocates or frees memory.  It needs no zeroing (each call writes all it reads).
+ *   Limit: (T + N) * D <= PQ_NOALLOC_SCRATCH_BYTES, else PQ_ERR_INVALID_ARG before anything is
+ *   launched.
+ *   First call on each device: looks up the scratch address with that device current; make it
+ *   before any stream capture.
+ *   Concurrency: calls on one device share the scratch.  Calls whose GPU work may overlap
+ *   (different streams without an event between them) race and can give wrong results; issue
+ *   them on one stream or order them with events.
+ *   Errors and timeouts are reported as for pq_w4a4_gemm.
+ */
+pq_status pq_w4a4_gemm_noalloc(const uint8_t* codes_A, const float* scales_A,
+                               const uint8_t* codes_W, const float* scales_W, int64_t T,
+                               int64_t N, int64_t D, int g, void* Y, pq_out_dtype out_dtype,
+                               void* stream);
+
 /*
  * pq_check_status — synchronises `stream`, then reads and clears the device status words
  * (the plan's, if plan != NULL, and the GEMM's).  Returns PQ_ERR_TIMEOUT if a bounded

@@ -522,6 +522,10 @@ pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t*
   return st;
 }
 
+cudaError_t gemm_status_address(unsigned int** status) {
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(status), g_gemm_status);
+}
+
 pq_status gemm_read_and_clear_status(unsigned int* bits) {
   unsigned int v = 0;
   pq_status st = cuda_fail(cudaMemcpyFromSymbol(&v, g_gemm_status, sizeof(v)), "read gemm status");

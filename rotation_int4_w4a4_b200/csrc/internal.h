@@ -77,5 +77,12 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
                       pq_out_dtype out_dtype, uint8_t* scratch, unsigned int* status,
                       cudaStream_t stream);
 pq_status gemm_read_and_clear_status(unsigned int* bits);
+// Device address of the GEMM's status word on the current device.
+cudaError_t gemm_status_address(unsigned int** status);
+// gemm_launch with the fixed device-array scratch of gemm_static_scratch.cu (no allocation).
+pq_status gemm_run_static_scratch(const uint8_t* codes_A, const float* scales_A,
+                                  const uint8_t* codes_W, const float* scales_W, int64_t T,
+                                  int64_t N, int64_t D, void* Y, pq_out_dtype out_dtype,
+                                  cudaStream_t stream);
 
 }  // namespace pq

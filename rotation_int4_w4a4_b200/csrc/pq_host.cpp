@@ -320,11 +320,12 @@ extern "C" pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t
   return cuda_fail(e, "pq_pack_weights launch");
 }
 
-extern "C" pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A,
-                                  const uint8_t* codes_W, const float* scales_W, int64_t T,
-                                  int64_t N, int64_t D, int g, void* Y, pq_out_dtype out_dtype,
-                                  void* stream) {
-  clear_error();
+namespace {
+
+// Argument checks shared by the GEMM entry points; nothing here touches the device.
+pq_status check_gemm_args(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
+                          const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
+                          pq_out_dtype out_dtype) {
   if (!codes_A || !scales_A || !codes_W || !scales_W || !Y) {
     set_error("all tensor pointers must be non-NULL");
     return PQ_ERR_INVALID_ARG;
@@ -343,8 +344,31 @@ extern "C" pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A,
     set_error("device pointers must be 16-byte aligned");
     return PQ_ERR_INVALID_ARG;
   }
+  return PQ_OK;
+}
+
+}  // namespace
+
+extern "C" pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A,
+                                  const uint8_t* codes_W, const float* scales_W, int64_t T,
+                                  int64_t N, int64_t D, int g, void* Y, pq_out_dtype out_dtype,
+                                  void* stream) {
+  clear_error();
+  pq_status st = check_gemm_args(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype);
+  if (st != PQ_OK) return st;
   return gemm_run(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype,
                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" pq_status pq_w4a4_gemm_noalloc(const uint8_t* codes_A, const float* scales_A,
+                                          const uint8_t* codes_W, const float* scales_W,
+                                          int64_t T, int64_t N, int64_t D, int g, void* Y,
+                                          pq_out_dtype out_dtype, void* stream) {
+  clear_error();
+  pq_status st = check_gemm_args(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype);
+  if (st != PQ_OK) return st;
+  return gemm_run_static_scratch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype,
+                                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" pq_status pq_check_status(const pq_plan* plan, void* stream) {

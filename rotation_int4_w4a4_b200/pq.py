@@ -26,8 +26,8 @@ KINDS = {"hadamard": PQ_HADAMARD, "givens": PQ_GIVENS, "smooth_hadamard": PQ_SMO
 
 # Every symbol the header declares.
 EXPORTS = ("pq_select_pairs", "pq_make_plan", "pq_destroy_plan", "pq_transform_quant",
-           "pq_pack_weights", "pq_w4a4_gemm", "pq_check_status", "pq_status_string",
-           "pq_last_error")
+           "pq_pack_weights", "pq_w4a4_gemm", "pq_w4a4_gemm_noalloc", "pq_check_status",
+           "pq_status_string", "pq_last_error")
 
 _c = ctypes
 _vp, _i64, _u64, _i32, _u32 = _c.c_void_p, _c.c_int64, _c.c_uint64, _c.c_int, _c.c_uint32
@@ -43,6 +43,8 @@ lib.pq_pack_weights.argtypes = [_vp, _vp, _i64, _vp, _vp, _vp, _vp]
 lib.pq_pack_weights.restype = _i32
 lib.pq_w4a4_gemm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _i32, _vp]
 lib.pq_w4a4_gemm.restype = _i32
+lib.pq_w4a4_gemm_noalloc.argtypes = lib.pq_w4a4_gemm.argtypes
+lib.pq_w4a4_gemm_noalloc.restype = _i32
 lib.pq_check_status.argtypes = [_vp, _vp]
 lib.pq_check_status.restype = _i32
 lib.pq_status_string.argtypes = [_i32]
@@ -161,6 +163,20 @@ def pq_w4a4_gemm(codes_A, scales_A, codes_W, scales_W, Y, T=None, N=None, D=None
         out_dtype = PQ_OUT_BF16 if Y.dtype == torch.bfloat16 else PQ_OUT_F32
     _check(lib.pq_w4a4_gemm(_ptr(codes_A), _ptr(scales_A), _ptr(codes_W), _ptr(scales_W),
                             T, N, D, g, _ptr(Y), out_dtype, _stream(stream)), "pq_w4a4_gemm")
+
+
+def pq_w4a4_gemm_noalloc(codes_A, scales_A, codes_W, scales_W, Y, T=None, N=None, D=None, g=128,
+                         out_dtype=None, stream=None) -> None:
+    """:func:`pq_w4a4_gemm` with the library's fixed scratch; (T + N) * D <= NOALLOC_SCRATCH_BYTES."""
+    T = codes_A.shape[0] if T is None else T
+    N = codes_W.shape[0] if N is None else N
+    D = codes_A.shape[1] * 2 if D is None else D
+    if out_dtype is None:
+        import torch
+        out_dtype = PQ_OUT_BF16 if Y.dtype == torch.bfloat16 else PQ_OUT_F32
+    _check(lib.pq_w4a4_gemm_noalloc(_ptr(codes_A), _ptr(scales_A), _ptr(codes_W), _ptr(scales_W),
+                                    T, N, D, g, _ptr(Y), out_dtype, _stream(stream)),
+           "pq_w4a4_gemm_noalloc")
 
 
 def pq_check_status(plan: Plan | None = None, stream=None) -> int:
