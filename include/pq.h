@@ -32,6 +32,9 @@
  *   16-byte aligned.  The library allocates no user-visible buffer.  A plan owns a few small
  *   device tables and a status word, allocated by pq_make_plan and freed by pq_destroy_plan;
  *   it is immutable after creation and may be used from several streams at once.
+ *   pq_w4a4_gemm takes (T + N) * D bytes of temporary scratch per call from a library-owned,
+ *   stream-ordered memory pool on the current device and returns it on the same stream; the
+ *   pool keeps freed memory for reuse, so it holds about the largest single call's need.
  *
  * Errors
  *   Every call returns pq_status and never throws, aborts or exits.  Arguments are validated
@@ -54,7 +57,7 @@ typedef enum pq_status {
   PQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, stride, alignment or plan */
   PQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. g != 128) */
   PQ_ERR_CUDA = 3,          /* a CUDA runtime call failed (message in pq_last_error) */
-  PQ_ERR_ALLOC = 4,         /* device allocation for a plan failed */
+  PQ_ERR_ALLOC = 4,         /* a device allocation (plan tables, GEMM scratch) failed */
   PQ_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up (see pq_check_status) */
 } pq_status;
 
@@ -155,6 +158,7 @@ pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t N, const f
  *   T >= 1, N >= 1 with N % 16 == 0, D % 128 == 0, g == 128.
  *   Y device [T][N] float32 (PQ_OUT_F32) or bf16 (PQ_OUT_BF16, RNE of the float32 result).
  *   Scales must be finite.  Every dot product fits int32 exactly (|d| <= 128*64).
+ *   Returns PQ_ERR_ALLOC if the stream-ordered scratch cannot be allocated.
  */
 pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                        const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
