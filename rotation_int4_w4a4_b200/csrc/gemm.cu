@@ -6,36 +6,35 @@
 //
 // Two kernels per call, ordered on the caller's stream:
 //
-// 1. expand_codes_kernel: int4 -> int8 for A and W into stream-ordered scratch.  Within each
-//    128-element group the low nibbles of the 64 packed bytes become K positions 0..63 and the
-//    high nibbles 64..127 (the same permutation on A and W, so every dot product is unchanged),
-//    each byte holding 16*code: no sign extension is needed and d = 256 * dot exactly.  The
-//    scratch rows are laid out so that one TMA box of 128 bytes x rows lands directly in the
-//    128-byte-swizzled K-major operand layout of the MMA.  (Unpacking inside the contraction
-//    kernel costs an extra shared-memory read and a double-size write per operand byte, and
-//    tensor-core operand reads take priority over that traffic on the shared-memory banks.)
+// 1. expand_codes_kernel: int4 codes -> E4M3 bytes for A and W into stream-ordered scratch.
+//    Every code in -8..7 is exact in E4M3, so the MMA's products and group sums (integers of
+//    magnitude <= 128 * 64 = 2^13) are exact in its float32 accumulator: d_G arrives in tensor
+//    memory as an exact float.  Within each 128-element group the low nibbles of the 64 packed
+//    bytes become K positions 0..63 and the high nibbles 64..127 (the same permutation on A and
+//    W, so every dot product is unchanged).  One TMA box of 128 bytes x rows then lands directly
+//    in the 128-byte-swizzled K-major operand layout.  (Unpacking inside the contraction kernel
+//    costs a shared-memory read and a double-size write per operand byte, and tensor-core operand
+//    reads take priority over that traffic on the shared-memory banks.)
 //
 // 2. w4a4_gemm_kernel: persistent, one CTA per SM.  The MMA computes the transposed tile
-//    D[n][t] (M = 128 output channels = TMEM lanes, N = 256 tokens), so every epilogue thread owns
-//    one output channel and its weight scale is a register constant; only the token scales are
-//    broadcast from shared memory.  The K loop runs one 128-wide group per step.  Warp roles
-//    (12 warps):
-//      warp 0      TMA producer: int8 tiles of W (128 x 128 B) and X (256 x 128 B) per group
+//    D[n][t] (M = 128 output channels = TMEM lanes, N = 256 tokens).  The K loop runs one
+//    128-wide group per step.  Warp roles (12 warps):
+//      warp 0      TMA producer: E4M3 tiles of W (128 x 128 B) and X (256 x 128 B) per group
 //                  into a 4-stage ring.
-//      warp 1      TMEM allocator and MMA issuer: 4 x tcgen05.mma kind::i8 (M128 N256 K32) per
-//                  group into a double-buffered int32 accumulator in tensor memory.
-//      warps 2..3  scale loaders: per group, the tile's 128 weight scales and 256 activation
-//                  scales are copied (cp.async, zero-filled past N / T) into an 8-stage ring.
-//      warps 4..11 epilogue (2 per TMEM lane quarter, 128 tokens each): per group, read the
-//                  int32 tile from TMEM and accumulate
-//                  acc += fl(d * sw) * sa / 256 in float32 registers (ascending group order) with
-//                  two packed f32x2 FMAs per column pair; after the last group, store Y.
-//    Exact int32 -> float32 conversion and weight scaling in one FMA: each accumulator buffer is
-//    pre-loaded with the bit pattern of C = 1.5*2^23; since |d| <= 2^21, (bits + d) is the float
-//    C + d.  The weight scale is rounded to a 22-bit significand (relative change <= 2^-22), which
-//    makes C * sw exact, so fma(C + d, sw, -C * sw) = fl(d * sw) with one rounding.  Weight scales
-//    must satisfy |sw| < 2^100 for C * sw to stay finite.  Every mbarrier wait is bounded; a timeout
-//    sets a status bit, the CTA drains its own copies and MMAs, frees tensor memory and returns.
+//      warp 1      TMEM allocator and MMA issuer: 4 x tcgen05.mma kind::f8f6f4 (M128 N256 K32)
+//                  per group into a double-buffered float32 accumulator; the first of the four
+//                  overwrites the buffer.
+//      warps 2..3  scale loaders: the tile's weight and activation scales for 4 groups at a time
+//                  ([row][4] float32, cp.async, zero-filled past N / T / G) into a 4-stage ring.
+//      warps 4..11 epilogue: 2 warps per TMEM lane quarter, 128 tokens each.  Tensor memory is
+//                  read with the 16x256b shape, so each thread holds 4 output channels x 32
+//                  tokens: per group it needs 4 weight scales and 32 token scales (a quarter of
+//                  the shared-memory traffic of one channel x 128 tokens per thread).  Per element
+//                  acc += fl(d * sw) * sa in float32 registers, groups in ascending order, with
+//                  one packed multiply and one packed FMA per element pair; after the last group
+//                  the tile is stored to Y.
+//    Every mbarrier wait is bounded; a timeout sets a status bit, the CTA drains its own copies
+//    and MMAs, frees tensor memory and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -51,27 +50,36 @@ __device__ unsigned int g_gemm_status = 0;
 
 namespace {
 
-constexpr int BM = 128;        // tile rows = output channels (weight rows), MMA M
-constexpr int BN = 256;        // tile columns = tokens (activation rows), MMA N
-constexpr int BK = 128;        // one quantisation group = 128 int8 = one 128-byte swizzle row
-constexpr int OP_STAGES = 4;   // operand ring
-constexpr int S_STAGES = 8;    // scale ring
-constexpr int NUM_THREADS = 384;
+constexpr int BM = 128;          // tile rows = output channels (weight rows), MMA M
+constexpr int BN = 256;          // tile columns = tokens (activation rows), MMA N
+constexpr int BK = 128;          // one quantisation group = 128 bytes = one 128-byte swizzle row
+constexpr int OP_STAGES = 4;     // operand ring
+constexpr int SC_GROUPS = 4;     // groups per scale stage
+constexpr int S_STAGES = 4;      // scale ring
 constexpr int NUM_EPI_WARPS = 8;
-constexpr int EPI_COLS = BN / (NUM_EPI_WARPS / 4);   // tokens per epilogue warp (64)
-constexpr int EPI_WARP0 = 4;
-constexpr int NUM_SCALE_THREADS = 64;  // warps 2 and 3
+constexpr int EPI_WARP0 = 4;     // warps 0..3 control, 4..11 epilogue
+constexpr int NUM_THREADS = 32 * (EPI_WARP0 + NUM_EPI_WARPS);
+constexpr int EPI_COLS = BN / (NUM_EPI_WARPS / 4);   // tokens per epilogue warp (128)
+constexpr int EPI_CHUNKS = EPI_COLS / 16;            // 16-token TMEM loads per lane half
+constexpr int NUM_SCALE_THREADS = 64;                // warps 2 and 3
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t kAccBias = 0x4B400000u;          // bit pattern of 1.5 * 2^23
-constexpr float kAccBiasF = 12582912.0f;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;    // 2 s
+constexpr uint64_t kWaitLimitNs = 2000000000ull;     // 2 s
 constexpr uint32_t kTxBytes = (BM + BN) * BK;
+// Register budget (setmaxnreg): launch allocation per thread and the control and epilogue
+// warps' shares; 128 * REG_CTRL + 256 * REG_EPI must not exceed 384 * REG_LAUNCH.
+constexpr uint32_t REG_LAUNCH = 168;
+constexpr uint32_t REG_CTRL = 56;
+constexpr uint32_t REG_EPI = 224;
+static_assert(REG_CTRL * 32 * EPI_WARP0 + REG_EPI * 32 * NUM_EPI_WARPS <= REG_LAUNCH * NUM_THREADS,
+              "setmaxnreg shares exceed the launch allocation");
+static_assert(REG_LAUNCH * NUM_THREADS <= 65536, "launch register allocation exceeds the SM");
+static_assert(EPI_COLS == 128, "the epilogue below assumes 128 tokens per warp");
 
 struct __align__(1024) GemmSmem {
-  uint8_t opA[OP_STAGES][BM * BK];   // weights, 16 KB per stage, 128-byte swizzle
-  uint8_t opB[OP_STAGES][BN * BK];   // activations, 32 KB per stage
-  float sc_w[S_STAGES][BM];          // weight scales of the tile's rows, one group per stage
-  float sc_a[S_STAGES][BN];          // activation scales of the tile's columns
+  uint8_t opA[OP_STAGES][BM * BK];          // weights, 16 KB per stage, 128-byte swizzle
+  uint8_t opB[OP_STAGES][BN * BK];          // activations, 32 KB per stage
+  float sc_w[S_STAGES][BM][SC_GROUPS];      // weight scales: [tile row][group of the stage]
+  float sc_a[S_STAGES][BN][SC_GROUPS];      // activation scales: [tile token][group]
   uint64_t op_full[OP_STAGES];
   uint64_t op_empty[OP_STAGES];
   uint64_t acc_full[2];
@@ -84,6 +92,7 @@ struct __align__(1024) GemmSmem {
 };
 
 constexpr size_t kSmemBytes = sizeof(GemmSmem) + 1024;   // + slack for 1024-byte alignment
+static_assert(kSmemBytes <= 232448, "shared memory exceeds 227 KB");
 
 __device__ __forceinline__ void raise_abort(GemmSmem& S, unsigned int* status) {
   S.abort_flag = 1;
@@ -116,8 +125,23 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------------------------ expand
-// One thread per 16 packed bytes (32 codes of one group): writes the 16 low-nibble bytes at K
-// offset 16p and the 16 high-nibble bytes at 64 + 16p of the group's 128-byte int8 row.
+// Four codes (one per byte of x, each 0..15 as two's-complement nibbles) -> four E4M3 bytes.
+// Byte permutes look the magnitudes up in two 8-entry tables (codes 0..7 and -8..-1); bit 3 of
+// each code selects between them.
+__device__ __forceinline__ uint32_t codes_to_e4m3(uint32_t x) {
+  constexpr uint32_t kPos0 = 0x44403800u, kPos1 = 0x4E4C4A48u;   // 0, 1, 2, 3 | 4, 5, 6, 7
+  constexpr uint32_t kNeg0 = 0xCACCCED0u, kNeg1 = 0xB8C0C4C8u;   // -8, -7, -6, -5 | -4, -3, -2, -1
+  const uint32_t idx = x & 0x07070707u;
+  const uint32_t t = idx | (idx >> 4);
+  const uint32_t sel = (t & 0xFFu) | ((t >> 8) & 0xFF00u);     // four 3-bit indices as nibbles
+  const uint32_t pos = __byte_perm(kPos0, kPos1, sel);
+  const uint32_t neg = __byte_perm(kNeg0, kNeg1, sel);
+  const uint32_t m = ((x >> 3) & 0x01010101u) * 0xFFu;
+  return (pos & ~m) | (neg & m);
+}
+
+// One thread per 16 packed bytes (32 codes of one group): writes the 16 low-nibble codes at K
+// offset 16p and the 16 high-nibble codes at 64 + 16p of the group's 128-byte row.
 __global__ void __launch_bounds__(256) expand_codes_kernel(const uint8_t* __restrict__ A, int64_t chunksA,
                                                            const uint8_t* __restrict__ W, int64_t chunksW,
                                                            uint8_t* __restrict__ A8, uint8_t* __restrict__ W8) {
@@ -129,18 +153,20 @@ __global__ void __launch_bounds__(256) expand_codes_kernel(const uint8_t* __rest
     const int64_t group = c >> 2;          // 4 chunks of 16 bytes per 64-byte packed group
     const int p = (int)(c & 3);
     uint8_t* dst = (isA ? A8 : W8) + group * 128 + 16 * p;
-    *reinterpret_cast<uint4*>(dst) = make_uint4((w.x << 4) & 0xF0F0F0F0u, (w.y << 4) & 0xF0F0F0F0u,
-                                                (w.z << 4) & 0xF0F0F0F0u, (w.w << 4) & 0xF0F0F0F0u);
+    *reinterpret_cast<uint4*>(dst) =
+        make_uint4(codes_to_e4m3(w.x & 0x0F0F0F0Fu), codes_to_e4m3(w.y & 0x0F0F0F0Fu),
+                   codes_to_e4m3(w.z & 0x0F0F0F0Fu), codes_to_e4m3(w.w & 0x0F0F0F0Fu));
     *reinterpret_cast<uint4*>(dst + 64) =
-        make_uint4(w.x & 0xF0F0F0F0u, w.y & 0xF0F0F0F0u, w.z & 0xF0F0F0F0u, w.w & 0xF0F0F0F0u);
+        make_uint4(codes_to_e4m3((w.x >> 4) & 0x0F0F0F0Fu), codes_to_e4m3((w.y >> 4) & 0x0F0F0F0Fu),
+                   codes_to_e4m3((w.z >> 4) & 0x0F0F0F0Fu), codes_to_e4m3((w.w >> 4) & 0x0F0F0F0Fu));
   }
 }
 
 // -------------------------------------------------------------------------- control
 __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA, const CUtensorMap& tmB,
                                             const float* __restrict__ scales_A, const float* __restrict__ scales_W,
-                                            uint32_t tmem, int T, int N, int G, int m_tiles, int num_tiles,
-                                            unsigned int* status) {
+                                            uint32_t tmem, int T, int N, int G, int scales_vec16, int m_tiles,
+                                            int num_tiles, unsigned int* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -165,7 +191,7 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
   } else if (warp == 1) {
     // ------------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = ptx::idesc_i8(BM, BN);
+      constexpr uint32_t idesc = ptx::idesc_e4m3_f32(BM, BN);
       int step = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
@@ -174,15 +200,17 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
           const uint32_t ph = (uint32_t)(step / OP_STAGES) & 1u;
           const int b = step & 1;
           const uint32_t u = (uint32_t)(step >> 1);
-          if (!wait_or_abort(S, &S.acc_empty[b], u & 1u, status)) { ok = false; break; }
+          // the first use of each buffer passes at once (parity of the phase before the first)
+          if (!wait_or_abort(S, &S.acc_empty[b], (u & 1u) ^ 1u, status)) { ok = false; break; }
           if (!wait_or_abort(S, &S.op_full[s], ph, status)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t a0 = ptx::smem_addr(S.opA[s]);
           const uint32_t b0 = ptx::smem_addr(S.opB[s]);
           const uint32_t d = tmem + (uint32_t)b * BN;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            ptx::umma_i8(d, ptx::smem_desc_sw128(a0 + 32 * k), ptx::smem_desc_sw128(b0 + 32 * k), idesc, 1u);
+          for (int k = 0; k < 4; ++k)   // k = 0 overwrites the buffer: each group starts from 0
+            ptx::umma_e4m3(d, ptx::smem_desc_sw128(a0 + 32 * k), ptx::smem_desc_sw128(b0 + 32 * k), idesc,
+                           k > 0 ? 1u : 0u);
           ptx::umma_commit(&S.op_empty[s]);
           ptx::umma_commit(&S.acc_full[b]);
         }
@@ -192,28 +220,33 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
     }
   } else {
     // ---------------------------------------------------------------- scale loaders
+    // Per stage: SC_GROUPS consecutive groups of the tile's 128 weight rows and 256 tokens.
     const int j = threadIdx.x - 64;                      // 0..63
-    int step = 0;
+    int cs = 0;                                          // scale stages filled so far
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
       const int m0 = (tile % m_tiles) * BM, n0 = (tile / m_tiles) * BN;
-      for (int kg = 0; kg < G; ++kg, ++step) {
-        const int ss = step % S_STAGES;
-        const uint32_t sph = (uint32_t)(step / S_STAGES) & 1u;
-        if (!warp_wait_or_abort(S, &S.sc_empty[ss], sph ^ 1u, status)) { ok = false; break; }
+      for (int kg0 = 0; kg0 < G; kg0 += SC_GROUPS, ++cs) {
+        const int st = cs % S_STAGES;
+        const uint32_t sph = (uint32_t)(cs / S_STAGES) & 1u;
+        if (!warp_wait_or_abort(S, &S.sc_empty[st], sph ^ 1u, status)) { ok = false; break; }
 #pragma unroll
-        for (int i = 0; i < BM / NUM_SCALE_THREADS; ++i) {
-          const int n = m0 + j + NUM_SCALE_THREADS * i;
-          const bool in = n < N;
-          ptx::cp_async4(&S.sc_w[ss][j + NUM_SCALE_THREADS * i], scales_W + (int64_t)(in ? n : 0) * G + kg, in ? 4u : 0u);
-        }
+        for (int i = 0; i < (BM + BN) / NUM_SCALE_THREADS; ++i) {
+          const int r = j + NUM_SCALE_THREADS * i;       // 0..127 weight rows, 128..383 tokens
+          const bool isw = r < BM;
+          const int row = isw ? m0 + r : n0 + (r - BM);
+          const bool in = row < (isw ? N : T);
+          const float* src = (isw ? scales_W : scales_A) + (int64_t)(in ? row : 0) * G + kg0;
+          float* dst = isw ? S.sc_w[st][r] : S.sc_a[st][r - BM];
+          if (scales_vec16) {
+            ptx::cp_async16(dst, src, in ? 16u : 0u);    // G % 4 == 0: 16-byte aligned rows
+          } else {
 #pragma unroll
-        for (int i = 0; i < BN / NUM_SCALE_THREADS; ++i) {
-          const int t = n0 + j + NUM_SCALE_THREADS * i;
-          const bool in = t < T;
-          ptx::cp_async4(&S.sc_a[ss][j + NUM_SCALE_THREADS * i], scales_A + (int64_t)(in ? t : 0) * G + kg, in ? 4u : 0u);
+            for (int e = 0; e < SC_GROUPS; ++e)
+              ptx::cp_async4(dst + e, in && kg0 + e < G ? src + e : src - kg0, in && kg0 + e < G ? 4u : 0u);
+          }
         }
-        ptx::cp_async_arrive_noinc(&S.sc_full[ss]);
+        ptx::cp_async_arrive_noinc(&S.sc_full[st]);
       }
     }
     ptx::cp_async_wait_all();
@@ -221,106 +254,107 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
 }
 
 // ------------------------------------------------------------------------- epilogue
+// Thread layout (16x256b loads): in warp ew, TMEM lane quarter sub = warp % 4 (rows 32 sub ..),
+// token half ch = ew / 4 (tokens 128 ch ..); lane L has g = L / 4, q = L % 4.  Its rows are
+// 32 sub + 16 h + g + 8 k and its tokens 128 ch + 16 c + 8 x + 2 q + e (h, k, x, e in {0, 1},
+// c in 0..7).  acc index: ((h * 2 + k) * 8 + c) * 4 + x * 2 + e.
 __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* __restrict__ Y, int T, int N,
                                              int G, int out_bf16, int m_tiles, int num_tiles, unsigned int* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ew = warp - EPI_WARP0;
   const int sub = warp & 3;          // TMEM lane quarter this warp may access
   const int ch = ew >> 2;            // token half of the tile
-  const uint32_t lane_base = (uint32_t)(sub * 32) << 16;
-  // Pre-load both accumulator buffers with the conversion bias, then release them.
-#pragma unroll
-  for (int b = 0; b < 2; ++b)
-#pragma unroll
-    for (int c = 0; c < EPI_COLS / 16; ++c) ptx::tmem_st16_fill(tmem + lane_base + b * BN + ch * EPI_COLS + 16 * c, kAccBias);
-  ptx::tmem_st_wait();
-  ptx::tc_fence_before();
-  __syncwarp();
-  if (lane == 0) {
-    ptx::mbar_arrive(&S.acc_empty[0]);
-    ptx::mbar_arrive(&S.acc_empty[1]);
-  }
-  int step = 0;
+  const int g = lane >> 2, q = lane & 3;
+  int step = 0, cs = 0;
   bool ok = true;
-  bool pending = false;              // re-arm stores of the previous step not yet waited for
-  int prev_b = 0, prev_ss = 0;
   for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
     const int m0 = (tile % m_tiles) * BM, n0 = (tile / m_tiles) * BN;
-    const int n = m0 + sub * 32 + lane;        // this thread's output channel
-    const int tcol = n0 + ch * EPI_COLS;       // first of this warp's tokens
-    float acc[EPI_COLS];                       // Y[tcol + j][n], float32
+    constexpr int kAcc = 4 * 2 * EPI_CHUNKS * 2;      // rows (h, k) x chunks x tokens (x, e)
+    static_assert(kAcc == EPI_COLS, "4 channels x EPI_COLS / 4 tokens per thread");
+    float acc[kAcc];
 #pragma unroll
-    for (int i = 0; i < EPI_COLS; ++i) acc[i] = 0.0f;
+    for (int i = 0; i < kAcc; ++i) acc[i] = 0.0f;
     for (int kg = 0; kg < G; ++kg, ++step) {
       const int b = step & 1;
       const uint32_t u = (uint32_t)(step >> 1);
-      const int ss = step % S_STAGES;
-      const uint32_t sph = (uint32_t)(step / S_STAGES) & 1u;
-      if (!warp_wait_or_abort(S, &S.sc_full[ss], sph, status)) { ok = false; break; }
-      // Weight scale / 256 (undoes the 16 x 16 of the expansion, exactly), rounded to a 22-bit
-      // significand so that C * sw is exact.
-      const float sw = __uint_as_float((__float_as_uint(S.sc_w[ss][sub * 32 + lane] * 0.00390625f) + 2u) & ~3u);
-      const float csw = -kAccBiasF * sw;
-      const uint64_t sw2 = ptx::f2_pack(sw, sw), csw2 = ptx::f2_pack(csw, csw);
-      const float4* sap = reinterpret_cast<const float4*>(&S.sc_a[ss][ch * EPI_COLS]);
+      const int st = cs % S_STAGES;
+      const int gi = kg % SC_GROUPS;
+      if (gi == 0 && !warp_wait_or_abort(S, &S.sc_full[st], (uint32_t)(cs / S_STAGES) & 1u, status)) {
+        ok = false;
+        break;
+      }
+      // This step's scales: one base address each, every other offset a constant.
+      const float* swb = &S.sc_w[st][32 * sub + g][gi];
+      const float* sab = &S.sc_a[st][ch * EPI_COLS + 2 * q][gi];
+      uint64_t sw2[4];                               // weight scale of row (h, k), twice
+#pragma unroll
+      for (int hk = 0; hk < 4; ++hk) {
+        const float sw = swb[(16 * (hk >> 1) + 8 * (hk & 1)) * SC_GROUPS];
+        sw2[hk] = ptx::f2_pack(sw, sw);
+      }
       if (!warp_wait_or_abort(S, &S.acc_full[b], u & 1u, status)) { ok = false; break; }
       ptx::tc_fence_after();
-      const uint32_t taddr = tmem + lane_base + (uint32_t)(b * BN + ch * EPI_COLS);
+      const uint32_t tbase = tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(b * BN + ch * EPI_COLS);
 #pragma unroll
-      for (int c = 0; c < EPI_COLS / 32; ++c) {
-        uint32_t r[32];
-        ptx::tmem_ld32(taddr + 32 * c, r);
-        ptx::tmem_ld_wait();
-        if (c == 0 && pending) {
-          // The previous buffer's bias stores were issued a whole TMEM load ago: complete them
-          // and hand that buffer back to the MMA.
-          ptx::tmem_st_wait();
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            ptx::mbar_arrive(&S.acc_empty[prev_b]);
-            ptx::mbar_arrive(&S.sc_empty[prev_ss]);
+      for (int c = 0; c < EPI_CHUNKS; ++c) {
+        uint64_t sa2[2];                             // token scales of columns 8x + 2q + {0, 1}
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+          sa2[x] = ptx::f2_pack(sab[(16 * c + 8 * x) * SC_GROUPS], sab[(16 * c + 8 * x + 1) * SC_GROUPS]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {                // lane half: rows 16 h + g + 8 k
+          uint32_t d[8];
+          ptx::tmem_ld_16x256b_x2(tbase + ((uint32_t)(16 * h) << 16) + 16 * c, d);
+          ptx::tmem_ld_wait(d);
+          if (c == EPI_CHUNKS - 1 && h == 1) {
+            // The whole group's tile is read: hand the buffer back to the MMA before the math.
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&S.acc_empty[b]);
           }
-          pending = false;
-        }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int i0 = 32 * c + 4 * j;
-          ptx::epi_fma4(acc[i0], acc[i0 + 1], acc[i0 + 2], acc[i0 + 3], sap[8 * c + j], sw2, csw2, r[4 * j],
-                        r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+          for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int i = ((h * 2 + k) * EPI_CHUNKS + c) * 4 + x * 2;
+              ptx::mul_fma2(acc[i], acc[i + 1], d[4 * x + 2 * k], d[4 * x + 2 * k + 1], sw2[h * 2 + k], sa2[x]);
+            }
         }
       }
-      // Re-arm this buffer with the conversion bias for the MMA two steps ahead; completion is
-      // awaited after the next step's first TMEM load.
-#pragma unroll
-      for (int c = 0; c < EPI_COLS / 4; ++c) ptx::tmem_st4_fill(taddr + 4 * c, kAccBias);
-      pending = true;
-      prev_b = b;
-      prev_ss = ss;
+      if (gi == SC_GROUPS - 1 || kg == G - 1) {
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&S.sc_empty[st]);
+        ++cs;
+      }
     }
     if (!ok) break;
-    // Y[t][n]: the 32 lanes of a warp write 32 consecutive channels of one token per store.
-    if (n < N) {
-      if (!out_bf16) {
-        float* ycol = reinterpret_cast<float*>(Y) + (int64_t)tcol * N + n;
+    // Y[t][n]: per store, 8 lanes (same q) write 8 consecutive channels of one token.  The
+    // thread's channels are nb + {0, 8, 16, 24}, its tokens tb + 16 c + 8 x + e.
+    const int nb = m0 + 32 * sub + g;
+    const int tb = n0 + ch * EPI_COLS + 2 * q;
+    bool nin[4];
 #pragma unroll
-        for (int j = 0; j < EPI_COLS; ++j)
-          if (tcol + j < T) ycol[(int64_t)j * N] = acc[j];
-      } else {
-        __nv_bfloat16* ycol = reinterpret_cast<__nv_bfloat16*>(Y) + (int64_t)tcol * N + n;
+    for (int hk = 0; hk < 4; ++hk) nin[hk] = nb + 8 * hk < N;
+    const size_t esz = out_bf16 ? 2 : 4;
+    char* row = reinterpret_cast<char*>(Y) + ((int64_t)tb * N + nb) * esz;
+    const int64_t row_step = (int64_t)N * esz;
 #pragma unroll
-        for (int j = 0; j < EPI_COLS; ++j)
-          if (tcol + j < T) ycol[(int64_t)j * N] = __float2bfloat16_rn(acc[j]);
+    for (int c = 0; c < EPI_CHUNKS; ++c) {
+#pragma unroll
+      for (int xe = 0; xe < 4; ++xe) {
+        const int dt = 8 * (xe >> 1) + (xe & 1);
+        if (tb + 16 * c + dt < T) {
+          char* p = row + dt * row_step;
+#pragma unroll
+          for (int hk = 0; hk < 4; ++hk) {
+            if (!nin[hk]) continue;
+            const float v = acc[(hk * EPI_CHUNKS + c) * 4 + xe];   // rows 16 h + 8 k = 8 hk
+            if (!out_bf16) reinterpret_cast<float*>(p)[8 * hk] = v;
+            else reinterpret_cast<__nv_bfloat16*>(p)[8 * hk] = __float2bfloat16_rn(v);
+          }
+        }
       }
-    }
-  }
-  if (pending) {
-    ptx::tmem_st_wait();
-    ptx::tc_fence_before();
-    __syncwarp();
-    if (lane == 0) {
-      ptx::mbar_arrive(&S.acc_empty[prev_b]);
-      ptx::mbar_arrive(&S.sc_empty[prev_ss]);
+      row += 16 * row_step;
     }
   }
 }
@@ -328,7 +362,7 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
 __global__ void __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const float* __restrict__ scales_A, const float* __restrict__ scales_W, void* __restrict__ Y,
-    int T, int N, int G, int out_bf16, int m_tiles, int n_tiles, unsigned int* status) {
+    int T, int N, int G, int scales_vec16, int out_bf16, int m_tiles, int n_tiles, unsigned int* status) {
   extern __shared__ unsigned char smem_raw[];
   GemmSmem& S = *reinterpret_cast<GemmSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -365,13 +399,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
   ptx::tc_fence_after();
   const uint32_t tmem = S.tmem_slot;
 
-  // Register budget: 384 threads x 168 at launch; warps 0..3 give back to 56, warps 4..11 take
-  // 224 (128 x 56 + 256 x 224 = 64512 = 384 x 168).
   if (warp < EPI_WARP0) {
-    ptx::setmaxnreg_dec<56>();
-    cta_control(S, tmA, tmB, scales_A, scales_W, tmem, T, N, G, m_tiles, num_tiles, status);
+    ptx::setmaxnreg_dec<REG_CTRL>();
+    cta_control(S, tmA, tmB, scales_A, scales_W, tmem, T, N, G, scales_vec16, m_tiles, num_tiles, status);
   } else {
-    ptx::setmaxnreg_inc<224>();
+    ptx::setmaxnreg_inc<REG_EPI>();
     cta_epilogue(S, tmem, Y, T, N, G, out_bf16, m_tiles, num_tiles, status);
   }
 
@@ -492,8 +524,24 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   const int grid = (int)(tiles < sms ? tiles : sms);
   e = cudaFuncSetAttribute(w4a4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm smem)");
+  // The warp roles re-divide the launch's registers with setmaxnreg; that only works when the
+  // kernel was compiled with exactly the budgeted count (otherwise an increase would never be
+  // granted), so refuse to launch anything else.
+  static int num_regs = -1;
+  if (num_regs < 0) {
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, w4a4_gemm_kernel);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(gemm)");
+    num_regs = fa.numRegs;
+  }
+  if (num_regs != (int)REG_LAUNCH) {
+    set_error("w4a4_gemm_kernel compiled with %d registers per thread, %u expected", num_regs, REG_LAUNCH);
+    return PQ_ERR_CUDA;
+  }
+  const int G = (int)(D / 128);
+  const int scales_vec16 = (G % SC_GROUPS == 0) ? 1 : 0;   // rows of 16-byte multiples
   w4a4_gemm_kernel<<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB, scales_A, scales_W, Y, (int)T, (int)N,
-                                                               (int)(D / 128), out_dtype == PQ_OUT_BF16 ? 1 : 0,
+                                                               G, scales_vec16, out_dtype == PQ_OUT_BF16 ? 1 : 0,
                                                                m_tiles, n_tiles, status);
   return cuda_fail(cudaGetLastError(), "w4a4_gemm_kernel launch");
 }

@@ -128,6 +128,24 @@ __device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
+// Instruction descriptor for kind::f8f6f4 with E4M3 A and B, float32 accumulator, both operands
+// K-major: D format bits 4-5 (1 = F32), A/B formats bits 7-9 / 10-12 (0 = E4M3), N/8 at bit 17,
+// M/16 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D (+)= A * B^T on E4M3 operands with float32 accumulation in tensor memory.
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on `bar` once all previously issued tcgen05 MMAs of this thread have completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -145,6 +163,26 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[15])
       : "r"(taddr)
       : "memory");
+}
+
+// 16 lanes x 256 bit, twice (16 columns): thread T receives r[4x + 0..1] = lane T/4, columns
+// 8x + 2(T%4) + 0..1 and r[4x + 2..3] = lane T/4 + 8, same columns (x = 0, 1), relative to the
+// lane and column of taddr.
+__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
+
+// Waits for this thread's TMEM loads and passes the 8 destination registers through the wait,
+// so that no use of them can be scheduled between the load and its completion (the compiler
+// sees the registers as defined by the load instruction itself).
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7])
+               :
+               : "memory");
 }
 
 // 32 lanes x 32 bit, 32 consecutive columns.
@@ -219,6 +257,13 @@ __device__ __forceinline__ void cp_async4(void* dst_smem, const void* src, uint3
                : "memory");
 }
 
+// 16-byte copy (L2 only); src_bytes < 16 zero-fills the rest (0 reads nothing).
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared::cta.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst_smem)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+
 // The mbarrier receives one arrival when all of this thread's earlier cp.async copies have
 // landed (the arrival counts toward the barrier's expected count).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
@@ -233,6 +278,15 @@ __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
   return r;
 }
+// (a0, a1) += (d0 * s, d1 * s) * (t0, t1) elementwise: one packed multiply, one packed FMA.
+// d0, d1 are float32 bit patterns; s2 = {s, s}; t2 = {t0, t1}.
+__device__ __forceinline__ void mul_fma2(float& a0, float& a1, uint32_t d0, uint32_t d1, uint64_t s2, uint64_t t2) {
+  asm("{ .reg .b64 d, a; mov.b64 d, {%2, %3}; mul.rn.f32x2 d, d, %4; mov.b64 a, {%0, %1};"
+      " fma.rn.f32x2 a, d, %5, a; mov.b64 {%0, %1}, a; }"
+      : "+f"(a0), "+f"(a1)
+      : "r"(d0), "r"(d1), "l"(s2), "l"(t2));
+}
+
 __device__ __forceinline__ uint64_t u2_pack(uint32_t lo, uint32_t hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
