@@ -107,7 +107,9 @@ pq_status pq_select_pairs(uint64_t seed, int D, int g, int K, int N, uint8_t* pa
  *           §2.3).  Activations are multiplied by exp(-beta) after the rotations and weights by
  *           exp(+beta), so that the product is unchanged before quantisation.
  *   flags   PQ_FLAG_* bits.
- *   cos/sin and exp(+-beta) are evaluated on the host in double precision and stored as float.
+ *   Givens: per group the K layers and exp(-+beta) are composed on the host in double precision
+ *   into one 128 x 128 matrix (one for activations, one for weights), stored as a bf16 pair
+ *   hi + lo (about 2^-17 relative); the transform is then a tensor-core product y = x R.
  *   The plan is created on the current device.  *out is set only on success.
  */
 pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int K, const uint8_t* pairs,

@@ -269,11 +269,11 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
   bool ok = true;
   for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
     const int m0 = (tile % m_tiles) * BM, n0 = (tile / m_tiles) * BN;
-    constexpr int kAcc = 4 * 2 * EPI_CHUNKS * 2;      // rows (h, k) x chunks x tokens (x, e)
-    static_assert(kAcc == EPI_COLS, "4 channels x EPI_COLS / 4 tokens per thread");
-    float acc[kAcc];
+    constexpr int kAcc2 = 4 * EPI_CHUNKS * 2;         // rows (h, k) x chunks x x; e is the pair
+    static_assert(2 * kAcc2 == EPI_COLS, "4 channels x EPI_COLS / 4 tokens per thread");
+    uint64_t acc2[kAcc2];                            // float32 pairs (tokens 2q, 2q + 1)
 #pragma unroll
-    for (int i = 0; i < kAcc; ++i) acc[i] = 0.0f;
+    for (int i = 0; i < kAcc2; ++i) acc2[i] = 0ull;
     for (int kg = 0; kg < G; ++kg, ++step) {
       const int b = step & 1;
       const uint32_t u = (uint32_t)(step >> 1);
@@ -283,43 +283,45 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
         ok = false;
         break;
       }
-      // This step's scales: one base address each, every other offset a constant.
-      const float* swb = &S.sc_w[st][32 * sub + g][gi];
-      const float* sab = &S.sc_a[st][ch * EPI_COLS + 2 * q][gi];
+      // This step's scales: one shared-memory base address each, every offset a constant.
+      const uint32_t swb = ptx::smem_addr(&S.sc_w[st][32 * sub + g][gi]);
+      const uint32_t sab = ptx::smem_addr(&S.sc_a[st][ch * EPI_COLS + 2 * q][gi]);
       uint64_t sw2[4];                               // weight scale of row (h, k), twice
 #pragma unroll
       for (int hk = 0; hk < 4; ++hk) {
-        const float sw = swb[(16 * (hk >> 1) + 8 * (hk & 1)) * SC_GROUPS];
+        const float sw = ptx::lds_f32(swb + 4 * SC_GROUPS * (16 * (hk >> 1) + 8 * (hk & 1)));
         sw2[hk] = ptx::f2_pack(sw, sw);
       }
       if (!warp_wait_or_abort(S, &S.acc_full[b], u & 1u, status)) { ok = false; break; }
       ptx::tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(b * BN + ch * EPI_COLS);
+      // 32 tokens x both lane halves per TMEM wait (4 waits per group).
 #pragma unroll
-      for (int c = 0; c < EPI_CHUNKS; ++c) {
-        uint64_t sa2[2];                             // token scales of columns 8x + 2q + {0, 1}
+      for (int cc = 0; cc < EPI_CHUNKS / 2; ++cc) {
+        uint32_t d0[16], d1[16];                     // lane halves h = 0, 1
+        ptx::tmem_ld_16x256b_x4(tbase + 32 * cc, d0);
+        ptx::tmem_ld_16x256b_x4(tbase + (16u << 16) + 32 * cc, d1);
+        uint64_t sa2[4];                             // token scales of columns 32cc + 8x + 2q + {0, 1}
 #pragma unroll
-        for (int x = 0; x < 2; ++x)
-          sa2[x] = ptx::f2_pack(sab[(16 * c + 8 * x) * SC_GROUPS], sab[(16 * c + 8 * x + 1) * SC_GROUPS]);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {                // lane half: rows 16 h + g + 8 k
-          uint32_t d[8];
-          ptx::tmem_ld_16x256b_x2(tbase + ((uint32_t)(16 * h) << 16) + 16 * c, d);
-          ptx::tmem_ld_wait(d);
-          if (c == EPI_CHUNKS - 1 && h == 1) {
-            // The whole group's tile is read: hand the buffer back to the MMA before the math.
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&S.acc_empty[b]);
-          }
-#pragma unroll
-          for (int x = 0; x < 2; ++x)
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const int i = ((h * 2 + k) * EPI_CHUNKS + c) * 4 + x * 2;
-              ptx::mul_fma2(acc[i], acc[i + 1], d[4 * x + 2 * k], d[4 * x + 2 * k + 1], sw2[h * 2 + k], sa2[x]);
-            }
+        for (int x = 0; x < 4; ++x)
+          sa2[x] = ptx::lds_pair<4 * SC_GROUPS>(sab + 4 * SC_GROUPS * (32 * cc + 8 * x));
+        const uint32_t after = ptx::tmem_ld_wait_token();
+        if (cc == EPI_CHUNKS / 2 - 1) {
+          // The whole group's tile is read: hand the buffer back to the MMA before the math.
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&S.acc_empty[b]);
         }
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int c = 2 * cc + (x >> 1);         // 16-token chunk of the accumulator layout
+            const int i0 = ((0 * 2 + k) * EPI_CHUNKS + c) * 2 + (x & 1);
+            const int i1 = ((1 * 2 + k) * EPI_CHUNKS + c) * 2 + (x & 1);
+            ptx::mul_fma2(acc2[i0], d0[4 * x + 2 * k], d0[4 * x + 2 * k + 1], sw2[0 * 2 + k], sa2[x], after);
+            ptx::mul_fma2(acc2[i1], d1[4 * x + 2 * k], d1[4 * x + 2 * k + 1], sw2[1 * 2 + k], sa2[x], after);
+          }
       }
       if (gi == SC_GROUPS - 1 || kg == G - 1) {
         __syncwarp();
@@ -348,7 +350,9 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
 #pragma unroll
           for (int hk = 0; hk < 4; ++hk) {
             if (!nin[hk]) continue;
-            const float v = acc[(hk * EPI_CHUNKS + c) * 4 + xe];   // rows 16 h + 8 k = 8 hk
+            float lo, hi;                                            // rows 16 h + 8 k = 8 hk
+            ptx::unpack2(acc2[(hk * EPI_CHUNKS + c) * 2 + (xe >> 1)], lo, hi);
+            const float v = (xe & 1) ? hi : lo;
             if (!out_bf16) reinterpret_cast<float*>(p)[8 * hk] = v;
             else reinterpret_cast<__nv_bfloat16*>(p)[8 * hk] = __float2bfloat16_rn(v);
           }

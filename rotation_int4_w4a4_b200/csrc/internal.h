@@ -14,14 +14,6 @@ namespace pq {
 constexpr int kGroup = 128;            // the only supported group size
 constexpr int kSmoothBlock = 128;      // rows per runtime-smoothing block
 
-// One Givens pair of one layer of one group, as the kernels read it (16 bytes).
-struct GivensPair {
-  uint32_t ij;   // i | j << 16  (i < j < 128)
-  float c;       // cos(theta)
-  float s;       // sin(theta)
-  uint32_t pad;
-};
-
 }  // namespace pq
 
 // Device status word bits.
@@ -35,12 +27,9 @@ struct pq_plan {
   int K;
   uint32_t flags;
   int device;
-  // Givens: pairs compacted per (group, layer): d_pairs[(gi*K + l)*64 + p], p < d_npairs[gi*K+l]
-  pq::GivensPair* d_pairs;
-  int* d_npairs;
-  int max_pairs;            // max over (group, layer) of the pair count
-  float* d_scale_act;       // [D] exp(-beta) or nullptr
-  float* d_scale_w;         // [D] exp(+beta) or nullptr
+  // Givens: tensor-core operands, bf16 [2 (activations, weights)][G][2 (hi, lo)][128 n][128 k]
+  // holding R^T of R = G_0 ... G_{K-1} diag(exp(-+beta)) per group (y = x R).
+  uint16_t* d_rot;
   unsigned int* d_status;   // device status word (PQ_DEV_* bits)
 };
 
@@ -63,9 +52,9 @@ cudaError_t launch_hadamard_rows(const pq_plan* plan, const void* X, int64_t row
 cudaError_t launch_smooth_hadamard(const pq_plan* plan, const void* X, int64_t T, int64_t ldx,
                                    uint8_t* codes, float* scales, float* smooth_out,
                                    cudaStream_t stream);
-cudaError_t launch_givens(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx,
-                          const float* post_scale, uint8_t* codes, float* scales,
-                          cudaStream_t stream);
+// y = x R per group on the tensor cores (rotate_mma.cu); weights = 0: activations, 1: weights.
+cudaError_t launch_givens_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
+                              uint8_t* codes, float* scales, cudaStream_t stream);
 pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                    const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
                    pq_out_dtype out_dtype, cudaStream_t stream);

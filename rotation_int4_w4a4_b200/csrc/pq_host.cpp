@@ -106,10 +106,7 @@ extern "C" pq_status pq_select_pairs(uint64_t seed, int D, int g, int K, int N,
 
 static void free_plan_tables(pq_plan* p) {
   if (!p) return;
-  if (p->d_pairs) cudaFree(p->d_pairs);
-  if (p->d_npairs) cudaFree(p->d_npairs);
-  if (p->d_scale_act) cudaFree(p->d_scale_act);
-  if (p->d_scale_w) cudaFree(p->d_scale_w);
+  if (p->d_rot) cudaFree(p->d_rot);
   if (p->d_status) cudaFree(p->d_status);
 }
 
@@ -129,6 +126,62 @@ static pq_status upload(T** dst, const T* src, size_t n, const char* what) {
   return cuda_fail(e, what);
 }
 
+// bf16 bit pattern of a float, round to nearest even (finite inputs).
+static uint16_t bf16_bits(float f) {
+  uint32_t b;
+  std::memcpy(&b, &f, 4);
+  return (uint16_t)((b + 0x7FFFu + ((b >> 16) & 1u)) >> 16);
+}
+
+static float bf16_value(uint16_t h) {
+  const uint32_t b = (uint32_t)h << 16;
+  float f;
+  std::memcpy(&f, &b, 4);
+  return f;
+}
+
+// Givens, tensor-core operands.  Per group, R = G_0 G_1 ... G_{K-1} in float64 for the row-vector
+// convention y = x R: layer l's pair (i, j, theta) replaces columns (i, j) of R by
+// (c col_i - s col_j, s col_i + c col_j).  Column n is then scaled by exp(-beta_n) for the
+// activations and exp(+beta_n) for the weights (R diag(exp(beta)) = M^-T, the rotations being
+// orthogonal).  Stored transposed (entry [n][k] = R[k][n]) as bf16 R_hi + R_lo.
+static void build_rotation_operands(int G, int K, const uint8_t* pairs, const float* angles, const float* beta,
+                                    std::vector<uint16_t>& out) {
+  constexpr int g = kGroup, half = kGroup / 2;
+  out.assign((size_t)2 * G * 2 * g * g, 0);
+  std::vector<double> R((size_t)g * g);
+  for (int gi = 0; gi < G; ++gi) {
+    std::fill(R.begin(), R.end(), 0.0);
+    for (int k = 0; k < g; ++k) R[(size_t)k * g + k] = 1.0;
+    for (int l = 0; l < K; ++l) {
+      for (int p = 0; p < half; ++p) {
+        const size_t slot = (size_t)(gi * K + l) * half + p;
+        const int i = pairs[2 * slot], j = pairs[2 * slot + 1];
+        if (i == PQ_NO_PAIR || j == PQ_NO_PAIR) continue;
+        const double c = std::cos((double)angles[slot]), s = std::sin((double)angles[slot]);
+        for (int r = 0; r < g; ++r) {
+          const double ri = R[(size_t)r * g + i], rj = R[(size_t)r * g + j];
+          R[(size_t)r * g + i] = c * ri - s * rj;
+          R[(size_t)r * g + j] = s * ri + c * rj;
+        }
+      }
+    }
+    for (int which = 0; which < 2; ++which) {
+      uint16_t* hi = out.data() + ((size_t)(which * G + gi) * 2 + 0) * g * g;
+      uint16_t* lo = out.data() + ((size_t)(which * G + gi) * 2 + 1) * g * g;
+      for (int n = 0; n < g; ++n) {
+        const double cs = beta ? std::exp((which == 0 ? -1.0 : 1.0) * (double)beta[gi * g + n]) : 1.0;
+        for (int k = 0; k < g; ++k) {
+          const double v = R[(size_t)k * g + n] * cs;
+          const uint16_t h = bf16_bits((float)v);
+          hi[(size_t)n * g + k] = h;
+          lo[(size_t)n * g + k] = bf16_bits((float)(v - (double)bf16_value(h)));
+        }
+      }
+    }
+  }
+}
+
 extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int K,
                                   const uint8_t* pairs, const float* angles, const float* beta,
                                   uint32_t flags) {
@@ -146,19 +199,13 @@ extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int
     return PQ_ERR_INVALID_ARG;
   }
   const int G = D / g, half = g / 2;
-  std::vector<GivensPair> table;
-  std::vector<int> npairs;
-  int max_pairs = 0;
   if (kind == PQ_GIVENS) {
     if (K < 1 || K > 64) { set_error("K=%d out of range 1..64", K); return PQ_ERR_INVALID_ARG; }
     if (!pairs || !angles) { set_error("Givens plan needs pairs and angles"); return PQ_ERR_INVALID_ARG; }
-    table.assign((size_t)G * K * half, GivensPair{0, 1.0f, 0.0f, 0});
-    npairs.assign((size_t)G * K, 0);
     std::vector<uint8_t> seen(g);
     for (int gi = 0; gi < G; ++gi) {
       for (int l = 0; l < K; ++l) {
         std::fill(seen.begin(), seen.end(), 0);
-        int n = 0;
         for (int p = 0; p < half; ++p) {
           size_t slot = (size_t)(gi * K + l) * half + p;
           uint8_t i = pairs[2 * slot], j = pairs[2 * slot + 1];
@@ -172,32 +219,16 @@ extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int
             return PQ_ERR_INVALID_ARG;
           }
           seen[i] = seen[j] = 1;
-          double th = (double)angles[slot];
-          if (!std::isfinite(th)) { set_error("non-finite angle at slot %zu", slot); return PQ_ERR_INVALID_ARG; }
-          GivensPair& e = table[(size_t)(gi * K + l) * half + n];
-          e.ij = (uint32_t)i | ((uint32_t)j << 16);
-          e.c = (float)std::cos(th);
-          e.s = (float)std::sin(th);
-          e.pad = 0;
-          ++n;
+          if (!std::isfinite(angles[slot])) { set_error("non-finite angle at slot %zu", slot); return PQ_ERR_INVALID_ARG; }
         }
-        npairs[(size_t)gi * K + l] = n;
-        if (n > max_pairs) max_pairs = n;
       }
+    }
+    if (beta) {
+      for (int c = 0; c < D; ++c)
+        if (!std::isfinite(beta[c])) { set_error("non-finite beta[%d]", c); return PQ_ERR_INVALID_ARG; }
     }
   } else {
     K = 0;
-  }
-  std::vector<float> sa, sw;
-  if (kind == PQ_GIVENS && beta) {
-    sa.resize(D);
-    sw.resize(D);
-    for (int c = 0; c < D; ++c) {
-      double b = (double)beta[c];
-      if (!std::isfinite(b)) { set_error("non-finite beta[%d]", c); return PQ_ERR_INVALID_ARG; }
-      sa[c] = (float)std::exp(-b);
-      sw[c] = (float)std::exp(b);
-    }
   }
   pq_plan* p = new (std::nothrow) pq_plan();
   if (!p) { set_error("host allocation failed"); return PQ_ERR_ALLOC; }
@@ -208,15 +239,11 @@ extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int
   p->G = G;
   p->K = K;
   p->flags = flags;
-  p->max_pairs = max_pairs;
   pq_status st = cuda_fail(cudaGetDevice(&p->device), "cudaGetDevice");
   if (st == PQ_OK && kind == PQ_GIVENS) {
-    st = upload(&p->d_pairs, table.data(), table.size(), "givens pair table");
-    if (st == PQ_OK) st = upload(&p->d_npairs, npairs.data(), npairs.size(), "givens pair counts");
-  }
-  if (st == PQ_OK && !sa.empty()) {
-    st = upload(&p->d_scale_act, sa.data(), sa.size(), "exp(-beta)");
-    if (st == PQ_OK) st = upload(&p->d_scale_w, sw.data(), sw.size(), "exp(+beta)");
+    std::vector<uint16_t> rot;
+    build_rotation_operands(G, K, pairs, angles, beta, rot);
+    st = upload(&p->d_rot, rot.data(), rot.size(), "givens tensor-core operands");
   }
   if (st == PQ_OK) st = upload<unsigned int>(&p->d_status, nullptr, 1, "status word");
   if (st != PQ_OK) {
@@ -274,7 +301,7 @@ extern "C" pq_status pq_transform_quant(const pq_plan* plan, const void* X, int6
       e = launch_hadamard_rows(plan, X, T, ldx, nullptr, nullptr, codes, scales, s);
       break;
     case PQ_GIVENS:
-      e = launch_givens(plan, X, T, ldx, plan->d_scale_act, codes, scales, s);
+      e = launch_givens_mma(plan, X, T, ldx, 0, codes, scales, s);
       break;
     case PQ_SMOOTH_HADAMARD:
       e = launch_smooth_hadamard(plan, X, T, ldx, codes, scales, smooth_out, s);
@@ -308,7 +335,7 @@ extern "C" pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t
       e = launch_hadamard_rows(plan, W, N, plan->D, nullptr, nullptr, codes_W, scales_W, s);
       break;
     case PQ_GIVENS:
-      e = launch_givens(plan, W, N, plan->D, plan->d_scale_w, codes_W, scales_W, s);
+      e = launch_givens_mma(plan, W, N, plan->D, 1, codes_W, scales_W, s);
       break;
     case PQ_SMOOTH_HADAMARD:
       if (plan->flags & PQ_FLAG_SMOOTH_AFTER_ROTATE)

@@ -135,6 +135,17 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// D (+)= A * B^T on 16-bit operands (types from the instruction descriptor), float32 accumulator.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D (+)= A * B^T on E4M3 operands with float32 accumulation in tensor memory.
 __device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -172,6 +183,38 @@ __device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t (&r)
   asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
                : "r"(taddr)
+               : "memory");
+}
+
+// Same shape, four times (32 columns): r[4x + 0..1] = lane T/4, columns 8x + 2(T%4) + 0..1;
+// r[4x + 2..3] = lane T/4 + 8 (x = 0..3).
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Waits for this thread's TMEM loads and returns a token (always 0).  Arithmetic on the loaded
+// registers takes the token as an input, so it cannot be scheduled before the wait (the
+// compiler sees the registers as defined by the load instruction itself).
+__device__ __forceinline__ uint32_t tmem_ld_wait_token() {
+  uint32_t t;
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n\tmov.u32 %0, 0;" : "=r"(t) : : "memory");
+  return t;
+}
+
+// Waits for this thread's TMEM loads, passing two 16-register destinations through the wait.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&a)[16], uint32_t (&b)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
+                 "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]), "+r"(a[15]),
+                 "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7]),
+                 "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15])
+               :
                : "memory");
 }
 
@@ -285,6 +328,35 @@ __device__ __forceinline__ void mul_fma2(float& a0, float& a1, uint32_t d0, uint
       " fma.rn.f32x2 a, d, %5, a; mov.b64 {%0, %1}, a; }"
       : "+f"(a0), "+f"(a1)
       : "r"(d0), "r"(d1), "l"(s2), "l"(t2));
+}
+
+// acc2 += (d0 * s, d1 * s) * t2 on a float32 pair held in one 64-bit register.  `after` is a
+// token from tmem_ld_wait_token: it orders this arithmetic after the wait for d0, d1.
+__device__ __forceinline__ void mul_fma2(uint64_t& acc2, uint32_t d0, uint32_t d1, uint64_t s2, uint64_t t2,
+                                         uint32_t after) {
+  asm("{ .reg .b64 d; mov.b64 d, {%1, %2}; mul.rn.f32x2 d, d, %3; fma.rn.f32x2 %0, d, %4, %0; }"
+      : "+l"(acc2)
+      : "r"(d0), "r"(d1), "l"(s2), "l"(t2), "r"(after));
+}
+
+// Two float32 values from shared memory (byte addresses a and a + stride) as one pair.
+template <int kStride>
+__device__ __forceinline__ uint64_t lds_pair(uint32_t a) {
+  uint64_t r;
+  asm volatile("{ .reg .f32 lo, hi; ld.shared.f32 lo, [%1]; ld.shared.f32 hi, [%1 + %2]; mov.b64 %0, {lo, hi}; }"
+               : "=l"(r)
+               : "r"(a), "n"(kStride));
+  return r;
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+  float r;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(r) : "r"(a));
+  return r;
+}
+
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
 
 __device__ __forceinline__ uint64_t u2_pack(uint32_t lo, uint32_t hi) {

@@ -1,0 +1,313 @@
+// Givens rotation + channel scale + INT4 quantisation on the tensor cores (sm_100a).
+//
+// ParoQuant page §2.2/§2.3: K layers of disjoint Givens pairs per 128-channel group, then the
+// channel scale exp(-beta) (activations) or exp(+beta) (weights).  Every layer and the scale are
+// linear and fixed by the plan, so per group they compose into one 128 x 128 matrix R_g and the
+// transform is y = x R_g for every row (ParoQuant page §6.4: rotation on the tensor cores).  The
+// plan stores R_g transposed (K-major for the MMA) as two bf16 terms R_hi + R_lo (R_lo carries
+// the rounding residual of R_hi, so R_hi + R_lo is R to about 2^-17 relative).  x is exact in
+// bf16 and every product is exact in the float32 accumulator, so y carries only that residual
+// and float32 summation error.
+//
+// One kernel per call, persistent, one CTA per SM.  Tiles are (128 rows, one group); each CTA
+// takes a contiguous range of tiles in group-major order so the group's operands stay resident.
+//   warp 0      TMA producer: the X tile (128 rows x 128 channels bf16, two 128-byte swizzled
+//               K-blocks) into a 3-stage ring; R_hi and R_lo of a new group into their slots.
+//   warp 1      TMEM allocator and MMA issuer: 2 terms x 2 K-blocks x 4 tcgen05.mma kind::f16
+//               (M128 N128 K16) per tile into a double-buffered float32 accumulator.
+//   warps 2..5  epilogue, one thread per row (TMEM lane): 128 values of y from tensor memory,
+//               absmax, scale = m / 7, codes = RNE(y * 7 / m), nibble-packed, stored.
+// Every mbarrier wait is bounded; a timeout sets the plan's status bit and the CTA drains.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace pq {
+namespace {
+
+constexpr int RT_M = 128;                 // rows per tile (MMA M, TMEM lanes)
+constexpr int RT_N = 128;                 // output channels (MMA N)
+constexpr int RT_KB = 64;                 // bf16 per 128-byte swizzle row (one K-block)
+constexpr int RT_STAGES = 3;
+constexpr int RT_THREADS = 192;
+constexpr uint32_t RT_TMEM_COLS = 256;    // two accumulator buffers of 128 columns
+constexpr uint64_t kRtWaitNs = 2000000000ull;
+constexpr uint32_t kTileBytes = RT_M * 128 * 2;        // one X tile: 32 KB
+constexpr uint32_t kRotBytes = 2 * RT_N * 128 * 2;     // R_hi and R_lo of one group: 64 KB
+constexpr float kRoundMagicR = 12582912.0f;            // 1.5 * 2^23
+
+struct __align__(1024) RotSmem {
+  uint8_t x[RT_STAGES][2][RT_M * 128];    // [stage][K-block][128 rows x 128 bytes]
+  uint8_t r[2][2][RT_N * 128];            // [term hi/lo][K-block][128 out channels x 128 bytes]
+  uint64_t x_full[RT_STAGES];
+  uint64_t x_empty[RT_STAGES];
+  uint64_t r_full;
+  uint64_t r_empty;
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_slot;
+  int abort_flag;
+};
+constexpr size_t kRotSmemBytes = sizeof(RotSmem) + 1024;
+static_assert(kRotSmemBytes <= 232448, "shared memory exceeds 227 KB");
+
+// D format F32 (bits 4-5 = 1), A and B BF16 (bits 7-9, 10-12 = 1), both K-major, N/8, M/16.
+constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(RT_N >> 3) << 17) |
+                                ((uint32_t)(RT_M >> 4) << 24);
+
+__device__ __forceinline__ bool rt_wait(RotSmem& S, uint64_t* bar, uint32_t parity, unsigned int* status) {
+  if (ptx::mbar_wait_bounded(bar, parity, &S.abort_flag, kRtWaitNs)) return true;
+  S.abort_flag = 1;
+  atomicOr(status, PQ_DEV_TIMEOUT);
+  return false;
+}
+
+__device__ __forceinline__ bool rt_warp_wait(RotSmem& S, uint64_t* bar, uint32_t parity, unsigned int* status) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = rt_wait(S, bar, parity, status) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
+__device__ __forceinline__ void rt_drain(uint64_t* bar, uint32_t parity) {
+  int never = 0;
+  (void)ptx::mbar_wait_bounded(bar, parity, &never, kRtWaitNs);
+}
+
+// 8 values -> 8 nibbles: byte k = q[2k] | q[2k+1] << 4, q = RNE(v * inv) (|q| <= 7).
+__device__ __forceinline__ uint32_t rt_pack8(const float* v, float inv) {
+  uint32_t b[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) b[k] = __float_as_uint(fmaf(v[k], inv, kRoundMagicR));
+  const uint32_t even = __byte_perm(__byte_perm(b[0], b[2], 0x0040), __byte_perm(b[4], b[6], 0x0040), 0x5410);
+  const uint32_t odd = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
+  return (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
+}
+
+// Tiles are numbered group-major: tile = gi * row_blocks + rb.  CTA c owns [begin, end).
+__global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
+    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmR, int64_t rows, int G,
+    int row_blocks, int64_t num_tiles, uint8_t* __restrict__ codes, float* __restrict__ scales,
+    unsigned int* status) {
+  extern __shared__ unsigned char smem_raw[];
+  RotSmem& S = *reinterpret_cast<RotSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t begin = num_tiles * blockIdx.x / gridDim.x;
+  const int64_t end = num_tiles * (blockIdx.x + 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < RT_STAGES; ++s) {
+      ptx::mbar_init(&S.x_full[s], 1);
+      ptx::mbar_init(&S.x_empty[s], 1);
+    }
+    ptx::mbar_init(&S.r_full, 1);
+    ptx::mbar_init(&S.r_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&S.acc_full[b], 1);
+      ptx::mbar_init(&S.acc_empty[b], 4);
+    }
+    ptx::mbar_init(&S.mma_done, 1);
+    S.abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tmap(&tmX);
+    ptx::prefetch_tmap(&tmR);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&S.tmem_slot, RT_TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = S.tmem_slot;
+
+  if (warp == 0) {
+    // --------------------------------------------------------------------- producer
+    if (lane == 0) {
+      int step = 0, loaded = 0;           // loaded: number of groups whose R was loaded
+      int cur_g = -1;
+      bool ok = true;
+      for (int64_t tile = begin; tile < end && ok; ++tile, ++step) {
+        const int gi = (int)(tile / row_blocks);
+        const int64_t r0 = (tile - (int64_t)gi * row_blocks) * RT_M;
+        if (gi != cur_g) {
+          // The previous group's R is free once every MMA issued for it has completed.
+          if (loaded > 0 && !rt_wait(S, &S.r_empty, (uint32_t)(loaded - 1) & 1u, status)) { ok = false; break; }
+          ptx::mbar_arrive_expect_tx(&S.r_full, kRotBytes);
+          for (int term = 0; term < 2; ++term)
+            for (int kb = 0; kb < 2; ++kb)
+              ptx::tma_load_2d(S.r[term][kb], &tmR, &S.r_full, kb * RT_KB, (gi * 2 + term) * RT_N);
+          cur_g = gi;
+          ++loaded;
+        }
+        const int s = step % RT_STAGES;
+        const uint32_t ph = (uint32_t)(step / RT_STAGES) & 1u;
+        if (!rt_wait(S, &S.x_empty[s], ph ^ 1u, status)) { ok = false; break; }
+        ptx::mbar_arrive_expect_tx(&S.x_full[s], kTileBytes);
+        for (int kb = 0; kb < 2; ++kb)
+          ptx::tma_load_2d(S.x[s][kb], &tmX, &S.x_full[s], gi * 128 + kb * RT_KB, (int)r0);
+      }
+      // Drain: every load issued lands before the CTA may exit.
+      for (int j = (step > RT_STAGES ? step - RT_STAGES : 0); j < step; ++j)
+        rt_drain(&S.x_full[j % RT_STAGES], (uint32_t)(j / RT_STAGES) & 1u);
+      if (loaded > 0) rt_drain(&S.r_full, (uint32_t)(loaded - 1) & 1u);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int step = 0, used = 0;             // used: groups whose R this thread has waited for
+      int cur_g = -1;
+      bool ok = true;
+      for (int64_t tile = begin; tile < end && ok; ++tile, ++step) {
+        const int gi = (int)(tile / row_blocks);
+        if (gi != cur_g) {
+          if (used > 0) ptx::umma_commit(&S.r_empty);   // the old R is free after these MMAs
+          if (!rt_wait(S, &S.r_full, (uint32_t)used & 1u, status)) { ok = false; break; }
+          cur_g = gi;
+          ++used;
+        }
+        const int s = step % RT_STAGES;
+        const uint32_t ph = (uint32_t)(step / RT_STAGES) & 1u;
+        const int b = step & 1;
+        const uint32_t u = (uint32_t)(step >> 1);
+        if (!rt_wait(S, &S.acc_empty[b], (u & 1u) ^ 1u, status)) { ok = false; break; }
+        if (!rt_wait(S, &S.x_full[s], ph, status)) { ok = false; break; }
+        ptx::tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)b * RT_N;
+        int n = 0;
+#pragma unroll
+        for (int term = 0; term < 2; ++term)
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+            const uint32_t a0 = ptx::smem_addr(S.x[s][kb]);
+            const uint32_t b0 = ptx::smem_addr(S.r[term][kb]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k, ++n)   // K16 per MMA = 32 bytes along the swizzled row
+              ptx::umma_f16(d, ptx::smem_desc_sw128(a0 + 32 * k), ptx::smem_desc_sw128(b0 + 32 * k), kIdescBf16,
+                            n > 0 ? 1u : 0u);
+          }
+        ptx::umma_commit(&S.x_empty[s]);
+        ptx::umma_commit(&S.acc_full[b]);
+      }
+      ptx::umma_commit(&S.mma_done);
+      rt_drain(&S.mma_done, 0);
+    }
+  } else {
+    // -------------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;         // TMEM lanes 32 quarter .. + 31
+    const int rl = quarter * 32 + lane;   // row within the tile
+    int step = 0;
+    for (int64_t tile = begin; tile < end; ++tile, ++step) {
+      const int gi = (int)(tile / row_blocks);
+      const int64_t t = (tile - (int64_t)gi * row_blocks) * RT_M + rl;
+      const int b = step & 1;
+      const uint32_t u = (uint32_t)(step >> 1);
+      if (!rt_warp_wait(S, &S.acc_full[b], u & 1u, status)) break;
+      ptx::tc_fence_after();
+      const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)b * RT_N;
+      float y[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        ptx::tmem_ld32(ta + 32 * c, r);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) y[32 * c + j] = __uint_as_float(r[j]);
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&S.acc_empty[b]);
+      float m = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) m = fmaxf(m, fabsf(y[i]));
+      const float inv = m > 0.0f ? 7.0f * __frcp_rn(m) : 0.0f;
+      if (t < rows) {
+        uint4* dst = reinterpret_cast<uint4*>(codes + t * (int64_t)G * 64 + gi * 64);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          dst[k] = make_uint4(rt_pack8(y + 32 * k, inv), rt_pack8(y + 32 * k + 8, inv),
+                              rt_pack8(y + 32 * k + 16, inv), rt_pack8(y + 32 * k + 24, inv));
+        scales[t * G + gi] = __fdiv_rn(m, 7.0f);
+      }
+    }
+  }
+
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, RT_TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFnR)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFnR encode_fn_r() {
+  static EncodeTiledFnR fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFnR>(p);
+  }
+  return fn;
+}
+
+// bf16 [rows][inner] (row stride ld elements) with a box of 64 x 128 and 128-byte swizzle.
+cudaError_t make_bf16_map(CUtensorMap* map, const void* base, int64_t rows, int64_t inner, int64_t ld) {
+  EncodeTiledFnR enc = encode_fn_r();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)RT_KB, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int rt_sm_count() {
+  int dev = 0, c = 0;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
+  return c;
+}
+
+}  // namespace
+
+cudaError_t launch_givens_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
+                              uint8_t* codes, float* scales, cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  CUtensorMap tmX, tmR;
+  cudaError_t e = make_bf16_map(&tmX, X, rows, plan->D, ldx);
+  if (e != cudaSuccess) return e;
+  const uint16_t* R = plan->d_rot + (size_t)(weights ? 1 : 0) * plan->G * 2 * RT_N * 128;
+  e = make_bf16_map(&tmR, R, (int64_t)plan->G * 2 * RT_N, 128, 128);
+  if (e != cudaSuccess) return e;
+  const int row_blocks = (int)((rows + RT_M - 1) / RT_M);
+  const int64_t tiles = (int64_t)row_blocks * plan->G;
+  const int sms = rt_sm_count();
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  e = cudaFuncSetAttribute(rotate_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRotSmemBytes);
+  if (e != cudaSuccess) return e;
+  rotate_mma_kernel<<<grid, RT_THREADS, kRotSmemBytes, stream>>>(tmX, tmR, rows, plan->G, row_blocks, tiles,
+                                                                codes, scales, plan->d_status);
+  return cudaGetLastError();
+}
+
+}  // namespace pq

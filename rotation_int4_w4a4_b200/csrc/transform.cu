@@ -121,15 +121,6 @@ __device__ __forceinline__ uint4 quant_pack32(const float (&v)[32], float inv) {
                     quant_pack8(v + 24, inv));
 }
 
-__device__ __forceinline__ void load32(const __nv_bfloat16* src, float (&v)[32]) {
-  const uint4* p = reinterpret_cast<const uint4*>(src);
-  const uint4 w0 = ld_stream(p), w1 = ld_stream(p + 1), w2 = ld_stream(p + 2), w3 = ld_stream(p + 3);
-  bf16x8_to_f32(w0, v);
-  bf16x8_to_f32(w1, v + 8);
-  bf16x8_to_f32(w2, v + 16);
-  bf16x8_to_f32(w3, v + 24);
-}
-
 __device__ __forceinline__ void scale32(float (&v)[32], const float* s) {
   const float4* p = reinterpret_cast<const float4*>(s);
 #pragma unroll
@@ -330,73 +321,6 @@ __global__ void __launch_bounds__(128) smooth_hadamard_kernel(
   }
 }
 
-// ---------------------------------------------------------------------------------------
-// Givens layers (ParoQuant page §2.2): one lane per row, the row's 128 channels of group gi
-// staged in shared memory as [channel][lane] (stride 33: conflict-free), the layer's pairs
-// read as warp-uniform broadcasts.  Then y *= post per channel, quantise, pack.
-constexpr int kGivensRows = 128;   // rows per CTA (4 warps x 32 lanes)
-
-__global__ void __launch_bounds__(128) givens_kernel(
-    const __nv_bfloat16* __restrict__ X, int64_t rows, int64_t ldx, int G, int K,
-    const GivensPair* __restrict__ pairs, const int* __restrict__ npairs,
-    const float* __restrict__ post, uint8_t* __restrict__ codes, float* __restrict__ scales) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  GivensPair* tbl = reinterpret_cast<GivensPair*>(smem_raw);
-  int* np = reinterpret_cast<int*>(tbl + K * 64);
-  float* tile = reinterpret_cast<float*>(np + ((K + 3) & ~3));
-  const int gi = blockIdx.y;
-  for (int i = threadIdx.x; i < K * 64; i += blockDim.x) tbl[i] = pairs[(size_t)gi * K * 64 + i];
-  for (int i = threadIdx.x; i < K; i += blockDim.x) np[i] = npairs[gi * K + i];
-  __syncthreads();
-
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* col = tile + w * (128 * 33) + lane;
-  const int64_t t = (int64_t)blockIdx.x * kGivensRows + w * 32 + lane;
-  if (t >= rows) return;
-  const uint4* src = reinterpret_cast<const uint4*>(X + t * ldx + gi * 128);
-#pragma unroll 4
-  for (int c16 = 0; c16 < 16; ++c16) {
-    float v[8];
-    bf16x8_to_f32(ld_stream(src + c16), v);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) col[(8 * c16 + k) * 33] = v[k];
-  }
-  for (int l = 0; l < K; ++l) {
-    const int n = np[l];
-    const GivensPair* e = tbl + l * 64;
-    for (int p = 0; p < n; ++p) {
-      const GivensPair pe = e[p];
-      const int i = pe.ij & 0xFFFF, j = pe.ij >> 16;
-      const float xi = col[i * 33], xj = col[j * 33];
-      col[i * 33] = fmaf(pe.c, xi, -pe.s * xj);
-      col[j * 33] = fmaf(pe.s, xi, pe.c * xj);
-    }
-  }
-  float m = 0.0f;
-  const float* ps = post ? post + gi * 128 : nullptr;
-  for (int c = 0; c < 128; ++c) {
-    float v = col[c * 33];
-    if (ps) {
-      v *= __ldg(ps + c);
-      col[c * 33] = v;
-    }
-    m = fmaxf(m, fabsf(v));
-  }
-  const float inv = quant_inv(m);
-  uint32_t words[16];
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    float v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = col[(8 * k + j) * 33];
-    words[k] = quant_pack8(v, inv);
-  }
-  uint4* dst = reinterpret_cast<uint4*>(codes + t * (int64_t)G * 64 + gi * 64);
-#pragma unroll
-  for (int k = 0; k < 4; ++k) dst[k] = make_uint4(words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]);
-  scales[t * G + gi] = __fdiv_rn(m, 7.0f);
-}
-
 int sm_count() {
   static int count[64] = {0};
   int dev = 0;
@@ -438,20 +362,6 @@ cudaError_t launch_smooth_hadamard(const pq_plan* plan, const void* X, int64_t T
   smooth_hadamard_kernel<<<grid, 128, 0, stream>>>(
       reinterpret_cast<const __nv_bfloat16*>(X), T, ldx, plan->G,
       (plan->flags & PQ_FLAG_SMOOTH_AFTER_ROTATE) ? 1 : 0, codes, scales, smooth_out);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_givens(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx,
-                          const float* post_scale, uint8_t* codes, float* scales,
-                          cudaStream_t stream) {
-  const size_t smem = (size_t)plan->K * 64 * sizeof(GivensPair) + ((plan->K + 3) & ~3) * sizeof(int) +
-                      (size_t)4 * 128 * 33 * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(givens_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((rows + kGivensRows - 1) / kGivensRows), (unsigned)plan->G);
-  givens_kernel<<<grid, 128, smem, stream>>>(reinterpret_cast<const __nv_bfloat16*>(X), rows, ldx,
-                                             plan->G, plan->K, plan->d_pairs, plan->d_npairs,
-                                             post_scale, codes, scales);
   return cudaGetLastError();
 }
 
