@@ -56,24 +56,30 @@ constexpr int BK = 128;          // one quantisation group = 128 bytes = one 128
 constexpr int OP_STAGES = 4;     // operand ring
 constexpr int SC_GROUPS = 4;     // groups per scale stage
 constexpr int S_STAGES = 4;      // scale ring
-constexpr int NUM_EPI_WARPS = 8;
-constexpr int EPI_WARP0 = 4;     // warps 0..3 control, 4..11 epilogue
+#ifndef PQ_GEMM_EPI_WARPS
+#define PQ_GEMM_EPI_WARPS 8
+#endif
+constexpr int NUM_EPI_WARPS = PQ_GEMM_EPI_WARPS;   // 8 or 16 (2 or 4 per TMEM lane quarter)
+constexpr int EPI_WARP0 = 4;     // warps 0..3 control, then the epilogue
 constexpr int NUM_THREADS = 32 * (EPI_WARP0 + NUM_EPI_WARPS);
-constexpr int EPI_COLS = BN / (NUM_EPI_WARPS / 4);   // tokens per epilogue warp (128)
-constexpr int EPI_CHUNKS = EPI_COLS / 16;            // 16-token TMEM loads per lane half
+constexpr int EPI_COLS = BN / (NUM_EPI_WARPS / 4);   // tokens per epilogue warp (128 or 64)
+constexpr int EPI_CHUNKS = EPI_COLS / 16;            // 16-token chunks of the accumulator layout
+constexpr int EPI_LDC = NUM_EPI_WARPS == 8 ? 32 : 16;  // tokens per TMEM load (per lane half)
+constexpr int EPI_NX = EPI_LDC / 8;                  // 16x256b repetitions per load
 constexpr int NUM_SCALE_THREADS = 64;                // warps 2 and 3
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;     // 2 s
 constexpr uint32_t kTxBytes = (BM + BN) * BK;
 // Register budget (setmaxnreg): launch allocation per thread and the control and epilogue
-// warps' shares; 128 * REG_CTRL + 256 * REG_EPI must not exceed 384 * REG_LAUNCH.
-constexpr uint32_t REG_LAUNCH = 168;
-constexpr uint32_t REG_CTRL = 56;
-constexpr uint32_t REG_EPI = 224;
+// warps' shares; 128 * REG_CTRL + 32 * NUM_EPI_WARPS * REG_EPI must not exceed
+// NUM_THREADS * REG_LAUNCH.
+constexpr uint32_t REG_LAUNCH = NUM_EPI_WARPS == 8 ? 168 : 96;
+constexpr uint32_t REG_CTRL = NUM_EPI_WARPS == 8 ? 56 : 48;
+constexpr uint32_t REG_EPI = NUM_EPI_WARPS == 8 ? 224 : 104;
 static_assert(REG_CTRL * 32 * EPI_WARP0 + REG_EPI * 32 * NUM_EPI_WARPS <= REG_LAUNCH * NUM_THREADS,
               "setmaxnreg shares exceed the launch allocation");
 static_assert(REG_LAUNCH * NUM_THREADS <= 65536, "launch register allocation exceeds the SM");
-static_assert(EPI_COLS == 128, "the epilogue below assumes 128 tokens per warp");
+static_assert(NUM_EPI_WARPS == 8 || NUM_EPI_WARPS == 16, "2 or 4 epilogue warps per lane quarter");
 
 struct __align__(1024) GemmSmem {
   uint8_t opA[OP_STAGES][BM * BK];          // weights, 16 KB per stage, 128-byte swizzle
@@ -295,28 +301,28 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
       if (!warp_wait_or_abort(S, &S.acc_full[b], u & 1u, status)) { ok = false; break; }
       ptx::tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(32 * sub) << 16) + (uint32_t)(b * BN + ch * EPI_COLS);
-      // 32 tokens x both lane halves per TMEM wait (4 waits per group).
+      // EPI_LDC tokens x both lane halves per TMEM wait.
 #pragma unroll
-      for (int cc = 0; cc < EPI_CHUNKS / 2; ++cc) {
-        uint32_t d0[16], d1[16];                     // lane halves h = 0, 1
-        ptx::tmem_ld_16x256b_x4(tbase + 32 * cc, d0);
-        ptx::tmem_ld_16x256b_x4(tbase + (16u << 16) + 32 * cc, d1);
-        uint64_t sa2[4];                             // token scales of columns 32cc + 8x + 2q + {0, 1}
+      for (int cc = 0; cc < EPI_COLS / EPI_LDC; ++cc) {
+        uint32_t d0[4 * EPI_NX], d1[4 * EPI_NX];     // lane halves h = 0, 1
+        ptx::tmem_ld_16x256b<EPI_NX>(tbase + EPI_LDC * cc, d0);
+        ptx::tmem_ld_16x256b<EPI_NX>(tbase + (16u << 16) + EPI_LDC * cc, d1);
+        uint64_t sa2[EPI_NX];                        // token scales of columns LDC cc + 8x + 2q + {0, 1}
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
-          sa2[x] = ptx::lds_pair<4 * SC_GROUPS>(sab + 4 * SC_GROUPS * (32 * cc + 8 * x));
+        for (int x = 0; x < EPI_NX; ++x)
+          sa2[x] = ptx::lds_pair<4 * SC_GROUPS>(sab + 4 * SC_GROUPS * (EPI_LDC * cc + 8 * x));
         const uint32_t after = ptx::tmem_ld_wait_token();
-        if (cc == EPI_CHUNKS / 2 - 1) {
+        if (cc == EPI_COLS / EPI_LDC - 1) {
           // The whole group's tile is read: hand the buffer back to the MMA before the math.
           ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&S.acc_empty[b]);
         }
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
+        for (int x = 0; x < EPI_NX; ++x)
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
-            const int c = 2 * cc + (x >> 1);         // 16-token chunk of the accumulator layout
+            const int c = (EPI_LDC / 16) * cc + (x >> 1);   // 16-token chunk of the accumulator layout
             const int i0 = ((0 * 2 + k) * EPI_CHUNKS + c) * 2 + (x & 1);
             const int i1 = ((1 * 2 + k) * EPI_CHUNKS + c) * 2 + (x & 1);
             ptx::mul_fma2(acc2[i0], d0[4 * x + 2 * k], d0[4 * x + 2 * k + 1], sw2[0 * 2 + k], sa2[x], after);

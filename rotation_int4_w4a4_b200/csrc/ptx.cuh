@@ -198,6 +198,13 @@ __device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)
       : "memory");
 }
 
+// 16x256b with X = 2 or 4 repetitions (16 or 32 columns), layout as above.
+template <int X>
+__device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, uint32_t (&r)[4 * X]) {
+  if constexpr (X == 2) tmem_ld_16x256b_x2(taddr, r);
+  else tmem_ld_16x256b_x4(taddr, r);
+}
+
 // Waits for this thread's TMEM loads and returns a token (always 0).  Arithmetic on the loaded
 // registers takes the token as an input, so it cannot be scheduled before the wait (the
 // compiler sees the registers as defined by the load instruction itself).
