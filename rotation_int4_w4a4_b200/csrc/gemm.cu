@@ -528,12 +528,15 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   const int64_t chunksA = T * (D / 32), chunksW = N * (D / 32);   // 16 packed bytes each
   const int64_t want = (chunksA + chunksW + 255) / 256;
   const int egrid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+  static bool attr_expand[64] = {}, attr_gemm[64] = {};
+  cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(expand_codes_kernel), 0, attr_expand);
+  if (e != cudaSuccess) return cuda_fail(e, "expand_codes_kernel attributes");
+  e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_kernel), (int)kSmemBytes, attr_gemm);
+  if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel attributes");
   expand_codes_kernel<<<egrid, 256, 0, stream>>>(codes_A, chunksA, codes_W, chunksW, A8, W8);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "expand_codes_kernel launch");
   const int grid = (int)(tiles < sms ? tiles : sms);
-  e = cudaFuncSetAttribute(w4a4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm smem)");
   // The warp roles re-divide the launch's registers with setmaxnreg; that only works when the
   // kernel was compiled with exactly the budgeted count (otherwise an increase would never be
   // granted), so refuse to launch anything else.

@@ -27,8 +27,10 @@ struct pq_plan {
   int K;
   uint32_t flags;
   int device;
-  // Givens: tensor-core operands, bf16 [2 (activations, weights)][G][2 (hi, lo)][128 n][128 k]
-  // holding R^T of R = G_0 ... G_{K-1} diag(exp(-+beta)) per group (y = x R).
+  // Tensor-core rotation operands (bf16, [n][k] = R[k][n]):
+  //   Givens:   [2 (activations, weights)][G][2 (hi, lo)][128][128] for R = G_0 ... G_{K-1}
+  //             diag(exp(-+beta)) per group (y = x R);
+  //   Hadamard: [128][128] unnormalised H_128 (also used by the smooth kinds' plans, unused there).
   uint16_t* d_rot;
   unsigned int* d_status;   // device status word (PQ_DEV_* bits)
 };
@@ -44,6 +46,24 @@ pq_status cuda_fail(cudaError_t err, const char* what);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Kernel attributes set once per device and kernel: the dynamic shared-memory limit and the
+// largest shared-memory carveout, so that consecutive kernels of this library find the SMs'
+// L1 / shared-memory split already as they need it.  `done` is the caller's per-kernel table.
+inline cudaError_t set_kernel_attributes(const void* func, int dyn_smem, bool (&done)[64]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  if (dyn_smem > 0) {
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
+    if (e != cudaSuccess) return e;
+  }
+  e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64) done[dev] = true;
+  return cudaSuccess;
+}
+
 // Kernel launchers (transform.cu, gemm.cu).  Arguments are already validated.
 // y = ((x * pre) H) * post per row-group (pre/post per channel, either may be null).
 cudaError_t launch_hadamard_rows(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx,
@@ -52,8 +72,9 @@ cudaError_t launch_hadamard_rows(const pq_plan* plan, const void* X, int64_t row
 cudaError_t launch_smooth_hadamard(const pq_plan* plan, const void* X, int64_t T, int64_t ldx,
                                    uint8_t* codes, float* scales, float* smooth_out,
                                    cudaStream_t stream);
-// y = x R per group on the tensor cores (rotate_mma.cu); weights = 0: activations, 1: weights.
-cudaError_t launch_givens_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
+// y = x R per group on the tensor cores (rotate_mma.cu) for PQ_GIVENS and PQ_HADAMARD plans;
+// weights = 0: activations, 1: weights.
+cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
                               uint8_t* codes, float* scales, cudaStream_t stream);
 pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                    const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,

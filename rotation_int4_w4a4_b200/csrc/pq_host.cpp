@@ -245,6 +245,14 @@ extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int
     build_rotation_operands(G, K, pairs, angles, beta, rot);
     st = upload(&p->d_rot, rot.data(), rot.size(), "givens tensor-core operands");
   }
+  if (st == PQ_OK && kind == PQ_HADAMARD) {
+    // Unnormalised Sylvester H_128: entry (k, n) = (-1)^popcount(k & n) (Hadamard page §2.1),
+    // symmetric, so [n][k] = [k][n]; +-1 in bf16 is 0x3F80 / 0xBF80.
+    std::vector<uint16_t> h((size_t)g * g);
+    for (int k = 0; k < g; ++k)
+      for (int n = 0; n < g; ++n) h[(size_t)n * g + k] = (__builtin_popcount(k & n) & 1) ? 0xBF80 : 0x3F80;
+    st = upload(&p->d_rot, h.data(), h.size(), "hadamard tensor-core operand");
+  }
   if (st == PQ_OK) st = upload<unsigned int>(&p->d_status, nullptr, 1, "status word");
   if (st != PQ_OK) {
     free_plan_tables(p);
@@ -298,10 +306,10 @@ extern "C" pq_status pq_transform_quant(const pq_plan* plan, const void* X, int6
   cudaError_t e = cudaSuccess;
   switch (plan->kind) {
     case PQ_HADAMARD:
-      e = launch_hadamard_rows(plan, X, T, ldx, nullptr, nullptr, codes, scales, s);
+      e = launch_rotate_mma(plan, X, T, ldx, 0, codes, scales, s);
       break;
     case PQ_GIVENS:
-      e = launch_givens_mma(plan, X, T, ldx, 0, codes, scales, s);
+      e = launch_rotate_mma(plan, X, T, ldx, 0, codes, scales, s);
       break;
     case PQ_SMOOTH_HADAMARD:
       e = launch_smooth_hadamard(plan, X, T, ldx, codes, scales, smooth_out, s);
@@ -332,10 +340,10 @@ extern "C" pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t
   cudaError_t e = cudaSuccess;
   switch (plan->kind) {
     case PQ_HADAMARD:
-      e = launch_hadamard_rows(plan, W, N, plan->D, nullptr, nullptr, codes_W, scales_W, s);
+      e = launch_rotate_mma(plan, W, N, plan->D, 1, codes_W, scales_W, s);
       break;
     case PQ_GIVENS:
-      e = launch_givens_mma(plan, W, N, plan->D, 1, codes_W, scales_W, s);
+      e = launch_rotate_mma(plan, W, N, plan->D, 1, codes_W, scales_W, s);
       break;
     case PQ_SMOOTH_HADAMARD:
       if (plan->flags & PQ_FLAG_SMOOTH_AFTER_ROTATE)

@@ -1,22 +1,25 @@
-// Givens rotation + channel scale + INT4 quantisation on the tensor cores (sm_100a).
+// Per-group rotation + INT4 quantisation on the tensor cores (sm_100a): y = x R per row and
+// 128-channel group, then scale = max|y| * scale_mult, codes = RNE(y * 7 / max|y|), nibble-packed.
 //
-// ParoQuant page §2.2/§2.3: K layers of disjoint Givens pairs per 128-channel group, then the
-// channel scale exp(-beta) (activations) or exp(+beta) (weights).  Every layer and the scale are
-// linear and fixed by the plan, so per group they compose into one 128 x 128 matrix R_g and the
-// transform is y = x R_g for every row (ParoQuant page §6.4: rotation on the tensor cores).  The
-// plan stores R_g transposed (K-major for the MMA) as two bf16 terms R_hi + R_lo (R_lo carries
-// the rounding residual of R_hi, so R_hi + R_lo is R to about 2^-17 relative).  x is exact in
-// bf16 and every product is exact in the float32 accumulator, so y carries only that residual
-// and float32 summation error.
+// Givens (ParoQuant page §2.2/§2.3): K layers of disjoint Givens pairs per group, then the channel
+// scale exp(-beta) (activations) or exp(+beta) (weights).  Every layer and the scale are linear
+// and fixed by the plan, so per group they compose into one 128 x 128 matrix R_g (ParoQuant page
+// §6.4: rotation on the tensor cores).  The plan stores R_g transposed (K-major for the MMA) as
+// two bf16 terms R_hi + R_lo (R_lo carries the rounding residual of R_hi, so R_hi + R_lo is R to
+// about 2^-17 relative).  x is exact in bf16 and every product is exact in the float32
+// accumulator, so y carries only that residual and float32 summation error.
+// Block Hadamard (Hadamard page §2.1/§6.1): R = H_128 unnormalised (+-1, exact in bf16, one
+// term, the same for every group); the 1/sqrt(128) is folded into the stored scale.
 //
 // One kernel per call, persistent, one CTA per SM.  Tiles are (128 rows, one group); each CTA
-// takes a contiguous range of tiles in group-major order so the group's operands stay resident.
+// takes a contiguous range of tiles in group-major order so the group's matrix stays resident.
 //   warp 0      TMA producer: the X tile (128 rows x 128 channels bf16, two 128-byte swizzled
-//               K-blocks) into a 3-stage ring; R_hi and R_lo of a new group into their slots.
-//   warp 1      TMEM allocator and MMA issuer: 2 terms x 2 K-blocks x 4 tcgen05.mma kind::f16
+//               K-blocks) into a 4-stage ring; the matrix terms of a new group into their slots.
+//   warp 1      TMEM allocator and MMA issuer: terms x 2 K-blocks x 4 tcgen05.mma kind::f16
 //               (M128 N128 K16) per tile into a double-buffered float32 accumulator.
-//   warps 2..5  epilogue, one thread per row (TMEM lane): 128 values of y from tensor memory,
-//               absmax, scale = m / 7, codes = RNE(y * 7 / m), nibble-packed, stored.
+//   warps 2..9  two epilogue warpgroups taking alternate tiles (one accumulator buffer each); one
+//               thread per row (TMEM lane): 128 values of y from tensor memory, absmax, quantise,
+//               pack, store.
 // Every mbarrier wait is bounded; a timeout sets the plan's status bit and the CTA drains.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -32,12 +35,12 @@ namespace {
 constexpr int RT_M = 128;                 // rows per tile (MMA M, TMEM lanes)
 constexpr int RT_N = 128;                 // output channels (MMA N)
 constexpr int RT_KB = 64;                 // bf16 per 128-byte swizzle row (one K-block)
-constexpr int RT_STAGES = 3;
-constexpr int RT_THREADS = 192;
+constexpr int RT_STAGES = 4;
+constexpr int RT_THREADS = 320;           // warps 0-1 control, 2-5 and 6-9 two epilogue warpgroups
 constexpr uint32_t RT_TMEM_COLS = 256;    // two accumulator buffers of 128 columns
 constexpr uint64_t kRtWaitNs = 2000000000ull;
 constexpr uint32_t kTileBytes = RT_M * 128 * 2;        // one X tile: 32 KB
-constexpr uint32_t kRotBytes = 2 * RT_N * 128 * 2;     // R_hi and R_lo of one group: 64 KB
+constexpr uint32_t kRotBytes = 2 * RT_N * 128 * 2;     // two terms of one matrix: 64 KB
 constexpr float kRoundMagicR = 12582912.0f;            // 1.5 * 2^23
 
 struct __align__(1024) RotSmem {
@@ -91,10 +94,12 @@ __device__ __forceinline__ uint32_t rt_pack8(const float* v, float inv) {
 }
 
 // Tiles are numbered group-major: tile = gi * row_blocks + rb.  CTA c owns [begin, end).
+// terms: 1 (R exact in bf16) or 2 (R_hi + R_lo).  r_groups: number of distinct matrices (G, or 1
+// when every group uses the same one).  scale_mult: stored scale = max|y| * scale_mult.
 __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
     const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmR, int64_t rows, int G,
-    int row_blocks, int64_t num_tiles, uint8_t* __restrict__ codes, float* __restrict__ scales,
-    unsigned int* status) {
+    int row_blocks, int64_t num_tiles, int terms, int r_groups, float scale_mult, uint8_t* __restrict__ codes,
+    float* __restrict__ scales, unsigned int* status) {
   extern __shared__ unsigned char smem_raw[];
   RotSmem& S = *reinterpret_cast<RotSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -111,7 +116,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
     ptx::mbar_init(&S.r_empty, 1);
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&S.acc_full[b], 1);
-      ptx::mbar_init(&S.acc_empty[b], 4);
+      ptx::mbar_init(&S.acc_empty[b], 4);   // the 4 warps of the warpgroup that owns buffer b
     }
     ptx::mbar_init(&S.mma_done, 1);
     S.abort_flag = 0;
@@ -133,20 +138,21 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
   if (warp == 0) {
     // --------------------------------------------------------------------- producer
     if (lane == 0) {
-      int step = 0, loaded = 0;           // loaded: number of groups whose R was loaded
-      int cur_g = -1;
+      int step = 0, loaded = 0;           // loaded: number of matrices loaded so far
+      int cur_r = -1;
       bool ok = true;
       for (int64_t tile = begin; tile < end && ok; ++tile, ++step) {
         const int gi = (int)(tile / row_blocks);
+        const int ri = r_groups > 1 ? gi : 0;
         const int64_t r0 = (tile - (int64_t)gi * row_blocks) * RT_M;
-        if (gi != cur_g) {
-          // The previous group's R is free once every MMA issued for it has completed.
+        if (ri != cur_r) {
+          // The previous matrix is free once every MMA issued with it has completed.
           if (loaded > 0 && !rt_wait(S, &S.r_empty, (uint32_t)(loaded - 1) & 1u, status)) { ok = false; break; }
-          ptx::mbar_arrive_expect_tx(&S.r_full, kRotBytes);
-          for (int term = 0; term < 2; ++term)
+          ptx::mbar_arrive_expect_tx(&S.r_full, kRotBytes / 2 * terms);
+          for (int term = 0; term < terms; ++term)
             for (int kb = 0; kb < 2; ++kb)
-              ptx::tma_load_2d(S.r[term][kb], &tmR, &S.r_full, kb * RT_KB, (gi * 2 + term) * RT_N);
-          cur_g = gi;
+              ptx::tma_load_2d(S.r[term][kb], &tmR, &S.r_full, kb * RT_KB, (ri * terms + term) * RT_N);
+          cur_r = ri;
           ++loaded;
         }
         const int s = step % RT_STAGES;
@@ -164,15 +170,16 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int step = 0, used = 0;             // used: groups whose R this thread has waited for
-      int cur_g = -1;
+      int step = 0, used = 0;             // used: matrices this thread has waited for
+      int cur_r = -1;
       bool ok = true;
       for (int64_t tile = begin; tile < end && ok; ++tile, ++step) {
         const int gi = (int)(tile / row_blocks);
-        if (gi != cur_g) {
-          if (used > 0) ptx::umma_commit(&S.r_empty);   // the old R is free after these MMAs
+        const int ri = r_groups > 1 ? gi : 0;
+        if (ri != cur_r) {
+          if (used > 0) ptx::umma_commit(&S.r_empty);   // the old matrix is free after these MMAs
           if (!rt_wait(S, &S.r_full, (uint32_t)used & 1u, status)) { ok = false; break; }
-          cur_g = gi;
+          cur_r = ri;
           ++used;
         }
         const int s = step % RT_STAGES;
@@ -184,8 +191,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
         ptx::tc_fence_after();
         const uint32_t d = tmem + (uint32_t)b * RT_N;
         int n = 0;
-#pragma unroll
-        for (int term = 0; term < 2; ++term)
+        for (int term = 0; term < terms; ++term)
 #pragma unroll
           for (int kb = 0; kb < 2; ++kb) {
             const uint32_t a0 = ptx::smem_addr(S.x[s][kb]);
@@ -203,10 +209,12 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
     }
   } else {
     // -------------------------------------------------------------------- epilogue
+    // Warpgroup wg takes the tiles of steps with step % 2 == wg, i.e. accumulator buffer wg.
+    const int wg = (warp - 2) >> 2;
     const int quarter = warp & 3;         // TMEM lanes 32 quarter .. + 31
     const int rl = quarter * 32 + lane;   // row within the tile
-    int step = 0;
-    for (int64_t tile = begin; tile < end; ++tile, ++step) {
+    int step = wg;
+    for (int64_t tile = begin + wg; tile < end; tile += 2, step += 2) {
       const int gi = (int)(tile / row_blocks);
       const int64_t t = (tile - (int64_t)gi * row_blocks) * RT_M + rl;
       const int b = step & 1;
@@ -236,7 +244,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
         for (int k = 0; k < 4; ++k)
           dst[k] = make_uint4(rt_pack8(y + 32 * k, inv), rt_pack8(y + 32 * k + 8, inv),
                               rt_pack8(y + 32 * k + 16, inv), rt_pack8(y + 32 * k + 24, inv));
-        scales[t * G + gi] = __fdiv_rn(m, 7.0f);
+        scales[t * G + gi] = m * scale_mult;
       }
     }
   }
@@ -290,23 +298,30 @@ int rt_sm_count() {
 
 }  // namespace
 
-cudaError_t launch_givens_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
+cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
                               uint8_t* codes, float* scales, cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
+  const bool givens = plan->kind == PQ_GIVENS;
+  const int terms = givens ? 2 : 1;
+  const int r_groups = givens ? plan->G : 1;
   CUtensorMap tmX, tmR;
   cudaError_t e = make_bf16_map(&tmX, X, rows, plan->D, ldx);
   if (e != cudaSuccess) return e;
-  const uint16_t* R = plan->d_rot + (size_t)(weights ? 1 : 0) * plan->G * 2 * RT_N * 128;
-  e = make_bf16_map(&tmR, R, (int64_t)plan->G * 2 * RT_N, 128, 128);
+  const uint16_t* R = plan->d_rot + (size_t)(weights && givens ? 1 : 0) * r_groups * terms * RT_N * 128;
+  e = make_bf16_map(&tmR, R, (int64_t)r_groups * terms * RT_N, 128, 128);
   if (e != cudaSuccess) return e;
   const int row_blocks = (int)((rows + RT_M - 1) / RT_M);
   const int64_t tiles = (int64_t)row_blocks * plan->G;
   const int sms = rt_sm_count();
   const int grid = (int)(tiles < sms ? tiles : sms);
-  e = cudaFuncSetAttribute(rotate_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRotSmemBytes);
+  // Givens: scale = m / 7.  Hadamard: R = H unnormalised, so y is sqrt(128) times the
+  // orthonormal rotation and scale = m / (7 sqrt(128)).
+  const float scale_mult = givens ? (1.0f / 7.0f) : 0.012626906806902634f;
+  static bool attr_done[64] = {};
+  e = set_kernel_attributes(reinterpret_cast<const void*>(rotate_mma_kernel), (int)kRotSmemBytes, attr_done);
   if (e != cudaSuccess) return e;
-  rotate_mma_kernel<<<grid, RT_THREADS, kRotSmemBytes, stream>>>(tmX, tmR, rows, plan->G, row_blocks, tiles,
-                                                                codes, scales, plan->d_status);
+  rotate_mma_kernel<<<grid, RT_THREADS, kRotSmemBytes, stream>>>(tmX, tmR, rows, plan->G, row_blocks, tiles, terms,
+                                                                r_groups, scale_mult, codes, scales, plan->d_status);
   return cudaGetLastError();
 }
 

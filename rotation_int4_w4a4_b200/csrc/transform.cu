@@ -350,6 +350,9 @@ cudaError_t launch_hadamard_rows(const pq_plan* plan, const void* X, int64_t row
   }
   const int64_t cap = (int64_t)sm_count() * per_sm;  // one resident wave, tasks strided over it
   const int grid = (int)(want < cap ? want : cap);
+  static bool attr_done[64] = {};
+  cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(hadamard_rows_kernel), 0, attr_done);
+  if (e != cudaSuccess) return e;
   hadamard_rows_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(X), rows,
                                                  ldx, plan->G, pre_scale, post_scale, codes, scales);
   return cudaGetLastError();
@@ -359,6 +362,9 @@ cudaError_t launch_smooth_hadamard(const pq_plan* plan, const void* X, int64_t T
                                    uint8_t* codes, float* scales, float* smooth_out,
                                    cudaStream_t stream) {
   dim3 grid((unsigned)((T + kSmoothBlock - 1) / kSmoothBlock), (unsigned)plan->G);
+  static bool attr_done[64] = {};
+  cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(smooth_hadamard_kernel), 0, attr_done);
+  if (e != cudaSuccess) return e;
   smooth_hadamard_kernel<<<grid, 128, 0, stream>>>(
       reinterpret_cast<const __nv_bfloat16*>(X), T, ldx, plan->G,
       (plan->flags & PQ_FLAG_SMOOTH_AFTER_ROTATE) ? 1 : 0, codes, scales, smooth_out);
