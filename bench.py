@@ -339,7 +339,7 @@ def run_ours(args, wl, rank, world, local_rank):
     ck = clocks.summary(t_roll, time.time())
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in; f32 transform; s8 MMA -> s32; f32 out",
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in; f32 transform; e4m3 MMA -> f32; f32 out",
             "data": "synthetic (seeded SplitMix64 generator)",
             "config": config_of(wl, l2_desc),
             "components": comps, "roofline": roof, "cpu_baseline": cpu,
@@ -420,6 +420,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="q_proj")
     ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--N", type=int, default=None, help="sweep workload: 4096 or 14336")
+    ap.add_argument("--kind", default=None, help="sweep workload: hadamard or givens")
     ap.add_argument("--l2", choices=["flush", "rotate"], default="flush",
                     help="cold L2 between steps: a 256 MiB write + read (default), or rotating sets "
                          "of inputs and outputs larger than twice the L2")
@@ -431,7 +433,7 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
     from rotation_int4_w4a4_b200 import inputs
-    wl = inputs.workload(args.workload, T=args.T)
+    wl = inputs.workload(args.workload, T=args.T, N=args.N, kind=args.kind)
 
     if args.impl == "reference":
         run_reference(args, wl, rank, world)

@@ -168,11 +168,34 @@ __global__ void __launch_bounds__(256) expand_codes_kernel(const uint8_t* __rest
   }
 }
 
+// Tile order.  0: weight tiles fastest.  1: token tiles fastest.  2: bands of TILE_BAND weight
+// tiles, token tiles fastest within a band.
+#ifndef PQ_TILE_ORDER
+#define PQ_TILE_ORDER 0
+#endif
+constexpr int TILE_BAND = 8;
+
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& m0, int& n0) {
+  if constexpr (PQ_TILE_ORDER == 0) {
+    m0 = (tile % m_tiles) * BM;
+    n0 = (tile / m_tiles) * BN;
+  } else if constexpr (PQ_TILE_ORDER == 1) {
+    m0 = (tile / n_tiles) * BM;
+    n0 = (tile % n_tiles) * BN;
+  } else {
+    const int per_band = TILE_BAND * n_tiles;
+    const int band = tile / per_band, r = tile - band * per_band;
+    const int rows = min(TILE_BAND, m_tiles - band * TILE_BAND);   // weight tiles in this band
+    m0 = (band * TILE_BAND + r % rows) * BM;
+    n0 = (r / rows) * BN;
+  }
+}
+
 // -------------------------------------------------------------------------- control
 __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA, const CUtensorMap& tmB,
                                             const float* __restrict__ scales_A, const float* __restrict__ scales_W,
                                             uint32_t tmem, int T, int N, int G, int scales_vec16, int m_tiles,
-                                            int num_tiles, unsigned int* status) {
+                                            int n_tiles, int num_tiles, unsigned int* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -180,7 +203,8 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
       int step = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile % m_tiles) * BM, n0 = (tile / m_tiles) * BN;
+        int m0, n0;
+        tile_coords(tile, m_tiles, n_tiles, m0, n0);
         for (int kg = 0; kg < G; ++kg, ++step) {
           const int s = step % OP_STAGES;
           const uint32_t ph = (uint32_t)(step / OP_STAGES) & 1u;
@@ -231,7 +255,8 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
     int cs = 0;                                          // scale stages filled so far
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      const int m0 = (tile % m_tiles) * BM, n0 = (tile / m_tiles) * BN;
+      int m0, n0;
+      tile_coords(tile, m_tiles, n_tiles, m0, n0);
       for (int kg0 = 0; kg0 < G; kg0 += SC_GROUPS, ++cs) {
         const int st = cs % S_STAGES;
         const uint32_t sph = (uint32_t)(cs / S_STAGES) & 1u;
@@ -265,7 +290,8 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
 // 32 sub + 16 h + g + 8 k and its tokens 128 ch + 16 c + 8 x + 2 q + e (h, k, x, e in {0, 1},
 // c in 0..7).  acc index: ((h * 2 + k) * 8 + c) * 4 + x * 2 + e.
 __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* __restrict__ Y, int T, int N,
-                                             int G, int out_bf16, int m_tiles, int num_tiles, unsigned int* status) {
+                                             int G, int out_bf16, int m_tiles, int n_tiles, int num_tiles,
+                                             unsigned int* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ew = warp - EPI_WARP0;
   const int sub = warp & 3;          // TMEM lane quarter this warp may access
@@ -274,7 +300,8 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
   int step = 0, cs = 0;
   bool ok = true;
   for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-    const int m0 = (tile % m_tiles) * BM, n0 = (tile / m_tiles) * BN;
+    int m0, n0;
+    tile_coords(tile, m_tiles, n_tiles, m0, n0);
     constexpr int kAcc2 = 4 * EPI_CHUNKS * 2;         // rows (h, k) x chunks x x; e is the pair
     static_assert(2 * kAcc2 == EPI_COLS, "4 channels x EPI_COLS / 4 tokens per thread");
     uint64_t acc2[kAcc2];                            // float32 pairs (tokens 2q, 2q + 1)
@@ -411,10 +438,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
 
   if (warp < EPI_WARP0) {
     ptx::setmaxnreg_dec<REG_CTRL>();
-    cta_control(S, tmA, tmB, scales_A, scales_W, tmem, T, N, G, scales_vec16, m_tiles, num_tiles, status);
+    cta_control(S, tmA, tmB, scales_A, scales_W, tmem, T, N, G, scales_vec16, m_tiles, n_tiles, num_tiles, status);
   } else {
     ptx::setmaxnreg_inc<REG_EPI>();
-    cta_epilogue(S, tmem, Y, T, N, G, out_bf16, m_tiles, num_tiles, status);
+    cta_epilogue(S, tmem, Y, T, N, G, out_bf16, m_tiles, n_tiles, num_tiles, status);
   }
 
   __syncwarp();

@@ -46,9 +46,8 @@ pq_status cuda_fail(cudaError_t err, const char* what);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Kernel attributes set once per device and kernel: the dynamic shared-memory limit and the
-// largest shared-memory carveout, so that consecutive kernels of this library find the SMs'
-// L1 / shared-memory split already as they need it.  `done` is the caller's per-kernel table.
+// Kernel attributes set once per device and kernel (the dynamic shared-memory limit), so that
+// launches do not repeat the driver call.  `done` is the caller's per-kernel table.
 inline cudaError_t set_kernel_attributes(const void* func, int dyn_smem, bool (&done)[64]) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -58,8 +57,6 @@ inline cudaError_t set_kernel_attributes(const void* func, int dyn_smem, bool (&
     e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
     if (e != cudaSuccess) return e;
   }
-  e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  if (e != cudaSuccess) return e;
   if (dev >= 0 && dev < 64) done[dev] = true;
   return cudaSuccess;
 }

@@ -1,0 +1,58 @@
+"""Run one workload's hot-path step a few times through the library, for profilers.
+
+    python -m rotation_int4_w4a4_b200.profile_step [--workload q_proj] [--repeat 3]
+
+Each repetition launches, in order, the activation transform (pq_transform_quant), the weight
+transform (pq_pack_weights) and the W4A4 GEMM (pq_w4a4_gemm) on the named synthetic workload,
+then checks the device status.  Nothing else runs on the GPU, so a profiler's kernel filter and
+launch skip select launches by position (e.g. -s 4 skips the first repetition of a 4-launch
+step).
+"""
+from __future__ import annotations
+
+import argparse
+
+import numpy as np
+
+
+def main() -> None:
+    import torch
+
+    from rotation_int4_w4a4_b200 import inputs, pq
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="q_proj")
+    ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--repeat", type=int, default=3)
+    args = ap.parse_args()
+    wl = inputs.workload(args.workload, T=args.T)
+    dev = torch.device("cuda")
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    X, W = bf16(wl.X), bf16(wl.W)
+    if wl.kind == "givens":
+        pairs = pq.pq_select_pairs(wl.pair_seed, wl.D, wl.g, wl.K, wl.g // 2)
+        plan = pq.Plan("givens", wl.D, K=wl.K, pairs=pairs, angles=wl.angles, beta=wl.beta)
+    else:
+        plan = pq.Plan(wl.kind, wl.D)
+    T, D, N, G = wl.T, wl.D, wl.N, wl.D // wl.g
+    ca = torch.empty((T, D // 2), dtype=torch.uint8, device=dev)
+    sa = torch.empty((T, G), dtype=torch.float32, device=dev)
+    cw = torch.empty((N, D // 2), dtype=torch.uint8, device=dev)
+    sw = torch.empty((N, G), dtype=torch.float32, device=dev)
+    Y = torch.empty((T, N), dtype=torch.float32, device=dev)
+    smooth = wl.kind == "smooth_hadamard"
+    sm = torch.empty(((T + 127) // 128, D), dtype=torch.float32, device=dev) if smooth else None
+    smooth_w = torch.ones(D, dtype=torch.float32, device=dev) if smooth else None
+    for _ in range(args.repeat):
+        pq.pq_transform_quant(plan, X, ca, sa, sm)
+        pq.pq_pack_weights(plan, W, cw, sw, smooth_w)
+        pq.pq_w4a4_gemm(ca, sa, cw, sw, Y)
+    pq.pq_check_status(plan)
+    print(f"{wl.name}: {args.repeat} steps, Y[0, :4] = {Y[0, :4].tolist()}")
+
+
+if __name__ == "__main__":
+    main()
