@@ -32,7 +32,7 @@
  *   16-byte aligned.  The library allocates no user-visible buffer.  A plan owns a few small
  *   device tables and a status word, allocated by pq_make_plan and freed by pq_destroy_plan;
  *   it is immutable after creation and may be used from several streams at once.
- *   pq_w4a4_gemm takes (T + N) * D bytes of temporary scratch per call from a library-owned,
+ *   pq_w4a4_gemm takes (T + N) * D bytes (more when split, below) of temporary scratch per call from a library-owned,
  *   stream-ordered memory pool on the current device and returns it on the same stream; the
  *   pool keeps freed memory for reuse, so it holds about the largest single call's need.
  *
@@ -161,6 +161,10 @@ pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t N, const f
  *   Y device [T][N] float32 (PQ_OUT_F32) or bf16 (PQ_OUT_BF16, RNE of the float32 result).
  *   Scales must be finite.  Every dot product fits int32 exactly (|d| <= 128*64).
  *   Returns PQ_ERR_ALLOC if the stream-ordered scratch cannot be allocated.
+ *   Few output tiles (fewer than half the SMs, e.g. decode shapes): the groups are split into
+ *   ranges of a multiple of 4 handled by different CTAs, and the float32 partial results are
+ *   added in ascending range order (4 * ranges * T * N extra scratch bytes); the result differs
+ *   from the unsplit order only by float32 rounding.
  */
 pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                        const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,

@@ -38,6 +38,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <mutex>
 
@@ -191,21 +192,38 @@ __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, 
   }
 }
 
+// Work units: an output tile and a range of groups.  With split-K (ksplit > 1) the groups of a
+// tile are divided into ranges of gs (a multiple of SC_GROUPS) and each unit writes a float32
+// partial tile; a reduction kernel then sums the ranges in ascending order.
+struct Work {
+  int m_tiles, n_tiles, num_tiles;
+  int ksplit, gs, G;
+  int units;
+};
+
+__device__ __forceinline__ void unit_coords(int u, const Work& wk, int& m0, int& n0, int& kr, int& k0, int& k1) {
+  const int tile = u / wk.ksplit;
+  kr = u - tile * wk.ksplit;
+  tile_coords(tile, wk.m_tiles, wk.n_tiles, m0, n0);
+  k0 = kr * wk.gs;
+  k1 = min(wk.G, k0 + wk.gs);
+}
+
 // -------------------------------------------------------------------------- control
 __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA, const CUtensorMap& tmB,
                                             const float* __restrict__ scales_A, const float* __restrict__ scales_W,
-                                            uint32_t tmem, int T, int N, int G, int scales_vec16, int m_tiles,
-                                            int n_tiles, int num_tiles, unsigned int* status) {
+                                            uint32_t tmem, int T, int N, int G, int scales_vec16, const Work& wk,
+                                            unsigned int* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int step = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        int m0, n0;
-        tile_coords(tile, m_tiles, n_tiles, m0, n0);
-        for (int kg = 0; kg < G; ++kg, ++step) {
+      for (int u = blockIdx.x; u < wk.units && ok; u += gridDim.x) {
+        int m0, n0, kr, k0, k1;
+        unit_coords(u, wk, m0, n0, kr, k0, k1);
+        for (int kg = k0; kg < k1; ++kg, ++step) {
           const int s = step % OP_STAGES;
           const uint32_t ph = (uint32_t)(step / OP_STAGES) & 1u;
           if (!wait_or_abort(S, &S.op_empty[s], ph ^ 1u, status)) { ok = false; break; }
@@ -224,8 +242,10 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
       constexpr uint32_t idesc = ptx::idesc_e4m3_f32(BM, BN);
       int step = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        for (int kg = 0; kg < G; ++kg, ++step) {
+      for (int u = blockIdx.x; u < wk.units && ok; u += gridDim.x) {
+        int m0, n0, kr, k0, k1;
+        unit_coords(u, wk, m0, n0, kr, k0, k1);
+        for (int kg = k0; kg < k1; ++kg, ++step) {
           const int s = step % OP_STAGES;
           const uint32_t ph = (uint32_t)(step / OP_STAGES) & 1u;
           const int b = step & 1;
@@ -254,10 +274,10 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
     const int j = threadIdx.x - 64;                      // 0..63
     int cs = 0;                                          // scale stages filled so far
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      int m0, n0;
-      tile_coords(tile, m_tiles, n_tiles, m0, n0);
-      for (int kg0 = 0; kg0 < G; kg0 += SC_GROUPS, ++cs) {
+    for (int u = blockIdx.x; u < wk.units && ok; u += gridDim.x) {
+      int m0, n0, kr, k0, k1;
+      unit_coords(u, wk, m0, n0, kr, k0, k1);
+      for (int kg0 = k0; kg0 < k1; kg0 += SC_GROUPS, ++cs) {
         const int st = cs % S_STAGES;
         const uint32_t sph = (uint32_t)(cs / S_STAGES) & 1u;
         if (!warp_wait_or_abort(S, &S.sc_empty[st], sph ^ 1u, status)) { ok = false; break; }
@@ -274,7 +294,7 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
           } else {
 #pragma unroll
             for (int e = 0; e < SC_GROUPS; ++e)
-              ptx::cp_async4(dst + e, in && kg0 + e < G ? src + e : src - kg0, in && kg0 + e < G ? 4u : 0u);
+              ptx::cp_async4(dst + e, in && kg0 + e < k1 ? src + e : src - kg0, in && kg0 + e < k1 ? 4u : 0u);
           }
         }
         ptx::cp_async_arrive_noinc(&S.sc_full[st]);
@@ -290,7 +310,7 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
 // 32 sub + 16 h + g + 8 k and its tokens 128 ch + 16 c + 8 x + 2 q + e (h, k, x, e in {0, 1},
 // c in 0..7).  acc index: ((h * 2 + k) * 8 + c) * 4 + x * 2 + e.
 __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* __restrict__ Y, int T, int N,
-                                             int G, int out_bf16, int m_tiles, int n_tiles, int num_tiles,
+                                             int G, int out_bf16, const Work& wk, float* __restrict__ ws,
                                              unsigned int* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ew = warp - EPI_WARP0;
@@ -299,19 +319,19 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
   const int g = lane >> 2, q = lane & 3;
   int step = 0, cs = 0;
   bool ok = true;
-  for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-    int m0, n0;
-    tile_coords(tile, m_tiles, n_tiles, m0, n0);
+  for (int u = blockIdx.x; u < wk.units && ok; u += gridDim.x) {
+    int m0, n0, kr, k0, k1;
+    unit_coords(u, wk, m0, n0, kr, k0, k1);
     constexpr int kAcc2 = 4 * EPI_CHUNKS * 2;         // rows (h, k) x chunks x x; e is the pair
     static_assert(2 * kAcc2 == EPI_COLS, "4 channels x EPI_COLS / 4 tokens per thread");
     uint64_t acc2[kAcc2];                            // float32 pairs (tokens 2q, 2q + 1)
 #pragma unroll
     for (int i = 0; i < kAcc2; ++i) acc2[i] = 0ull;
-    for (int kg = 0; kg < G; ++kg, ++step) {
+    for (int kg = k0; kg < k1; ++kg, ++step) {
       const int b = step & 1;
       const uint32_t u = (uint32_t)(step >> 1);
       const int st = cs % S_STAGES;
-      const int gi = kg % SC_GROUPS;
+      const int gi = (kg - k0) % SC_GROUPS;
       if (gi == 0 && !warp_wait_or_abort(S, &S.sc_full[st], (uint32_t)(cs / S_STAGES) & 1u, status)) {
         ok = false;
         break;
@@ -356,7 +376,7 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
             ptx::mul_fma2(acc2[i1], d1[4 * x + 2 * k], d1[4 * x + 2 * k + 1], sw2[1 * 2 + k], sa2[x], after);
           }
       }
-      if (gi == SC_GROUPS - 1 || kg == G - 1) {
+      if (gi == SC_GROUPS - 1 || kg == k1 - 1) {
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&S.sc_empty[st]);
         ++cs;
@@ -370,8 +390,12 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
     bool nin[4];
 #pragma unroll
     for (int hk = 0; hk < 4; ++hk) nin[hk] = nb + 8 * hk < N;
-    const size_t esz = out_bf16 ? 2 : 4;
-    char* row = reinterpret_cast<char*>(Y) + ((int64_t)tb * N + nb) * esz;
+    // Split-K: this unit's float32 partial tile goes to ws[kr]; the reduction writes Y.
+    const bool partial = wk.ksplit > 1;
+    const int bf16_out = partial ? 0 : out_bf16;
+    void* dstY = partial ? static_cast<void*>(ws + (int64_t)kr * T * N) : Y;
+    const size_t esz = bf16_out ? 2 : 4;
+    char* row = reinterpret_cast<char*>(dstY) + ((int64_t)tb * N + nb) * esz;
     const int64_t row_step = (int64_t)N * esz;
 #pragma unroll
     for (int c = 0; c < EPI_CHUNKS; ++c) {
@@ -386,7 +410,7 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
             float lo, hi;                                            // rows 16 h + 8 k = 8 hk
             ptx::unpack2(acc2[(hk * EPI_CHUNKS + c) * 2 + (xe >> 1)], lo, hi);
             const float v = (xe & 1) ? hi : lo;
-            if (!out_bf16) reinterpret_cast<float*>(p)[8 * hk] = v;
+            if (!bf16_out) reinterpret_cast<float*>(p)[8 * hk] = v;
             else reinterpret_cast<__nv_bfloat16*>(p)[8 * hk] = __float2bfloat16_rn(v);
           }
         }
@@ -399,12 +423,20 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
 __global__ void __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const float* __restrict__ scales_A, const float* __restrict__ scales_W, void* __restrict__ Y,
-    int T, int N, int G, int scales_vec16, int out_bf16, int m_tiles, int n_tiles, unsigned int* status) {
+    int T, int N, int G, int scales_vec16, int out_bf16, int m_tiles, int n_tiles, int ksplit, int gs,
+    float* __restrict__ ws, unsigned int* status) {
   extern __shared__ unsigned char smem_raw[];
   GemmSmem& S = *reinterpret_cast<GemmSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int num_tiles = m_tiles * n_tiles;
+  Work wk;
+  wk.m_tiles = m_tiles;
+  wk.n_tiles = n_tiles;
+  wk.num_tiles = m_tiles * n_tiles;
+  wk.ksplit = ksplit;
+  wk.gs = gs;
+  wk.G = G;
+  wk.units = wk.num_tiles * ksplit;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < OP_STAGES; ++s) {
@@ -438,10 +470,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
 
   if (warp < EPI_WARP0) {
     ptx::setmaxnreg_dec<REG_CTRL>();
-    cta_control(S, tmA, tmB, scales_A, scales_W, tmem, T, N, G, scales_vec16, m_tiles, n_tiles, num_tiles, status);
+    cta_control(S, tmA, tmB, scales_A, scales_W, tmem, T, N, G, scales_vec16, wk, status);
   } else {
     ptx::setmaxnreg_inc<REG_EPI>();
-    cta_epilogue(S, tmem, Y, T, N, G, out_bf16, m_tiles, n_tiles, num_tiles, status);
+    cta_epilogue(S, tmem, Y, T, N, G, out_bf16, wk, ws, status);
   }
 
   __syncwarp();
@@ -450,6 +482,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Split-K reduction: Y = sum over kr of ws[kr] (ascending), float32 or bf16 (RNE) out.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __restrict__ ws, int ksplit, int64_t n4,
+                                                            void* __restrict__ Y, int out_bf16) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    float4 a = ws[i];
+    for (int kr = 1; kr < ksplit; ++kr) {
+      const float4 b = ws[(int64_t)kr * n4 + i];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    if (!out_bf16) {
+      reinterpret_cast<float4*>(Y)[i] = a;
+    } else {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+      reinterpret_cast<uint2*>(Y)[i] =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+    }
   }
 }
 
@@ -533,9 +588,29 @@ int device_sm_count() {
 
 size_t gemm_scratch_bytes(int64_t T, int64_t N, int64_t D) { return (size_t)(T + N) * (size_t)D; }
 
+int gemm_ksplit(int64_t T, int64_t N, int64_t D, int* gs_out) {
+  const int G = (int)(D / 128);
+  const int64_t tiles = ((N + BM - 1) / BM) * ((T + BN - 1) / BN);
+  const int sms = device_sm_count();
+  int ks = 1, gs = G;
+  if (G >= 2 * SC_GROUPS && tiles * 2 <= sms) {
+    const int want = (int)std::min<int64_t>(sms / tiles, G / SC_GROUPS);
+    gs = ((G + want - 1) / want + SC_GROUPS - 1) / SC_GROUPS * SC_GROUPS;   // multiple of 4 groups
+    ks = (G + gs - 1) / gs;
+    if (ks < 2) { ks = 1; gs = G; }
+  }
+  if (gs_out) *gs_out = gs;
+  return ks;
+}
+
+size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t D) {
+  const int ks = gemm_ksplit(T, N, D, nullptr);
+  return ks > 1 ? (size_t)ks * (size_t)T * (size_t)N * sizeof(float) : 0;
+}
+
 pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W, const float* scales_W,
                       int64_t T, int64_t N, int64_t D, void* Y, pq_out_dtype out_dtype, uint8_t* scratch,
-                      unsigned int* status, cudaStream_t stream) {
+                      float* ws, unsigned int* status, cudaStream_t stream) {
   uint8_t* A8 = scratch;
   uint8_t* W8 = scratch + (size_t)T * (size_t)D;
   // MMA operand A = weights (M = output channels), B = activations (N = tokens).
@@ -563,7 +638,10 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   expand_codes_kernel<<<egrid, 256, 0, stream>>>(codes_A, chunksA, codes_W, chunksW, A8, W8);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "expand_codes_kernel launch");
-  const int grid = (int)(tiles < sms ? tiles : sms);
+  int gs = (int)(D / 128);
+  const int ksplit = ws ? gemm_ksplit(T, N, D, &gs) : 1;
+  const int64_t units = tiles * ksplit;
+  const int grid = (int)(units < sms ? units : sms);
   // The warp roles re-divide the launch's registers with setmaxnreg; that only works when the
   // kernel was compiled with exactly the budgeted count (otherwise an increase would never be
   // granted), so refuse to launch anything else.
@@ -582,8 +660,19 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   const int scales_vec16 = (G % SC_GROUPS == 0) ? 1 : 0;   // rows of 16-byte multiples
   w4a4_gemm_kernel<<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB, scales_A, scales_W, Y, (int)T, (int)N,
                                                                G, scales_vec16, out_dtype == PQ_OUT_BF16 ? 1 : 0,
-                                                               m_tiles, n_tiles, status);
-  return cuda_fail(cudaGetLastError(), "w4a4_gemm_kernel launch");
+                                                               m_tiles, n_tiles, ksplit, gs, ws, status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel launch");
+  if (ksplit > 1) {
+    const int64_t n4 = T * N / 4;                              // N % 16 == 0
+    const int64_t rwant = (n4 + 255) / 256;
+    const int rgrid = (int)(rwant < (int64_t)sms * 8 ? rwant : (int64_t)sms * 8);
+    splitk_reduce_kernel<<<rgrid, 256, 0, stream>>>(reinterpret_cast<const float4*>(ws), ksplit, n4, Y,
+                                                    out_dtype == PQ_OUT_BF16 ? 1 : 0);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "splitk_reduce_kernel launch");
+  }
+  return PQ_OK;
 }
 
 pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W, const float* scales_W,
@@ -596,15 +685,18 @@ pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t*
   cudaMemPool_t pool = nullptr;
   e = scratch_pool(&pool);
   if (e != cudaSuccess) return cuda_fail(e, "scratch memory pool");
+  // Operand scratch, then (small problems) the split-K partial tiles.
+  const size_t op_bytes = (gemm_scratch_bytes(T, N, D) + 255) & ~(size_t)255;
+  const size_t ws_bytes = gemm_workspace_bytes(T, N, D);
   void* scratch = nullptr;
-  e = cudaMallocFromPoolAsync(&scratch, gemm_scratch_bytes(T, N, D), pool, stream);
+  e = cudaMallocFromPoolAsync(&scratch, op_bytes + ws_bytes, pool, stream);
   if (e != cudaSuccess) {
-    set_error("cudaMallocFromPoolAsync(%zu bytes of GEMM scratch): %s", gemm_scratch_bytes(T, N, D),
-              cudaGetErrorString(e));
+    set_error("cudaMallocFromPoolAsync(%zu bytes of GEMM scratch): %s", op_bytes + ws_bytes, cudaGetErrorString(e));
     return PQ_ERR_ALLOC;
   }
+  float* ws = ws_bytes ? reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + op_bytes) : nullptr;
   pq_status st = gemm_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype,
-                             static_cast<uint8_t*>(scratch), status, stream);
+                             static_cast<uint8_t*>(scratch), ws, status, stream);
   e = cudaFreeAsync(scratch, stream);
   if (st == PQ_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(gemm scratch)");
   return st;

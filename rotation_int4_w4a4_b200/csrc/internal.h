@@ -78,10 +78,15 @@ pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t*
                    pq_out_dtype out_dtype, cudaStream_t stream);
 // Bytes of int8 operand scratch the GEMM needs: (T + N) * D.
 size_t gemm_scratch_bytes(int64_t T, int64_t N, int64_t D);
-// Expansion + contraction launches on `stream` using caller-provided scratch.
+// Split-K factor for a problem (1 = none) and the groups per range; the float32 partial-tile
+// workspace it needs (0 when unsplit).
+int gemm_ksplit(int64_t T, int64_t N, int64_t D, int* gs_out);
+size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t D);
+// Expansion + contraction (+ split-K reduction) launches on `stream` using caller-provided
+// scratch; ws = nullptr disables split-K.
 pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                       const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
-                      pq_out_dtype out_dtype, uint8_t* scratch, unsigned int* status,
+                      pq_out_dtype out_dtype, uint8_t* scratch, float* ws, unsigned int* status,
                       cudaStream_t stream);
 pq_status gemm_read_and_clear_status(unsigned int* bits);
 // Device address of the GEMM's status word on the current device.

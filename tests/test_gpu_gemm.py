@@ -77,6 +77,23 @@ def test_random_codes_bf16(pq):
     assert np.all(np.abs(Y - ref) <= ulp)
 
 
+@pytest.mark.parametrize("T,N,D,out", [(1, 4096, 4096, "f32"), (16, 512, 2048, "bf16"),
+                                       (256, 1024, 4096, "f32"), (3, 4096, 1024, "bf16")])
+def test_split_k_small_T(pq, T, N, D, out):
+    """Few output tiles: the groups are split across CTAs and the float32 partial tiles are
+    reduced in ascending order; same tolerances as the unsplit path."""
+    ca, sa = inputs.random_codes(41 + T, T, D)
+    cw, sw = inputs.random_codes(43 + N, N, D)
+    Y = run_gemm(pq, ca, sa, cw, sw, out=out)
+    r = oracle.gemm(ca, sa, cw, sw)
+    if out == "f32":
+        assert rel_fro(Y, r.y64) < 1e-5
+    else:
+        ref = oracle.bf16_round(r.y32)
+        ulp = np.maximum(np.abs(ref), 2.0 ** -126) * 2.0 ** -7
+        assert np.all(np.abs(Y - ref) <= ulp)
+
+
 def test_oracle_codes_end_to_end_tiny(pq):
     """The tiny Givens workload: the oracle's own activation and weight codes through the GPU GEMM."""
     wl = inputs.workload("tiny")
