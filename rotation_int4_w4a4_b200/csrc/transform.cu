@@ -204,7 +204,9 @@ __global__ void __launch_bounds__(256) hadamard_rows_kernel(
 // (warp w, slot = lane/4, q = lane%4) holds rows 32k + 8w + slot (k = 0..3), channels 32q..+31.
 // after_rotate = false: s = max|x| per channel over the tile's rows, y = (x / s) H.
 // after_rotate = true:  s = max|x H| per channel (rotated channels), y = (x H) / s.
-__global__ void __launch_bounds__(128) smooth_hadamard_kernel(
+// Four CTAs per SM (128 registers per thread): the kernel is latency-bound, and the extra
+// resident tiles outweigh a few spilled registers (measured on down_proj: 217 -> 172 us).
+__global__ void __launch_bounds__(128, 4) smooth_hadamard_kernel(
     const __nv_bfloat16* __restrict__ X, int64_t T, int64_t ldx, int G, int after_rotate,
     uint8_t* __restrict__ codes, float* __restrict__ scales, float* __restrict__ smooth_out) {
   __shared__ __align__(16) float red[4][4][32];
