@@ -169,27 +169,12 @@ __global__ void __launch_bounds__(256) expand_codes_kernel(const uint8_t* __rest
   }
 }
 
-// Tile order.  0: weight tiles fastest.  1: token tiles fastest.  2: bands of TILE_BAND weight
-// tiles, token tiles fastest within a band.
-#ifndef PQ_TILE_ORDER
-#define PQ_TILE_ORDER 0
-#endif
-constexpr int TILE_BAND = 8;
-
+// Tile order: weight tiles fastest, so the CTAs running at the same time share a token tile.
+// (Token-fastest and banded orders were measured no faster.)
 __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& m0, int& n0) {
-  if constexpr (PQ_TILE_ORDER == 0) {
-    m0 = (tile % m_tiles) * BM;
-    n0 = (tile / m_tiles) * BN;
-  } else if constexpr (PQ_TILE_ORDER == 1) {
-    m0 = (tile / n_tiles) * BM;
-    n0 = (tile % n_tiles) * BN;
-  } else {
-    const int per_band = TILE_BAND * n_tiles;
-    const int band = tile / per_band, r = tile - band * per_band;
-    const int rows = min(TILE_BAND, m_tiles - band * TILE_BAND);   // weight tiles in this band
-    m0 = (band * TILE_BAND + r % rows) * BM;
-    n0 = (r / rows) * BN;
-  }
+  (void)n_tiles;
+  m0 = (tile % m_tiles) * BM;
+  n0 = (tile / m_tiles) * BN;
 }
 
 // Work units: an output tile and a range of groups.  With split-K (ksplit > 1) the groups of a

@@ -90,10 +90,6 @@ __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // ------------------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* slot_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot_smem)),
@@ -115,17 +111,6 @@ __device__ __forceinline__ void tc_fence_before() {
 
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, int8 x int8 -> int32.
-__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
 }
 
 // Instruction descriptor for kind::f8f6f4 with E4M3 A and B, float32 accumulator, both operands
@@ -162,18 +147,6 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_addr(bar))
                : "memory");
-}
-
-// 32 lanes x 32 bit, 16 consecutive columns: thread i of the warp gets lane (base + i).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
 }
 
 // 16 lanes x 256 bit, twice (16 columns): thread T receives r[4x + 0..1] = lane T/4, columns
@@ -214,27 +187,6 @@ __device__ __forceinline__ uint32_t tmem_ld_wait_token() {
   return t;
 }
 
-// Waits for this thread's TMEM loads, passing two 16-register destinations through the wait.
-__device__ __forceinline__ void tmem_ld_wait(uint32_t (&a)[16], uint32_t (&b)[16]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
-                 "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]), "+r"(a[15]),
-                 "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7]),
-                 "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15])
-               :
-               : "memory");
-}
-
-// Waits for this thread's TMEM loads and passes the 8 destination registers through the wait,
-// so that no use of them can be scheduled between the load and its completion (the compiler
-// sees the registers as defined by the load instruction itself).
-__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[8]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7])
-               :
-               : "memory");
-}
-
 // 32 lanes x 32 bit, 32 consecutive columns.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -251,33 +203,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Store the same 32-bit value into 16 consecutive columns of the warp's 32 lanes.
-__device__ __forceinline__ void tmem_st16_fill(uint32_t taddr, uint32_t v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
-      "r"(v)
-      : "memory");
-}
-
-// Store the same 32-bit value into 4 consecutive columns of the warp's 32 lanes (needs only 4
-// live copies of the value).
-__device__ __forceinline__ void tmem_st4_fill(uint32_t taddr, uint32_t v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %1, %1, %1};" ::"r"(taddr), "r"(v) : "memory");
-}
-
-// Store the same 32-bit value into 32 consecutive columns of the warp's 32 lanes.
-__device__ __forceinline__ void tmem_st32_fill(uint32_t taddr, uint32_t v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {"
-      "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
-      "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
-      "r"(v)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
 // ------------------------------------------------------------------------ descriptors
 // Shared-memory matrix descriptor (tcgen05 format): K-major operand in the 128-byte swizzle
 // layout (8-row x 128-byte atoms, atoms 1024 bytes apart); start address >> 4 in bits 0..13,
@@ -291,12 +216,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;
-}
-
-// Instruction descriptor, kind::i8: D int32 (bits 4..5 = 2), A and B signed int8 (bits 7..9 and
-// 10..12 = 1), both K-major, N >> 3 in bits 17..22, M >> 4 in bits 24..28.
-__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
-  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // -------------------------------------------------------------- cp.async (4-byte, zero-fill)
@@ -366,11 +285,6 @@ __device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
 
-__device__ __forceinline__ uint64_t u2_pack(uint32_t lo, uint32_t hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
-  return r;
-}
 __device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
@@ -384,39 +298,10 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t r;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
   return r;
-}
-
-// Four columns k of one accumulator row, two f32x2 FMAs per column pair:
-//   u_k = fma(bits(r_k), sw, csw)   with csw = -(1.5*2^23)*sw exact  ->  u_k = fl(d_k * sw)
-//   a_k = fma(u_k, s_k, a_k)
-// r_k are raw TMEM words holding 1.5*2^23 + d_k (an exact float); sw2/csw2 hold the row's
-// scale pair, s = (s0, s1, s2, s3) the four column scales.
-__device__ __forceinline__ void epi_fma4(float& a0, float& a1, float& a2, float& a3, float4 s, uint64_t sw2,
-                                         uint64_t csw2, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
-  asm("{\n\t.reg .b64 s01, s23, q01, q23, c01, c23;\n\t"
-      "mov.b64 q01, {%8, %9};\n\t"
-      "mov.b64 q23, {%10, %11};\n\t"
-      "fma.rn.f32x2 q01, q01, %12, %13;\n\t"
-      "fma.rn.f32x2 q23, q23, %12, %13;\n\t"
-      "mov.b64 s01, {%4, %5};\n\t"
-      "mov.b64 s23, {%6, %7};\n\t"
-      "mov.b64 c01, {%0, %1};\n\t"
-      "mov.b64 c23, {%2, %3};\n\t"
-      "fma.rn.f32x2 c01, q01, s01, c01;\n\t"
-      "fma.rn.f32x2 c23, q23, s23, c23;\n\t"
-      "mov.b64 {%0, %1}, c01;\n\t"
-      "mov.b64 {%2, %3}, c23;\n\t}"
-      : "+f"(a0), "+f"(a1), "+f"(a2), "+f"(a3)
-      : "f"(s.x), "f"(s.y), "f"(s.z), "f"(s.w), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "l"(sw2), "l"(csw2));
 }
 
 // -------------------------------------------------------------------- register budget
