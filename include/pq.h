@@ -203,6 +203,16 @@ pq_status pq_w4a4_gemm_noalloc(const uint8_t* codes_A, const float* scales_A,
  */
 pq_status pq_check_status(const pq_plan* plan, void* stream);
 
+/*
+ * pq_selftest_wait_timeout — diagnostic, no counterpart in the pages.  Launches on `stream` one
+ * thread that waits on a shared-memory barrier nothing will complete, using the same bounded
+ * wait as every pipeline barrier of the library's kernels; after limit_ns (1 us .. 100 ms,
+ * else PQ_ERR_INVALID_ARG) it gives up and sets the GEMM status word, so the next
+ * pq_check_status returns PQ_ERR_TIMEOUT (and clears it).  Nothing faults or traps; the
+ * context stays usable.
+ */
+pq_status pq_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
 /* Static description of a status code. */
 const char* pq_status_string(pq_status status);
 

@@ -493,6 +493,18 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __rest
   }
 }
 
+// Diagnostic: one thread waits on an mbarrier that never completes, with the same bounded
+// wait every pipeline barrier above uses; when it gives up it sets the GEMM status word.
+__global__ void wait_timeout_kernel(uint64_t limit_ns, unsigned int* status) {
+  __shared__ uint64_t bar;
+  __shared__ int never;
+  if (threadIdx.x != 0) return;
+  never = 0;
+  ptx::mbar_init(&bar, 1);
+  ptx::fence_mbar_init();
+  if (!ptx::mbar_wait_bounded(&bar, 0, &never, limit_ns)) atomicOr(status, PQ_DEV_TIMEOUT);
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
@@ -685,6 +697,14 @@ pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t*
   e = cudaFreeAsync(scratch, stream);
   if (st == PQ_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(gemm scratch)");
   return st;
+}
+
+pq_status gemm_wait_timeout_selftest(uint64_t limit_ns, cudaStream_t stream) {
+  unsigned int* status = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_gemm_status);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(gemm status)");
+  wait_timeout_kernel<<<1, 32, 0, stream>>>(limit_ns, status);
+  return cuda_fail(cudaGetLastError(), "wait_timeout_kernel launch");
 }
 
 cudaError_t gemm_status_address(unsigned int** status) {

@@ -89,6 +89,8 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
                       pq_out_dtype out_dtype, uint8_t* scratch, float* ws, unsigned int* status,
                       cudaStream_t stream);
 pq_status gemm_read_and_clear_status(unsigned int* bits);
+// Launches the bounded-wait diagnostic (a wait that cannot complete, limited to limit_ns).
+pq_status gemm_wait_timeout_selftest(uint64_t limit_ns, cudaStream_t stream);
 // Device address of the GEMM's status word on the current device.
 cudaError_t gemm_status_address(unsigned int** status);
 // gemm_launch with the fixed device-array scratch of gemm_static_scratch.cu (no allocation).

@@ -406,6 +406,15 @@ extern "C" pq_status pq_w4a4_gemm_noalloc(const uint8_t* codes_A, const float* s
                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
+extern "C" pq_status pq_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  clear_error();
+  if (limit_ns < 1000 || limit_ns > 100000000) {
+    set_error("limit_ns=%llu must be within [1 us, 100 ms]", (unsigned long long)limit_ns);
+    return PQ_ERR_INVALID_ARG;
+  }
+  return gemm_wait_timeout_selftest(limit_ns, reinterpret_cast<cudaStream_t>(stream));
+}
+
 extern "C" pq_status pq_check_status(const pq_plan* plan, void* stream) {
   clear_error();
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -27,7 +27,7 @@ KINDS = {"hadamard": PQ_HADAMARD, "givens": PQ_GIVENS, "smooth_hadamard": PQ_SMO
 # Every symbol the header declares.
 EXPORTS = ("pq_select_pairs", "pq_make_plan", "pq_destroy_plan", "pq_transform_quant",
            "pq_pack_weights", "pq_w4a4_gemm", "pq_w4a4_gemm_noalloc", "pq_check_status",
-           "pq_status_string", "pq_last_error")
+           "pq_selftest_wait_timeout", "pq_status_string", "pq_last_error")
 
 _c = ctypes
 _vp, _i64, _u64, _i32, _u32 = _c.c_void_p, _c.c_int64, _c.c_uint64, _c.c_int, _c.c_uint32
@@ -45,6 +45,8 @@ lib.pq_w4a4_gemm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _i
 lib.pq_w4a4_gemm.restype = _i32
 lib.pq_w4a4_gemm_noalloc.argtypes = lib.pq_w4a4_gemm.argtypes
 lib.pq_w4a4_gemm_noalloc.restype = _i32
+lib.pq_selftest_wait_timeout.argtypes = [_u64, _vp]
+lib.pq_selftest_wait_timeout.restype = _i32
 lib.pq_check_status.argtypes = [_vp, _vp]
 lib.pq_check_status.restype = _i32
 lib.pq_status_string.argtypes = [_i32]
@@ -177,6 +179,11 @@ def pq_w4a4_gemm_noalloc(codes_A, scales_A, codes_W, scales_W, Y, T=None, N=None
     _check(lib.pq_w4a4_gemm_noalloc(_ptr(codes_A), _ptr(scales_A), _ptr(codes_W), _ptr(scales_W),
                                     T, N, D, g, _ptr(Y), out_dtype, _stream(stream)),
            "pq_w4a4_gemm_noalloc")
+
+
+def pq_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Launch the bounded-wait diagnostic; the next pq_check_status reports PQ_ERR_TIMEOUT."""
+    _check(lib.pq_selftest_wait_timeout(limit_ns, _stream(stream)), "pq_selftest_wait_timeout")
 
 
 def pq_check_status(plan: Plan | None = None, stream=None) -> int:

@@ -106,6 +106,22 @@ def test_oracle_codes_end_to_end_tiny(pq):
     assert rel_fro(Y, ref.y64) < 1e-5
 
 
+@pytest.mark.parametrize("T,N", [(1, 14336), (16, 4096), (4096, 14336)])
+def test_sweep_shapes_sampled(pq, T, N):
+    """Decode/prefill sweep shapes at D = 4096 (split and unsplit launches), sampled rows."""
+    import torch
+    D = 4096
+    ca, sa = inputs.random_codes(3000 + T, T, D)
+    cw, sw = inputs.random_codes(4000 + N, N, D)
+    Y = torch.empty((T, N), dtype=torch.float32, device="cuda")
+    pq.pq_w4a4_gemm(to_dev(ca), to_dev(sa), to_dev(cw), to_dev(sw), Y)
+    pq.pq_check_status()
+    rows = np.unique(np.array([0, T // 2, T - 1]))
+    Ys = Y[torch.from_numpy(rows).cuda()].cpu().numpy()
+    ref = oracle.gemm(ca[rows], sa[rows], cw, sw)
+    assert rel_fro(Ys, ref.y64) < 1e-5
+
+
 @pytest.mark.parametrize("name", ["q_proj", "up_proj", "down_proj"])
 def test_full_size_sampled_rows(pq, name):
     """The full workload shapes in the launch configuration the benchmark uses, checked on a

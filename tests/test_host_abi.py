@@ -94,3 +94,11 @@ def test_gemm_and_transform_validation(pq):
     assert L.pq_transform_quant(None, p, 4, 128, p, p, None, None) == pq.PQ_ERR_INVALID_ARG
     assert L.pq_pack_weights(None, p, 4, None, p, p, None) == pq.PQ_ERR_INVALID_ARG
     L.pq_destroy_plan(None)                              # no-op
+
+
+def test_selftest_wait_timeout_validation(pq):
+    """The limit is checked before anything is launched (runs without a GPU)."""
+    for bad in (0, 999, 100_000_001):
+        assert pq.lib.pq_selftest_wait_timeout(bad, None) == pq.PQ_ERR_INVALID_ARG
+        assert b"limit_ns" in pq.lib.pq_last_error()
+
