@@ -187,8 +187,16 @@ def job_value(world, tokens_per_rank_step, steps, total_ms):
     return world * tokens_per_rank_step * steps / (total_ms * 1e-3)
 
 
-# Kernels one step launches: transform_quant, pack_weights, int4 -> int8 expansion, GEMM.
+# Kernels one step launches: transform_quant, pack_weights, int4 -> E4M3 expansion, GEMM; plus
+# the split-K reduction when the GEMM has fewer 128 x 256 output tiles than half the SMs and at
+# least 8 groups (the library's rule for splitting the group range).
 LAUNCHES_PER_STEP = 4
+
+
+def launches_per_step(T, N, D, sms):
+    tiles = -(-N // 128) * -(-T // 256)
+    split = D // 128 >= 8 and 2 * tiles <= sms and min(sms // tiles, D // 512) >= 2
+    return LAUNCHES_PER_STEP + (1 if split else 0)
 
 
 # ------------------------------------------------------------------------ GPU arm
@@ -345,7 +353,7 @@ def run_ours(args, wl, rank, world, local_rank):
             "components": comps, "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": job_value(world, wl.T, 1, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": ck, "wall_s_timed_region": w1 - w0}
+            "gpu_launches": launches_per_step(wl.T, wl.N, wl.D, torch.cuda.get_device_properties(dev).multi_processor_count) * args.steps, "clocks": ck, "wall_s_timed_region": w1 - w0}
     print(json.dumps(line), flush=True)
 
 

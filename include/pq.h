@@ -32,9 +32,10 @@
  *   16-byte aligned.  The library allocates no user-visible buffer.  A plan owns a few small
  *   device tables and a status word, allocated by pq_make_plan and freed by pq_destroy_plan;
  *   it is immutable after creation and may be used from several streams at once.
- *   pq_w4a4_gemm takes (T + N) * D bytes (more when split, below) of temporary scratch per call from a library-owned,
- *   stream-ordered memory pool on the current device and returns it on the same stream; the
- *   pool keeps freed memory for reuse, so it holds about the largest single call's need.
+ *   pq_w4a4_gemm takes (T + N) * D bytes (more when split, see there) of temporary scratch per
+ *   call from a library-owned, stream-ordered memory pool on the current device and returns it
+ *   on the same stream; the pool keeps freed memory for reuse, so it holds about the largest
+ *   single call's need.
  *
  * Errors
  *   Every call returns pq_status and never throws, aborts or exits.  Arguments are validated
