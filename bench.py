@@ -194,8 +194,10 @@ LAUNCHES_PER_STEP = 4
 
 
 def launches_per_step(T, N, D, sms):
-    tiles = -(-N // 128) * -(-T // 256)
-    split = D // 128 >= 8 and 2 * tiles <= sms and min(sms // tiles, D // 512) >= 2
+    # the GEMM's tiles are 256 channels x 256 tokens, one per CTA pair (sms // 2 pairs)
+    tiles = -(-N // 256) * -(-T // 256)
+    pairs = sms // 2
+    split = D // 128 >= 8 and 2 * tiles <= pairs and min(pairs // tiles, D // 512) >= 2
     return LAUNCHES_PER_STEP + (1 if split else 0)
 
 

@@ -162,8 +162,9 @@ pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t N, const f
  *   Y device [T][N] float32 (PQ_OUT_F32) or bf16 (PQ_OUT_BF16, RNE of the float32 result).
  *   Scales must be finite.  Every dot product fits int32 exactly (|d| <= 128*64).
  *   Returns PQ_ERR_ALLOC if the stream-ordered scratch cannot be allocated.
- *   Few output tiles (fewer than half the SMs, e.g. decode shapes): the groups are split into
- *   ranges of a multiple of 4 handled by different CTAs, and the float32 partial results are
+ *   Output tiles are 256 channels x 256 tokens, one per pair of SMs.  Few tiles (at most half
+ *   the SM pairs, e.g. decode shapes): the groups are split into ranges of a multiple of 4
+ *   handled by different SM pairs, and the float32 partial results are
  *   added in ascending range order (4 * ranges * T * N extra scratch bytes); the result differs
  *   from the unsplit order only by float32 rounding.
  */

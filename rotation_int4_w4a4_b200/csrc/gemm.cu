@@ -16,25 +16,33 @@
 //    costs a shared-memory read and a double-size write per operand byte, and tensor-core operand
 //    reads take priority over that traffic on the shared-memory banks.)
 //
-// 2. w4a4_gemm_kernel: persistent, one CTA per SM.  The MMA computes the transposed tile
-//    D[n][t] (M = 128 output channels = TMEM lanes, N = 256 tokens).  The K loop runs one
-//    128-wide group per step.  Warp roles (12 warps):
-//      warp 0      TMA producer: E4M3 tiles of W (128 x 128 B) and X (256 x 128 B) per group
-//                  into a 4-stage ring.
-//      warp 1      TMEM allocator and MMA issuer: 4 x tcgen05.mma kind::f8f6f4 (M128 N256 K32)
-//                  per group into a double-buffered float32 accumulator; the first of the four
-//                  overwrites the buffer.
-//      warps 2..3  scale loaders: the tile's weight and activation scales for 4 groups at a time
-//                  ([row][4] float32, cp.async, zero-filled past N / T / G) into a 4-stage ring.
+// 2. w4a4_gemm_kernel: persistent, one CTA per SM, launched as clusters of two CTAs (a CTA
+//    pair on one SM pair) that share every MMA (tcgen05 cta_group::2).  A pair's tile is
+//    256 output channels x 256 tokens: the even CTA's MMA (M = 256, N = 256) reads weight rows
+//    0..127 and tokens 0..127 from its own shared memory and weight rows 128..255 and tokens
+//    128..255 from its peer's, and each CTA's tensor memory receives its own 128 channels x
+//    256 tokens (D[n][t], channels = TMEM lanes).  Each SM thus loads 32 KB of operands per
+//    group instead of the 48 KB a single CTA needs for 128 x 256, for the same tensor-core
+//    work.  The K loop runs one 128-wide group per step.  Warp roles (12 warps per CTA):
+//      warp 0      TMA producer: this CTA's 128 weight rows and 128 tokens per group into a
+//                  6-stage ring; the bytes of both CTAs complete on the even CTA's barrier.
+//      warp 1      TMEM allocator (both CTAs) and, in the even CTA only, the MMA issuer:
+//                  4 x tcgen05.mma.cta_group::2 kind::f8f6f4 (M256 N256 K32) per group into a
+//                  double-buffered float32 accumulator (the first of the four overwrites the
+//                  buffer); one multicast commit frees both CTAs' stage, another tells both
+//                  epilogues the group is done.
+//      warps 2..3  scale loaders: the CTA's weight scales and the tile's activation scales for
+//                  4 groups at a time (cp.async, zero-filled past N / T / G) into a 4-stage ring.
 //      warps 4..11 epilogue: 2 warps per TMEM lane quarter, 128 tokens each.  Tensor memory is
 //                  read with the 16x256b shape, so each thread holds 4 output channels x 32
 //                  tokens: per group it needs 4 weight scales and 32 token scales (a quarter of
 //                  the shared-memory traffic of one channel x 128 tokens per thread).  Per element
 //                  acc += fl(d * sw) * sa in float32 registers, groups in ascending order, with
-//                  one packed multiply and one packed FMA per element pair; after the last group
+//                  one packed multiply and one packed FMA per element pair; each warp hands its
+//                  part of the buffer back to the even CTA's MMA issuer; after the last group
 //                  the tile is stored to Y.
 //    Every mbarrier wait is bounded; a timeout sets a status bit, the CTA drains its own copies
-//    and MMAs, frees tensor memory and returns.
+//    and MMAs, meets its peer (bounded), frees tensor memory and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -51,40 +59,40 @@ __device__ unsigned int g_gemm_status = 0;
 
 namespace {
 
-constexpr int BM = 128;          // tile rows = output channels (weight rows), MMA M
+constexpr int BM = 128;          // output channels (weight rows) per CTA = its TMEM lanes
+constexpr int PAIR_M = 2 * BM;   // a CTA pair's MMA has M = 256 (128 rows in each CTA)
 constexpr int BN = 256;          // tile columns = tokens (activation rows), MMA N
+constexpr int BN_HALF = BN / 2;  // tokens staged by each CTA of the pair
 constexpr int BK = 128;          // one quantisation group = 128 bytes = one 128-byte swizzle row
-constexpr int OP_STAGES = 4;     // operand ring
+constexpr int OP_STAGES = 6;     // operand ring
 constexpr int SC_GROUPS = 4;     // groups per scale stage
 constexpr int S_STAGES = 4;      // scale ring
-#ifndef PQ_GEMM_EPI_WARPS
-#define PQ_GEMM_EPI_WARPS 8
-#endif
-constexpr int NUM_EPI_WARPS = PQ_GEMM_EPI_WARPS;   // 8 or 16 (2 or 4 per TMEM lane quarter)
-constexpr int EPI_WARP0 = 4;     // warps 0..3 control, then the epilogue
+constexpr int NUM_EPI_WARPS = 8;   // 2 per TMEM lane quarter
+constexpr int EPI_WARP0 = 4;       // warps 0..3 control, then the epilogue
 constexpr int NUM_THREADS = 32 * (EPI_WARP0 + NUM_EPI_WARPS);
-constexpr int EPI_COLS = BN / (NUM_EPI_WARPS / 4);   // tokens per epilogue warp (128 or 64)
+constexpr int EPI_COLS = BN / (NUM_EPI_WARPS / 4);   // tokens per epilogue warp: 128
 constexpr int EPI_CHUNKS = EPI_COLS / 16;            // 16-token chunks of the accumulator layout
-constexpr int EPI_LDC = NUM_EPI_WARPS == 8 ? 32 : 16;  // tokens per TMEM load (per lane half)
+// Tokens per tensor-memory wait (per lane half).  16 (one 16x256b.x2 load per lane half) was
+// measured faster than 32 or than overlapping the next chunk's load with this chunk's math.
+constexpr int EPI_LDC = 16;
 constexpr int EPI_NX = EPI_LDC / 8;                  // 16x256b repetitions per load
 constexpr int NUM_SCALE_THREADS = 64;                // warps 2 and 3
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;     // 2 s
-constexpr uint32_t kTxBytes = (BM + BN) * BK;
+constexpr uint32_t kTxBytes = 2 * (BM + BN_HALF) * BK;   // both CTAs' tiles, on the even CTA's barrier
 // Register budget (setmaxnreg): launch allocation per thread and the control and epilogue
 // warps' shares; 128 * REG_CTRL + 32 * NUM_EPI_WARPS * REG_EPI must not exceed
 // NUM_THREADS * REG_LAUNCH.
-constexpr uint32_t REG_LAUNCH = NUM_EPI_WARPS == 8 ? 168 : 96;
-constexpr uint32_t REG_CTRL = NUM_EPI_WARPS == 8 ? 56 : 48;
-constexpr uint32_t REG_EPI = NUM_EPI_WARPS == 8 ? 224 : 104;
+constexpr uint32_t REG_LAUNCH = 168;
+constexpr uint32_t REG_CTRL = 56;
+constexpr uint32_t REG_EPI = 224;
 static_assert(REG_CTRL * 32 * EPI_WARP0 + REG_EPI * 32 * NUM_EPI_WARPS <= REG_LAUNCH * NUM_THREADS,
               "setmaxnreg shares exceed the launch allocation");
 static_assert(REG_LAUNCH * NUM_THREADS <= 65536, "launch register allocation exceeds the SM");
-static_assert(NUM_EPI_WARPS == 8 || NUM_EPI_WARPS == 16, "2 or 4 epilogue warps per lane quarter");
 
 struct __align__(1024) GemmSmem {
-  uint8_t opA[OP_STAGES][BM * BK];          // weights, 16 KB per stage, 128-byte swizzle
-  uint8_t opB[OP_STAGES][BN * BK];          // activations, 32 KB per stage
+  uint8_t opA[OP_STAGES][BM * BK];          // this CTA's 128 weight rows, 16 KB per stage, 128-byte swizzle
+  uint8_t opB[OP_STAGES][BN_HALF * BK];     // this CTA's 128 of the tile's 256 tokens, 16 KB per stage
   float sc_w[S_STAGES][BM][SC_GROUPS];      // weight scales: [tile row][group of the stage]
   float sc_a[S_STAGES][BN][SC_GROUPS];      // activation scales: [tile token][group]
   uint64_t op_full[OP_STAGES];
@@ -94,6 +102,7 @@ struct __align__(1024) GemmSmem {
   uint64_t sc_full[S_STAGES];
   uint64_t sc_empty[S_STAGES];
   uint64_t mma_done;
+  uint64_t pair_done;
   uint32_t tmem_slot;
   int abort_flag;
 };
@@ -169,11 +178,12 @@ __global__ void __launch_bounds__(256) expand_codes_kernel(const uint8_t* __rest
   }
 }
 
-// Tile order: weight tiles fastest, so the CTAs running at the same time share a token tile.
-// (Token-fastest and banded orders were measured no faster.)
+// Tile order: weight tiles fastest, so the CTA pairs running at the same time share a token
+// tile.  A tile is PAIR_M weight rows x BN tokens, computed by one CTA pair; m0 is the pair's
+// first row.  (Token-fastest and banded orders were measured no faster.)
 __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& m0, int& n0) {
   (void)n_tiles;
-  m0 = (tile % m_tiles) * BM;
+  m0 = (tile % m_tiles) * PAIR_M;
   n0 = (tile / m_tiles) * BN;
 }
 
@@ -184,6 +194,8 @@ struct Work {
   int m_tiles, n_tiles, num_tiles;
   int ksplit, gs, G;
   int units;
+  int first, stride;     // this CTA pair's first unit and the number of pairs in the grid
+  int rank;              // 0 = even CTA (issues the pair's MMAs), 1 = odd CTA
 };
 
 __device__ __forceinline__ void unit_coords(int u, const Work& wk, int& m0, int& n0, int& kr, int& k0, int& k1) {
@@ -202,32 +214,42 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
+    // Both CTAs of the pair load their own halves (weight rows m0 + 128 rank, tokens
+    // n0 + 128 rank); all bytes complete on the even CTA's full barrier, whose MMA reads both.
     if (lane == 0) {
+      const uint32_t full0 = ptx::mapa_shared(ptx::smem_addr(&S.op_full[0]), 0);
       int step = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < wk.units && ok; u += gridDim.x) {
+      for (int u = wk.first; u < wk.units && ok; u += wk.stride) {
         int m0, n0, kr, k0, k1;
         unit_coords(u, wk, m0, n0, kr, k0, k1);
         for (int kg = k0; kg < k1; ++kg, ++step) {
           const int s = step % OP_STAGES;
           const uint32_t ph = (uint32_t)(step / OP_STAGES) & 1u;
           if (!wait_or_abort(S, &S.op_empty[s], ph ^ 1u, status)) { ok = false; break; }
-          ptx::mbar_arrive_expect_tx(&S.op_full[s], kTxBytes);
-          ptx::tma_load_2d(S.opA[s], &tmA, &S.op_full[s], kg * BK, m0);
-          ptx::tma_load_2d(S.opB[s], &tmB, &S.op_full[s], kg * BK, n0);
+          if (wk.rank == 0) ptx::mbar_arrive_expect_tx(&S.op_full[s], kTxBytes);
+          ptx::tma_load_2d_pair(S.opA[s], &tmA, full0 + 8u * s, kg * BK, m0 + BM * wk.rank);
+          ptx::tma_load_2d_pair(S.opB[s], &tmB, full0 + 8u * s, kg * BK, n0 + BN_HALF * wk.rank);
         }
       }
-      // Drain: every load issued lands before the CTA may exit.
+      // Drain: every stage's last use is released by the pair's MMAs (so every load issued has
+      // landed and every release aimed at this CTA has arrived) before the CTA may exit.
+      if (wk.rank == 0)
+        for (int j = (step > OP_STAGES ? step - OP_STAGES : 0); j < step; ++j)
+          drain_wait(&S.op_full[j % OP_STAGES], (uint32_t)(j / OP_STAGES) & 1u);
       for (int j = (step > OP_STAGES ? step - OP_STAGES : 0); j < step; ++j)
-        drain_wait(&S.op_full[j % OP_STAGES], (uint32_t)(j / OP_STAGES) & 1u);
+        drain_wait(&S.op_empty[j % OP_STAGES], (uint32_t)(j / OP_STAGES) & 1u);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = ptx::idesc_e4m3_f32(BM, BN);
+    // The even CTA issues M256 x N256 pair MMAs: its tensor memory receives weight rows
+    // m0 .. m0 + 127, the odd CTA's rows m0 + 128 ..; both CTAs' stages and accumulator buffers
+    // are released by one multicast commit.
+    if (lane == 0 && wk.rank == 0) {
+      constexpr uint32_t idesc = ptx::idesc_e4m3_f32(PAIR_M, BN);
       int step = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < wk.units && ok; u += gridDim.x) {
+      for (int u = wk.first; u < wk.units && ok; u += wk.stride) {
         int m0, n0, kr, k0, k1;
         unit_coords(u, wk, m0, n0, kr, k0, k1);
         for (int kg = k0; kg < k1; ++kg, ++step) {
@@ -244,14 +266,17 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
           const uint32_t d = tmem + (uint32_t)b * BN;
 #pragma unroll
           for (int k = 0; k < 4; ++k)   // k = 0 overwrites the buffer: each group starts from 0
-            ptx::umma_e4m3(d, ptx::smem_desc_sw128(a0 + 32 * k), ptx::smem_desc_sw128(b0 + 32 * k), idesc,
-                           k > 0 ? 1u : 0u);
-          ptx::umma_commit(&S.op_empty[s]);
-          ptx::umma_commit(&S.acc_full[b]);
+            ptx::umma_e4m3_pair(d, ptx::smem_desc_sw128(a0 + 32 * k), ptx::smem_desc_sw128(b0 + 32 * k), idesc,
+                                k > 0 ? 1u : 0u);
+          ptx::umma_commit_pair(&S.op_empty[s], 0x3);
+          ptx::umma_commit_pair(&S.acc_full[b], 0x3);
         }
       }
-      ptx::umma_commit(&S.mma_done);
+      ptx::umma_commit_pair(&S.mma_done, 0x1);
       drain_wait(&S.mma_done, 0);
+      // Both CTAs' epilogues release the last two buffers here before this CTA may exit.
+      for (int j = (step > 2 ? step - 2 : 0); j < step; ++j)
+        drain_wait(&S.acc_empty[j & 1], (uint32_t)(j >> 1) & 1u);
     }
   } else {
     // ---------------------------------------------------------------- scale loaders
@@ -259,7 +284,7 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
     const int j = threadIdx.x - 64;                      // 0..63
     int cs = 0;                                          // scale stages filled so far
     bool ok = true;
-    for (int u = blockIdx.x; u < wk.units && ok; u += gridDim.x) {
+    for (int u = wk.first; u < wk.units && ok; u += wk.stride) {
       int m0, n0, kr, k0, k1;
       unit_coords(u, wk, m0, n0, kr, k0, k1);
       for (int kg0 = k0; kg0 < k1; kg0 += SC_GROUPS, ++cs) {
@@ -270,7 +295,7 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
         for (int i = 0; i < (BM + BN) / NUM_SCALE_THREADS; ++i) {
           const int r = j + NUM_SCALE_THREADS * i;       // 0..127 weight rows, 128..383 tokens
           const bool isw = r < BM;
-          const int row = isw ? m0 + r : n0 + (r - BM);
+          const int row = isw ? m0 + BM * wk.rank + r : n0 + (r - BM);
           const bool in = row < (isw ? N : T);
           const float* src = (isw ? scales_W : scales_A) + (int64_t)(in ? row : 0) * G + kg0;
           float* dst = isw ? S.sc_w[st][r] : S.sc_a[st][r - BM];
@@ -302,9 +327,11 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
   const int sub = warp & 3;          // TMEM lane quarter this warp may access
   const int ch = ew >> 2;            // token half of the tile
   const int g = lane >> 2, q = lane & 3;
+  // Accumulator buffers are handed back to the even CTA, whose thread issues the pair's MMAs.
+  const uint32_t acc_empty0 = ptx::mapa_shared(ptx::smem_addr(&S.acc_empty[0]), 0);
   int step = 0, cs = 0;
   bool ok = true;
-  for (int u = blockIdx.x; u < wk.units && ok; u += gridDim.x) {
+  for (int u = wk.first; u < wk.units && ok; u += wk.stride) {
     int m0, n0, kr, k0, k1;
     unit_coords(u, wk, m0, n0, kr, k0, k1);
     constexpr int kAcc2 = 4 * EPI_CHUNKS * 2;         // rows (h, k) x chunks x x; e is the pair
@@ -348,15 +375,16 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
           // The whole group's tile is read: hand the buffer back to the MMA before the math.
           ptx::tc_fence_before();
           __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&S.acc_empty[b]);
+          if (lane == 0) ptx::mbar_arrive_remote(acc_empty0 + 8u * b);
         }
 #pragma unroll
         for (int x = 0; x < EPI_NX; ++x)
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
-            const int c = (EPI_LDC / 16) * cc + (x >> 1);   // 16-token chunk of the accumulator layout
-            const int i0 = ((0 * 2 + k) * EPI_CHUNKS + c) * 2 + (x & 1);
-            const int i1 = ((1 * 2 + k) * EPI_CHUNKS + c) * 2 + (x & 1);
+            const int xx = (EPI_LDC / 8) * cc + x;          // 8-token block of the warp's 128
+            const int c = xx >> 1;                          // 16-token chunk of the accumulator layout
+            const int i0 = ((0 * 2 + k) * EPI_CHUNKS + c) * 2 + (xx & 1);
+            const int i1 = ((1 * 2 + k) * EPI_CHUNKS + c) * 2 + (xx & 1);
             ptx::mul_fma2(acc2[i0], d0[4 * x + 2 * k], d0[4 * x + 2 * k + 1], sw2[0 * 2 + k], sa2[x], after);
             ptx::mul_fma2(acc2[i1], d1[4 * x + 2 * k], d1[4 * x + 2 * k + 1], sw2[1 * 2 + k], sa2[x], after);
           }
@@ -370,7 +398,7 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
     if (!ok) break;
     // Y[t][n]: per store, 8 lanes (same q) write 8 consecutive channels of one token.  The
     // thread's channels are nb + {0, 8, 16, 24}, its tokens tb + 16 c + 8 x + e.
-    const int nb = m0 + 32 * sub + g;
+    const int nb = m0 + BM * wk.rank + 32 * sub + g;
     const int tb = n0 + ch * EPI_COLS + 2 * q;
     bool nin[4];
 #pragma unroll
@@ -405,7 +433,7 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
   }
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const float* __restrict__ scales_A, const float* __restrict__ scales_W, void* __restrict__ Y,
     int T, int N, int G, int scales_vec16, int out_bf16, int m_tiles, int n_tiles, int ksplit, int gs,
@@ -422,6 +450,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
   wk.gs = gs;
   wk.G = G;
   wk.units = wk.num_tiles * ksplit;
+  wk.rank = (int)ptx::cluster_ctarank();
+  wk.first = (int)(blockIdx.x >> 1);
+  wk.stride = (int)(gridDim.x >> 1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < OP_STAGES; ++s) {
@@ -430,13 +461,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&S.acc_full[b], 1);
-      ptx::mbar_init(&S.acc_empty[b], NUM_EPI_WARPS);
+      ptx::mbar_init(&S.acc_empty[b], 2 * NUM_EPI_WARPS);   // both CTAs' epilogue warps
     }
     for (int s = 0; s < S_STAGES; ++s) {
       ptx::mbar_init(&S.sc_full[s], NUM_SCALE_THREADS);
       ptx::mbar_init(&S.sc_empty[s], NUM_EPI_WARPS);
     }
     ptx::mbar_init(&S.mma_done, 1);
+    ptx::mbar_init(&S.pair_done, 1);
     S.abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -445,11 +477,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
     ptx::prefetch_tmap(&tmB);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(&S.tmem_slot, TMEM_COLS);
-    ptx::tmem_relinquish();
+    ptx::tmem_alloc_pair(&S.tmem_slot, TMEM_COLS);
+    ptx::tmem_relinquish_pair();
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  ptx::cluster_sync();   // both CTAs' barriers initialised and tensor memory allocated
   ptx::tc_fence_after();
   const uint32_t tmem = S.tmem_slot;
 
@@ -464,9 +496,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
   __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
+  // Neither CTA leaves while its peer may still arrive on its barriers or read its tiles.
+  if (threadIdx.x == 0) {
+    ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_addr(&S.pair_done), (uint32_t)wk.rank ^ 1u));
+    int never = 0;
+    if (!ptx::mbar_wait_bounded_cl(&S.pair_done, 0, &never, kWaitLimitNs)) atomicOr(status, PQ_DEV_TIMEOUT);
+  }
+  __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, TMEM_COLS);
+    ptx::tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 
@@ -585,13 +624,14 @@ int device_sm_count() {
 
 size_t gemm_scratch_bytes(int64_t T, int64_t N, int64_t D) { return (size_t)(T + N) * (size_t)D; }
 
+// Split-K when the tiles fill at most half of the CTA pairs the device can run at once.
 int gemm_ksplit(int64_t T, int64_t N, int64_t D, int* gs_out) {
   const int G = (int)(D / 128);
-  const int64_t tiles = ((N + BM - 1) / BM) * ((T + BN - 1) / BN);
-  const int sms = device_sm_count();
+  const int64_t tiles = ((N + PAIR_M - 1) / PAIR_M) * ((T + BN - 1) / BN);
+  const int pairs = device_sm_count() / 2;
   int ks = 1, gs = G;
-  if (G >= 2 * SC_GROUPS && tiles * 2 <= sms) {
-    const int want = (int)std::min<int64_t>(sms / tiles, G / SC_GROUPS);
+  if (G >= 2 * SC_GROUPS && tiles * 2 <= pairs) {
+    const int want = (int)std::min<int64_t>(pairs / tiles, G / SC_GROUPS);
     gs = ((G + want - 1) / want + SC_GROUPS - 1) / SC_GROUPS * SC_GROUPS;   // multiple of 4 groups
     ks = (G + gs - 1) / gs;
     if (ks < 2) { ks = 1; gs = G; }
@@ -614,9 +654,9 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   CUtensorMap tmA, tmB;
   pq_status st = make_operand_map(&tmA, W8, N, D, BM);
   if (st != PQ_OK) return st;
-  st = make_operand_map(&tmB, A8, T, D, BN);
+  st = make_operand_map(&tmB, A8, T, D, BN_HALF);
   if (st != PQ_OK) return st;
-  const int m_tiles = (int)((N + BM - 1) / BM);
+  const int m_tiles = (int)((N + PAIR_M - 1) / PAIR_M);
   const int n_tiles = (int)((T + BN - 1) / BN);
   const int64_t tiles = (int64_t)m_tiles * n_tiles;
   if (tiles >= ((int64_t)1 << 31)) {
@@ -638,7 +678,31 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   int gs = (int)(D / 128);
   const int ksplit = ws ? gemm_ksplit(T, N, D, &gs) : 1;
   const int64_t units = tiles * ksplit;
-  const int grid = (int)(units < sms ? units : sms);
+  // CTA pairs (clusters of 2) resident at once: one per SM pair when every pair can host one.
+  static int max_pairs = -1;
+  if (max_pairs < 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, w4a4_gemm_kernel, &cfg);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(gemm)");
+    if (n < 1) {
+      set_error("w4a4_gemm_kernel: no CTA pair fits on this device");
+      return PQ_ERR_UNSUPPORTED;
+    }
+    max_pairs = n;
+  }
+  const int64_t pairs = max_pairs;
+  const int grid = 2 * (int)(units < pairs ? units : pairs);
   // The warp roles re-divide the launch's registers with setmaxnreg; that only works when the
   // kernel was compiled with exactly the budgeted count (otherwise an increase would never be
   // granted), so refuse to launch anything else.
