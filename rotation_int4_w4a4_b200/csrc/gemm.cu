@@ -550,13 +550,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
+  static std::atomic<EncodeTiledFn> cache{nullptr};
+  EncodeTiledFn fn = cache.load(std::memory_order_acquire);
   if (!fn) {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+        q == cudaDriverEntryPointSuccess) {
       fn = reinterpret_cast<EncodeTiledFn>(p);
+      cache.store(fn, std::memory_order_release);
+    }
   }
   return fn;
 }
@@ -587,11 +590,11 @@ pq_status make_operand_map(CUtensorMap* map, const uint8_t* base, int64_t rows, 
 // synchronisation (which made each call pay for fresh page mappings).
 cudaError_t scratch_pool(cudaMemPool_t* out) {
   static std::mutex mu;
-  static cudaMemPool_t pools[64] = {};
+  static cudaMemPool_t pools[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
   if (!pools[dev]) {
     cudaMemPoolProps props = {};
@@ -613,11 +616,37 @@ cudaError_t scratch_pool(cudaMemPool_t* out) {
   return cudaSuccess;
 }
 
-int device_sm_count() {
-  int dev = 0, c = 0;
-  cudaGetDevice(&dev);
-  if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
-  return c;
+// CTA pairs (clusters of 2) of w4a4_gemm_kernel resident at once on the current device: one
+// per SM pair when every pair can host one.  Needs the kernel's shared-memory attribute set.
+pq_status gemm_max_pairs(int sms, int* out) {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  const bool slot = dev >= 0 && dev < kMaxDevices;
+  int n = slot ? cache[dev].load(std::memory_order_relaxed) : 0;
+  if (n < 1) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    e = cudaOccupancyMaxActiveClusters(&n, w4a4_gemm_kernel, &cfg);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(gemm)");
+    if (n < 1) {
+      set_error("w4a4_gemm_kernel: no CTA pair fits on this device");
+      return PQ_ERR_UNSUPPORTED;
+    }
+    if (slot) cache[dev].store(n, std::memory_order_relaxed);
+  }
+  *out = n;
+  return PQ_OK;
 }
 
 }  // namespace
@@ -667,7 +696,7 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   const int64_t chunksA = T * (D / 32), chunksW = N * (D / 32);   // 16 packed bytes each
   const int64_t want = (chunksA + chunksW + 255) / 256;
   const int egrid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
-  static bool attr_expand[64] = {}, attr_gemm[64] = {};
+  static std::atomic<bool> attr_expand[kMaxDevices], attr_gemm[kMaxDevices];
   cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(expand_codes_kernel), 0, attr_expand);
   if (e != cudaSuccess) return cuda_fail(e, "expand_codes_kernel attributes");
   e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_kernel), (int)kSmemBytes, attr_gemm);
@@ -678,40 +707,22 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   int gs = (int)(D / 128);
   const int ksplit = ws ? gemm_ksplit(T, N, D, &gs) : 1;
   const int64_t units = tiles * ksplit;
-  // CTA pairs (clusters of 2) resident at once: one per SM pair when every pair can host one.
-  static int max_pairs = -1;
-  if (max_pairs < 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
-    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = 2;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, w4a4_gemm_kernel, &cfg);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(gemm)");
-    if (n < 1) {
-      set_error("w4a4_gemm_kernel: no CTA pair fits on this device");
-      return PQ_ERR_UNSUPPORTED;
-    }
-    max_pairs = n;
-  }
+  int max_pairs = 0;
+  st = gemm_max_pairs(sms, &max_pairs);
+  if (st != PQ_OK) return st;
   const int64_t pairs = max_pairs;
   const int grid = 2 * (int)(units < pairs ? units : pairs);
   // The warp roles re-divide the launch's registers with setmaxnreg; that only works when the
   // kernel was compiled with exactly the budgeted count (otherwise an increase would never be
   // granted), so refuse to launch anything else.
-  static int num_regs = -1;
+  static std::atomic<int> num_regs_cache{-1};       // a property of the kernel binary
+  int num_regs = num_regs_cache.load(std::memory_order_relaxed);
   if (num_regs < 0) {
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, w4a4_gemm_kernel);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(gemm)");
     num_regs = fa.numRegs;
+    num_regs_cache.store(num_regs, std::memory_order_relaxed);
   }
   if (num_regs != (int)REG_LAUNCH) {
     set_error("w4a4_gemm_kernel compiled with %d registers per thread, %u expected", num_regs, REG_LAUNCH);

@@ -28,8 +28,6 @@ static __device__ __align__(256) uint8_t g_static_scratch[PQ_NOALLOC_SCRATCH_BYT
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-
 struct DeviceSetup {
   bool ready = false;
   uint8_t* scratch = nullptr;

@@ -1,6 +1,7 @@
 // Internal declarations shared by the host code and the kernel launchers of libpq.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cstdio>
 #include <string>
@@ -46,19 +47,39 @@ pq_status cuda_fail(cudaError_t err, const char* what);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Per-device caches below hold one slot per device index; devices beyond the table are
+// served without caching.  Every cached value is the same whichever thread computes it first,
+// so concurrent first calls from several host threads only repeat an idempotent query.
+constexpr int kMaxDevices = 64;
+
 // Kernel attributes set once per device and kernel (the dynamic shared-memory limit), so that
 // launches do not repeat the driver call.  `done` is the caller's per-kernel table.
-inline cudaError_t set_kernel_attributes(const void* func, int dyn_smem, bool (&done)[64]) {
+inline cudaError_t set_kernel_attributes(const void* func, int dyn_smem, std::atomic<bool> (&done)[kMaxDevices]) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  const bool slot = dev >= 0 && dev < kMaxDevices;
+  if (slot && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
   if (dyn_smem > 0) {
     e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
     if (e != cudaSuccess) return e;
   }
-  if (dev >= 0 && dev < 64) done[dev] = true;
+  if (slot) done[dev].store(true, std::memory_order_release);
   return cudaSuccess;
+}
+
+// Multiprocessor count of the current device (148 if it cannot be read).
+inline int device_sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  const bool slot = dev >= 0 && dev < kMaxDevices;
+  int c = slot ? cache[dev].load(std::memory_order_relaxed) : 0;
+  if (c <= 0) {
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
+    if (slot) cache[dev].store(c, std::memory_order_relaxed);
+  }
+  return c;
 }
 
 // Kernel launchers (transform.cu, gemm.cu).  Arguments are already validated.

@@ -264,13 +264,16 @@ typedef CUresult (*EncodeTiledFnR)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapFloatOOBfill);
 
 EncodeTiledFnR encode_fn_r() {
-  static EncodeTiledFnR fn = nullptr;
+  static std::atomic<EncodeTiledFnR> cache{nullptr};
+  EncodeTiledFnR fn = cache.load(std::memory_order_acquire);
   if (!fn) {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+        q == cudaDriverEntryPointSuccess) {
       fn = reinterpret_cast<EncodeTiledFnR>(p);
+      cache.store(fn, std::memory_order_release);
+    }
   }
   return fn;
 }
@@ -289,13 +292,6 @@ cudaError_t make_bf16_map(CUtensorMap* map, const void* base, int64_t rows, int6
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-int rt_sm_count() {
-  int dev = 0, c = 0;
-  cudaGetDevice(&dev);
-  if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
-  return c;
-}
-
 }  // namespace
 
 cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
@@ -312,12 +308,12 @@ cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, 
   if (e != cudaSuccess) return e;
   const int row_blocks = (int)((rows + RT_M - 1) / RT_M);
   const int64_t tiles = (int64_t)row_blocks * plan->G;
-  const int sms = rt_sm_count();
+  const int sms = device_sm_count();
   const int grid = (int)(tiles < sms ? tiles : sms);
   // Givens: scale = m / 7.  Hadamard: R = H unnormalised, so y is sqrt(128) times the
   // orthonormal rotation and scale = m / (7 sqrt(128)).
   const float scale_mult = givens ? (1.0f / 7.0f) : 0.012626906806902634f;
-  static bool attr_done[64] = {};
+  static std::atomic<bool> attr_done[kMaxDevices];
   e = set_kernel_attributes(reinterpret_cast<const void*>(rotate_mma_kernel), (int)kRotSmemBytes, attr_done);
   if (e != cudaSuccess) return e;
   rotate_mma_kernel<<<grid, RT_THREADS, kRotSmemBytes, stream>>>(tmX, tmR, rows, plan->G, row_blocks, tiles, terms,

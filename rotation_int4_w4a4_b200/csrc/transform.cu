@@ -323,19 +323,6 @@ __global__ void __launch_bounds__(128, 4) smooth_hadamard_kernel(
   }
 }
 
-int sm_count() {
-  static int count[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return 148;
-  if (!count[dev]) {
-    int c = 0;
-    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
-    count[dev] = c;
-  }
-  return count[dev];
-}
-
 }  // namespace
 
 cudaError_t launch_hadamard_rows(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx,
@@ -344,15 +331,17 @@ cudaError_t launch_hadamard_rows(const pq_plan* plan, const void* X, int64_t row
   const int64_t R = rows * plan->G;
   const int64_t tasks = (R + 7) / 8;                // one warp-task = 8 row-groups
   const int64_t want = (tasks + 7) / 8;             // 8 warps per block
-  static int per_sm = 0;
-  if (!per_sm) {
-    int b = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, hadamard_rows_kernel, 256, 0) != cudaSuccess || b < 1) b = 2;
-    per_sm = b;
+  static std::atomic<int> per_sm_cache{0};           // a property of the kernel binary
+  int per_sm = per_sm_cache.load(std::memory_order_relaxed);
+  if (per_sm < 1) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hadamard_rows_kernel, 256, 0) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 2;
+    per_sm_cache.store(per_sm, std::memory_order_relaxed);
   }
-  const int64_t cap = (int64_t)sm_count() * per_sm;  // one resident wave, tasks strided over it
+  const int64_t cap = (int64_t)device_sm_count() * per_sm;  // one resident wave, tasks strided over it
   const int grid = (int)(want < cap ? want : cap);
-  static bool attr_done[64] = {};
+  static std::atomic<bool> attr_done[kMaxDevices];
   cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(hadamard_rows_kernel), 0, attr_done);
   if (e != cudaSuccess) return e;
   hadamard_rows_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(X), rows,
@@ -364,7 +353,7 @@ cudaError_t launch_smooth_hadamard(const pq_plan* plan, const void* X, int64_t T
                                    uint8_t* codes, float* scales, float* smooth_out,
                                    cudaStream_t stream) {
   dim3 grid((unsigned)((T + kSmoothBlock - 1) / kSmoothBlock), (unsigned)plan->G);
-  static bool attr_done[64] = {};
+  static std::atomic<bool> attr_done[kMaxDevices];
   cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(smooth_hadamard_kernel), 0, attr_done);
   if (e != cudaSuccess) return e;
   smooth_hadamard_kernel<<<grid, 128, 0, stream>>>(
