@@ -78,10 +78,12 @@ def test_random_codes_bf16(pq):
 
 
 @pytest.mark.parametrize("T,N,D,out", [(1, 4096, 4096, "f32"), (16, 512, 2048, "bf16"),
-                                       (256, 1024, 4096, "f32"), (3, 4096, 1024, "bf16")])
+                                       (256, 1024, 4096, "f32"), (3, 4096, 1024, "bf16"),
+                                       (1, 272, 4096, "f32"), (5, 16, 1024, "bf16")])
 def test_split_k_small_T(pq, T, N, D, out):
-    """Few output tiles: the groups are split across CTAs and the float32 partial tiles are
-    reduced in ascending order; same tolerances as the unsplit path."""
+    """Few output tiles: the groups are split across CTA pairs and the float32 partial tiles are
+    reduced in ascending order; same tolerances as the unsplit path.  N = 272 and N = 16 leave
+    the odd CTA of the last pair with no channel inside N."""
     ca, sa = inputs.random_codes(41 + T, T, D)
     cw, sw = inputs.random_codes(43 + N, N, D)
     Y = run_gemm(pq, ca, sa, cw, sw, out=out)
