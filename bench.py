@@ -187,18 +187,15 @@ def job_value(world, tokens_per_rank_step, steps, total_ms):
     return world * tokens_per_rank_step * steps / (total_ms * 1e-3)
 
 
-# Kernels one step launches: transform_quant, pack_weights, int4 -> E4M3 expansion, GEMM; plus
-# the split-K reduction when the GEMM has fewer 128 x 256 output tiles than half the SMs and at
-# least 8 groups (the library's rule for splitting the group range).
+# Kernels one step launches: transform_quant and pack_weights (one each), then the GEMM's own
+# launches as the library reports them for these sizes on the current device (operand
+# expansion and contraction, plus the split-K reduction when it splits the group range).
 LAUNCHES_PER_STEP = 4
 
 
-def launches_per_step(T, N, D, sms):
-    # the GEMM's tiles are 256 channels x 256 tokens, one per CTA pair (sms // 2 pairs)
-    tiles = -(-N // 256) * -(-T // 256)
-    pairs = sms // 2
-    split = D // 128 >= 8 and 2 * tiles <= pairs and min(pairs // tiles, D // 512) >= 2
-    return LAUNCHES_PER_STEP + (1 if split else 0)
+def launches_per_step(T, N, D):
+    from rotation_int4_w4a4_b200 import pq
+    return 2 + pq.pq_w4a4_gemm_launch_count(T, N, D)
 
 
 # ------------------------------------------------------------------------ GPU arm
@@ -355,7 +352,7 @@ def run_ours(args, wl, rank, world, local_rank):
             "components": comps, "roofline": roof, "cpu_baseline": cpu,
             "e2e": {"value": job_value(world, wl.T, 1, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": launches_per_step(wl.T, wl.N, wl.D, torch.cuda.get_device_properties(dev).multi_processor_count) * args.steps, "clocks": ck, "wall_s_timed_region": w1 - w0}
+            "gpu_launches": launches_per_step(wl.T, wl.N, wl.D) * args.steps, "clocks": ck, "wall_s_timed_region": w1 - w0}
     print(json.dumps(line), flush=True)
 
 

@@ -198,6 +198,16 @@ pq_status pq_w4a4_gemm_noalloc(const uint8_t* codes_A, const float* scales_A,
                                void* stream);
 
 /*
+ * pq_w4a4_gemm_launch_count — host-only query, no counterpart in the pages.  Writes to
+ * *launches the number of kernels one pq_w4a4_gemm call with these sizes launches on the
+ * current device: 2 (operand expansion, contraction) or 3 (plus the split-K reduction, chosen
+ * when the 256 x 256 output tiles fill at most half of the device's SM pairs).
+ * pq_w4a4_gemm_noalloc never splits and always launches 2.  Sizes are validated as for
+ * pq_w4a4_gemm (PQ_ERR_INVALID_ARG otherwise).  Without a usable device the count assumes 148 SMs.
+ */
+pq_status pq_w4a4_gemm_launch_count(int64_t T, int64_t N, int64_t D, int* launches);
+
+/*
  * pq_check_status — synchronises `stream`, then reads and clears the device status words
  * (the plan's, if plan != NULL, and the GEMM's).  Returns PQ_ERR_TIMEOUT if a bounded
  * device-side wait gave up since the last check (the affected output is incomplete),

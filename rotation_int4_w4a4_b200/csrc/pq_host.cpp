@@ -357,6 +357,18 @@ extern "C" pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t
 
 namespace {
 
+// Size checks shared by the GEMM entry points and the launch-count query.
+pq_status check_gemm_sizes(int64_t T, int64_t N, int64_t D) {
+  if (T < 1 || N < 1 || D < kGroup) { set_error("T, N must be >= 1 and D >= 128"); return PQ_ERR_INVALID_ARG; }
+  if (D % kGroup != 0) { set_error("D=%lld must be a multiple of 128", (long long)D); return PQ_ERR_INVALID_ARG; }
+  if (N % 16 != 0) { set_error("N=%lld must be a multiple of 16", (long long)N); return PQ_ERR_INVALID_ARG; }
+  if (T >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || D >= ((int64_t)1 << 24)) {
+    set_error("T, N must be < 2^31 and D < 2^24");
+    return PQ_ERR_INVALID_ARG;
+  }
+  return PQ_OK;
+}
+
 // Argument checks shared by the GEMM entry points; nothing here touches the device.
 pq_status check_gemm_args(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                           const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
@@ -366,14 +378,9 @@ pq_status check_gemm_args(const uint8_t* codes_A, const float* scales_A, const u
     return PQ_ERR_INVALID_ARG;
   }
   if (g != kGroup) { set_error("g=%d: only g=128 is supported", g); return PQ_ERR_UNSUPPORTED; }
-  if (T < 1 || N < 1 || D < g) { set_error("T, N must be >= 1 and D >= 128"); return PQ_ERR_INVALID_ARG; }
-  if (D % g != 0) { set_error("D=%lld must be a multiple of 128", (long long)D); return PQ_ERR_INVALID_ARG; }
-  if (N % 16 != 0) { set_error("N=%lld must be a multiple of 16", (long long)N); return PQ_ERR_INVALID_ARG; }
+  pq_status st = check_gemm_sizes(T, N, D);
+  if (st != PQ_OK) return st;
   if (out_dtype != PQ_OUT_F32 && out_dtype != PQ_OUT_BF16) { set_error("bad out_dtype"); return PQ_ERR_INVALID_ARG; }
-  if (T >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || D >= ((int64_t)1 << 24)) {
-    set_error("T, N must be < 2^31 and D < 2^24");
-    return PQ_ERR_INVALID_ARG;
-  }
   if (!aligned16(codes_A) || !aligned16(scales_A) || !aligned16(codes_W) ||
       !aligned16(scales_W) || !aligned16(Y)) {
     set_error("device pointers must be 16-byte aligned");
@@ -404,6 +411,18 @@ extern "C" pq_status pq_w4a4_gemm_noalloc(const uint8_t* codes_A, const float* s
   if (st != PQ_OK) return st;
   return gemm_run_static_scratch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype,
                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" pq_status pq_w4a4_gemm_launch_count(int64_t T, int64_t N, int64_t D, int* launches) {
+  clear_error();
+  if (!launches) {
+    set_error("launches must be non-NULL");
+    return PQ_ERR_INVALID_ARG;
+  }
+  pq_status st = check_gemm_sizes(T, N, D);
+  if (st != PQ_OK) return st;
+  *launches = gemm_ksplit(T, N, D, nullptr) > 1 ? 3 : 2;
+  return PQ_OK;
 }
 
 extern "C" pq_status pq_selftest_wait_timeout(uint64_t limit_ns, void* stream) {

@@ -26,7 +26,8 @@ KINDS = {"hadamard": PQ_HADAMARD, "givens": PQ_GIVENS, "smooth_hadamard": PQ_SMO
 
 # Every symbol the header declares.
 EXPORTS = ("pq_select_pairs", "pq_make_plan", "pq_destroy_plan", "pq_transform_quant",
-           "pq_pack_weights", "pq_w4a4_gemm", "pq_w4a4_gemm_noalloc", "pq_check_status",
+           "pq_pack_weights", "pq_w4a4_gemm", "pq_w4a4_gemm_noalloc", "pq_w4a4_gemm_launch_count",
+           "pq_check_status",
            "pq_selftest_wait_timeout", "pq_status_string", "pq_last_error")
 
 _c = ctypes
@@ -45,6 +46,8 @@ lib.pq_w4a4_gemm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _i
 lib.pq_w4a4_gemm.restype = _i32
 lib.pq_w4a4_gemm_noalloc.argtypes = lib.pq_w4a4_gemm.argtypes
 lib.pq_w4a4_gemm_noalloc.restype = _i32
+lib.pq_w4a4_gemm_launch_count.argtypes = [_i64, _i64, _i64, _c.POINTER(_i32)]
+lib.pq_w4a4_gemm_launch_count.restype = _i32
 lib.pq_selftest_wait_timeout.argtypes = [_u64, _vp]
 lib.pq_selftest_wait_timeout.restype = _i32
 lib.pq_check_status.argtypes = [_vp, _vp]
@@ -179,6 +182,13 @@ def pq_w4a4_gemm_noalloc(codes_A, scales_A, codes_W, scales_W, Y, T=None, N=None
     _check(lib.pq_w4a4_gemm_noalloc(_ptr(codes_A), _ptr(scales_A), _ptr(codes_W), _ptr(scales_W),
                                     T, N, D, g, _ptr(Y), out_dtype, _stream(stream)),
            "pq_w4a4_gemm_noalloc")
+
+
+def pq_w4a4_gemm_launch_count(T: int, N: int, D: int) -> int:
+    """Kernels one pq_w4a4_gemm call of these sizes launches on the current device (2 or 3)."""
+    n = _i32(0)
+    _check(lib.pq_w4a4_gemm_launch_count(T, N, D, _c.byref(n)), "pq_w4a4_gemm_launch_count")
+    return n.value
 
 
 def pq_selftest_wait_timeout(limit_ns: int, stream=None) -> None:

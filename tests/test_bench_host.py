@@ -78,7 +78,9 @@ def test_job_value_is_weak_scaling():
     one = bench.job_value(1, 2048, 10, 5.0)
     assert bench.job_value(4, 2048, 10, 5.0) == pytest.approx(4 * one)
     assert bench.LAUNCHES_PER_STEP == 4
-    assert bench.launches_per_step(2048, 4096, 4096, 148) == 4      # 128 pair tiles: no split
-    assert bench.launches_per_step(1, 4096, 4096, 148) == 5         # 16 pair tiles: split-K + reduce
-    assert bench.launches_per_step(16, 14336, 4096, 148) == 4       # 56 pair tiles: no split
-    assert bench.launches_per_step(1, 4096, 256, 148) == 4          # 2 groups: no split
+    # No GPU here: the library counts with B200's 148 SMs (74 SM pairs).
+    assert bench.launches_per_step(2048, 4096, 4096) == 4      # 128 pair tiles: no split
+    assert bench.launches_per_step(1, 4096, 4096) == 5         # 16 pair tiles: split-K + reduce
+    assert bench.launches_per_step(16, 14336, 4096) == 4       # 56 pair tiles: no split
+    assert bench.launches_per_step(1, 4096, 256) == 4          # 2 groups: no split
+    assert bench.launches_per_step(1, 272, 4096) == 5          # 2 pair tiles, ragged N: split

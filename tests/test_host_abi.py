@@ -102,3 +102,20 @@ def test_selftest_wait_timeout_validation(pq):
         assert pq.lib.pq_selftest_wait_timeout(bad, None) == pq.PQ_ERR_INVALID_ARG
         assert b"limit_ns" in pq.lib.pq_last_error()
 
+
+
+def test_gemm_launch_count_query(pq):
+    """Host-only query (no GPU here, so 148 SMs are assumed): sizes are validated as for the
+    GEMM, and the count is 2 or 3 (with the split-K reduction)."""
+    import ctypes
+    L = pq.lib
+    n = ctypes.c_int(-1)
+    assert L.pq_w4a4_gemm_launch_count(4, 24, 128, ctypes.byref(n)) == pq.PQ_ERR_INVALID_ARG
+    assert L.pq_w4a4_gemm_launch_count(4, 16, 200, ctypes.byref(n)) == pq.PQ_ERR_INVALID_ARG
+    assert L.pq_w4a4_gemm_launch_count(0, 16, 128, ctypes.byref(n)) == pq.PQ_ERR_INVALID_ARG
+    assert L.pq_w4a4_gemm_launch_count(4, 16, 128, None) == pq.PQ_ERR_INVALID_ARG
+    assert n.value == -1
+    assert pq.pq_w4a4_gemm_launch_count(4096, 14336, 4096) == 2   # 896 pair tiles
+    assert pq.pq_w4a4_gemm_launch_count(1, 14336, 4096) == 2      # 56 pair tiles > 74 / 2
+    assert pq.pq_w4a4_gemm_launch_count(256, 4096, 4096) == 3     # 16 pair tiles, 32 groups
+    assert pq.pq_w4a4_gemm_launch_count(1, 4096, 512) == 2        # 4 groups: never split
