@@ -70,12 +70,22 @@ def _check(status: int, where: str) -> None:
         raise PQError(status, where)
 
 
-def _ptr(x):
-    """Device pointer of a tensor (or None -> NULL)."""
+def _ptr(x, rows_strided=False):
+    """Device pointer of a tensor (None -> NULL; an int passes through as a raw address).
+
+    The library reads and writes dense row-major device buffers, so a tensor must live on a
+    CUDA device and be contiguous; with rows_strided (the activations, whose row stride is
+    passed as ldx) only the last dimension must be contiguous.  Anything else would be read at
+    the wrong addresses, so it is rejected here instead.
+    """
     if x is None:
         return None
     if isinstance(x, int):
         return x
+    if not getattr(x, "is_cuda", False):
+        raise ValueError("expected a CUDA tensor: the library takes device pointers")
+    if not (x.stride(-1) == 1 if rows_strided else x.is_contiguous()):
+        raise ValueError("expected a contiguous tensor" + (" along its last dimension" if rows_strided else ""))
     return x.data_ptr()
 
 
@@ -146,7 +156,7 @@ def pq_transform_quant(plan: Plan, X, codes, scales, smooth_out=None, T=None, ld
     """X bf16 [T, ldx] -> codes uint8 [T, D/2], scales float32 [T, D/g] (device tensors)."""
     T = X.shape[0] if T is None else T
     ldx = X.stride(0) if ldx is None else ldx
-    _check(lib.pq_transform_quant(plan.handle, _ptr(X), T, ldx, _ptr(codes), _ptr(scales),
+    _check(lib.pq_transform_quant(plan.handle, _ptr(X, rows_strided=True), T, ldx, _ptr(codes), _ptr(scales),
                                   _ptr(smooth_out), _stream(stream)), "pq_transform_quant")
 
 

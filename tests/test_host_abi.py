@@ -119,3 +119,33 @@ def test_gemm_launch_count_query(pq):
     assert pq.pq_w4a4_gemm_launch_count(1, 14336, 4096) == 2      # 56 pair tiles > 74 / 2
     assert pq.pq_w4a4_gemm_launch_count(256, 4096, 4096) == 3     # 16 pair tiles, 32 groups
     assert pq.pq_w4a4_gemm_launch_count(1, 4096, 512) == 2        # 4 groups: never split
+
+
+def test_binding_rejects_host_and_strided_tensors(pq):
+    """The binding checks device and layout before any call reaches the library."""
+    import torch
+    with pytest.raises(ValueError, match="CUDA"):
+        pq._ptr(torch.zeros(4, 4))
+
+    class FakeCuda:                       # stands in for a CUDA tensor on this GPU-less box
+        is_cuda = True
+
+        def __init__(self, contiguous, inner):
+            self._c, self._s = contiguous, inner
+
+        def is_contiguous(self):
+            return self._c
+
+        def stride(self, dim):
+            return self._s
+
+        def data_ptr(self):
+            return 4096
+
+    assert pq._ptr(FakeCuda(True, 1)) == 4096
+    with pytest.raises(ValueError, match="contiguous"):
+        pq._ptr(FakeCuda(False, 1))
+    assert pq._ptr(FakeCuda(False, 1), rows_strided=True) == 4096   # padded rows (ldx > D)
+    with pytest.raises(ValueError, match="last dimension"):
+        pq._ptr(FakeCuda(False, 2), rows_strided=True)
+    assert pq._ptr(None) is None and pq._ptr(16) == 16
