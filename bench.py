@@ -1,21 +1,27 @@
 """Benchmark of the rotation + INT4 W4A4 hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload q_proj]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload down_proj] [--T T --N N --kind hadamard|givens] [--l2 flush|rotate]
 
-One step = one pass of the whole path over one batch: pq_transform_quant(X) (rotate +
+One step = one pass of the whole path over one batch: pq_transform_quant(X) (rotate/smooth +
 quantise the activations), pq_pack_weights(W) (rotate + quantise the weights), pq_w4a4_gemm
-(codes -> Y float32).  Default workload: the block-Hadamard q_proj shape, X bf16 [2048, 4096],
-W bf16 [4096, 4096], g = 128 (synthetic, seeded).  L2 is flushed (256 MiB write, then a 256 MiB read) between timed
-steps; each step is timed with CUDA events on the launching stream, and the sum over K steps is
-reduced with MAX over ranks.  N > 1 runs independent replicas (no data-path collective):
-``scaling`` is weak and ``value`` is the total over ranks.
+(codes -> Y float32).  Default workload: the largest configuration, the runtime-smoothing +
+block-Hadamard FFN down-projection, X bf16 [8192, 14336] Laplace(0, 1) with 16 outlier channels,
+W bf16 [4096, 14336], g = 128 (synthetic, seeded).  The same run also measures, under "also",
+the Givens K=16 up-projection (the 4096 x 14336 x 4096 W4A4 GEMM) and the block-Hadamard q_proj
+shape.  L2 is flushed (256 MiB write, then a 256 MiB read) before every timed step; each call is
+timed with CUDA events on the launching stream, and the sum over K steps is reduced with MAX over
+ranks.  N > 1 runs independent replicas (no data-path collective): ``scaling`` is weak and
+``value`` is the total over ranks.
 
-The reference arm (``--impl reference``) times the CPU oracle on this machine's host cores on a
-bounded sample of the same workload, extrapolated to a full step.
+The reference arm (``--impl reference``) times the CPU oracle on this machine's host cores (one
+worker process per core, each on a bounded sample of the same workload) and extrapolates the
+sample to a full step.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -30,12 +36,20 @@ if ROOT not in sys.path:
 
 METRIC = "rotate+quant GB/s (% HBM peak); W4A4 GEMM TOPS (% INT8 tensor peak)"
 UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "down_proj"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # Nominal dense ratio of the contraction's tensor dtype to bf16: the GEMM's MMAs are E4M3
 # (kind::f8f6f4), 4.5 PFLOP/s dense like int8's 4.5 POPS, against 2.25 PFLOP/s for bf16.
 INT8_OVER_BF16 = 4.5 / 2.25
 FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 * 1000 * 1000                     # B200 L2
+# GEMM calls with at most this many tokens are bounded by the weight bytes, not the tensor cores
+# (the crossover at the measured peaks is T ~ 180): they are reported in GB/s against HBM.
+DECODE_T_MAX = 128
+# Kernel sources whose DRAM counters profiles/traffic.json records; a change to any of them
+# makes the recorded traffic stale (reported as null).
+KERNEL_SOURCES = ("rotation_int4_w4a4_b200/csrc/gemm.cu", "rotation_int4_w4a4_b200/csrc/ptx.cuh",
+                  "rotation_int4_w4a4_b200/csrc/rotate_mma.cu", "rotation_int4_w4a4_b200/csrc/transform.cu")
 
 
 def load_peaks():
@@ -48,7 +62,7 @@ def load_peaks():
 
 
 def algorithmic(wl):
-    """Algorithmic bytes / ops per kernel launch for the workload."""
+    """Algorithmic bytes / ops per call for the workload (each figure is per launch of that call)."""
     T, D, N, g = wl.T, wl.D, wl.N, wl.g
     per_elem = 2 + 0.5 + 4.0 / g                     # bf16 in, nibble out, one f32 scale / group
     smooth = 4.0 / g if wl.kind == "smooth_hadamard" else 0.0
@@ -56,8 +70,17 @@ def algorithmic(wl):
         "transform_quant_bytes": T * D * (per_elem + smooth),
         "pack_weights_bytes": N * D * per_elem,
         "gemm_ops": 2.0 * T * N * D,
+        # packed codes and scales of both operands in, float32 Y out
         "gemm_bytes": T * D / 2 + N * D / 2 + (T + N) * (D // g) * 4 + T * N * 4,
     }
+
+
+def sources_digest():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 # ------------------------------------------------------------------------- clocks
@@ -120,48 +143,187 @@ class ClockSampler:
 
 
 # -------------------------------------------------------------------- CPU oracle
-def oracle_sample(wl, x_rows=128, w_rows=1024):
-    """Time the oracle on a bounded sample and extrapolate to one full step (seconds)."""
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+MAX_WORKERS = 64          # oracle worker processes at most (each holds its own float64 sample)
+
+
+def sample_spec(wl, x_rows=128, w_elems=1024 * 4096):
+    """What one oracle sample processes: the first x_rows rows of X (whole 128-row smoothing
+    blocks) and the first rows of W up to about w_elems elements, with the workload's transform
+    parameters.  X and W go to memory-mapped .npy files, so that worker processes share the
+    pages instead of receiving a pickled copy each."""
+    import tempfile
+
+    import numpy as np
+
+    import oracle
+    pairs = oracle.select_pairs(wl.pair_seed, wl.D, wl.g, wl.K, wl.g // 2) if wl.kind == "givens" else None
+    x_rows = min(wl.T, max(x_rows, 128) if wl.kind == "smooth_hadamard" else x_rows)
+    w_rows = min(wl.N, max(64, (w_elems // wl.D) // 64 * 64))
+    d = tempfile.mkdtemp(prefix="pq_oracle_sample_")
+    paths = {}
+    for k, a in (("X", wl.X[:x_rows]), ("W", wl.W[:w_rows])):
+        paths[k] = os.path.join(d, k + ".npy")
+        np.save(paths[k], np.ascontiguousarray(a))
+    return {"kind": wl.kind, "D": wl.D, "g": wl.g, "K": wl.K, "T": wl.T, "N": wl.N,
+            "pairs": pairs, "angles": wl.angles, "beta": wl.beta, "paths": paths, "dir": d,
+            "x_rows": x_rows, "w_rows": w_rows}
+
+
+def drop_spec(spec):
+    for p in spec["paths"].values():
+        try:
+            os.remove(p)
+        except OSError:
+            pass
+    try:
+        os.rmdir(spec["dir"])
+    except OSError:
+        pass
+
+
+def _oracle_sample_worker(spec, barrier=None):
+    """Time the oracle once on the sample (one thread): transform, weight pack, GEMM seconds."""
     import numpy as np
     from threadpoolctl import threadpool_limits
 
     import oracle
-    plan = oracle.Plan(wl.kind, wl.D, wl.g, wl.K, None, wl.angles, wl.beta)
-    if wl.kind == "givens":
-        plan.pairs = oracle.select_pairs(wl.pair_seed, wl.D, wl.g, wl.K, wl.g // 2)
-    xs = wl.X[:max(x_rows, 128) if wl.kind == "smooth_hadamard" else x_rows]
-    ws = wl.W[:w_rows]
+    X = np.array(np.load(spec["paths"]["X"], mmap_mode="r"))
+    W = np.array(np.load(spec["paths"]["W"], mmap_mode="r"))
+    plan = oracle.Plan(spec["kind"], spec["D"], spec["g"], spec["K"], spec["pairs"], spec["angles"], spec["beta"])
+    if barrier is not None:
+        barrier.wait()
     with threadpool_limits(limits=1):
         t0 = time.perf_counter()
-        a = oracle.transform_quant(xs, plan)
+        a = oracle.transform_quant(X, plan)
         t1 = time.perf_counter()
-        w = oracle.pack_weights(ws, plan)
+        w = oracle.pack_weights(W, plan)
         t2 = time.perf_counter()
-        oracle.gemm(a.codes, a.scales, w.codes, w.scales, wl.g)
+        oracle.gemm(a.codes, a.scales, w.codes, w.scales, spec["g"])
         t3 = time.perf_counter()
-    xr = xs.shape[0]
-    full = (t1 - t0) * wl.T / xr + (t2 - t1) * wl.N / w_rows + (t3 - t2) * (wl.T / xr) * (wl.N / w_rows)
-    sample = (f"oracle (numpy float64, 1 thread) on X rows 0..{xr - 1} and W rows 0..{w_rows - 1}: "
-              f"transform {t1 - t0:.3f}s, weight pack {t2 - t1:.3f}s, GEMM {t3 - t2:.3f}s, "
-              f"extrapolated linearly to T={wl.T}, N={wl.N}")
-    return full, t3 - t0, sample
+    return t1 - t0, t2 - t1, t3 - t2
 
 
-def run_reference(args, wl, rank, world):
+def extrapolate(spec, times):
+    """Seconds of one full step from one sample's (transform, pack, GEMM) seconds: the
+    transform scales with the rows of X, the weight pack with the rows of W, the GEMM with
+    their product."""
+    xr, wr = spec["x_rows"], spec["w_rows"]
+    tx, tw, tg = times
+    return tx * spec["T"] / xr + tw * spec["N"] / wr + tg * (spec["T"] / xr) * (spec["N"] / wr)
+
+
+class OraclePool:
+    """One spawned worker process per host core, up to MAX_WORKERS (spawn: safe whatever the
+    parent process has done with CUDA); every worker times the same sample at the same moment."""
+
+    def __init__(self, spec, workers):
+        import multiprocessing as mp
+        self.spec, self.workers = spec, workers
+        ctx = mp.get_context("spawn")
+        self.pool = ctx.Pool(workers) if workers > 1 else None
+        self.mgr = ctx.Manager() if workers > 1 else None
+
+    def run(self):
+        """Returns (per-worker sample seconds (t_x, t_w, t_g), wall seconds of the round)."""
+        if self.pool is None:
+            t0 = time.perf_counter()
+            r = [_oracle_sample_worker(self.spec)]
+            return r, time.perf_counter() - t0
+        barrier = self.mgr.Barrier(self.workers)
+        t0 = time.perf_counter()
+        r = self.pool.starmap(_oracle_sample_worker, [(self.spec, barrier)] * self.workers)
+        return r, time.perf_counter() - t0
+
+    def close(self):
+        if self.pool is not None:
+            self.pool.close()
+            self.pool.join()
+            self.mgr.shutdown()
+
+
+def default_workers():
+    return max(1, min(host_cores(), MAX_WORKERS))
+
+
+def cpu_baseline(wl, workers=None):
+    """The oracle as it stands on this host: one thread, then one worker process per core (up to
+    MAX_WORKERS) at once.  value = the all-core aggregate: every worker is an independent oracle
+    instance, so the host's throughput is the sum of the workers' extrapolated tokens/s."""
+    spec = sample_spec(wl)
+    try:
+        single = _oracle_sample_worker(spec)
+        full1 = extrapolate(spec, single)
+        workers = default_workers() if workers is None else workers
+        pool = OraclePool(spec, workers)
+        try:
+            res, wall = pool.run()
+        finally:
+            pool.close()
+    finally:
+        drop_spec(spec)
+    agg = sum(wl.T / extrapolate(spec, r) for r in res)
+    xr, wr = spec["x_rows"], spec["w_rows"]
+    sample = (f"oracle (numpy float64, BLAS pinned to 1 thread per process) on X rows 0..{xr - 1} and "
+              f"W rows 0..{wr - 1}: one thread: transform {single[0]:.3f}s, weight pack {single[1]:.3f}s, "
+              f"GEMM {single[2]:.3f}s; {workers} processes at once ({host_cores()} host cores): "
+              f"{wall:.2f}s wall; extrapolated linearly to T={wl.T}, N={wl.N}")
+    return {"value": agg, "unit": UNIT, "cores": workers, "kind": "oracle", "sample": sample,
+            "cpu_model": cpu_model(), "host_cores": host_cores(),
+            "single_thread": {"value": wl.T / full1, "unit": UNIT, "cores": 1}}
+
+
+def run_reference(args, wl, rank, world, workers=None):
+    """The reference arm: the oracle on this host's cores (rank 0 only; other ranks exit).
+    Each step is one round of the all-core sample; ms_per_step is that round's wall time and
+    value the tokens/s its extrapolation gives for the full workload."""
     if rank != 0:
         return
-    steps = []
-    for i in range(args.warmup + args.steps):
-        full, spent, sample = oracle_sample(wl)
-        if i >= args.warmup:
-            steps.append(full)
-    total = sum(steps)
-    value = wl.T * len(steps) / total
+    spec = sample_spec(wl)
+    workers = default_workers() if workers is None else workers
+    vals, walls = [], []
+    try:
+        pool = OraclePool(spec, workers)
+        try:
+            for i in range(args.warmup + args.steps):
+                res, wall = pool.run()
+                if i >= args.warmup:
+                    vals.append(sum(wl.T / extrapolate(spec, r) for r in res))
+                    walls.append(wall)
+        finally:
+            pool.close()
+    finally:
+        drop_spec(spec)
+    value = statistics.mean(vals)
+    xr, wr = spec["x_rows"], spec["w_rows"]
+    ms = 1e3 * statistics.mean(walls)
+    sample = (f"oracle (numpy float64, 1 thread per process, {workers} processes) on X rows 0..{xr - 1} "
+              f"and W rows 0..{wr - 1} per process and step, extrapolated linearly to T={wl.T}, N={wl.N}; "
+              f"a step is one such round ({ms:.0f} ms wall)")
     line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(steps),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64 (oracle)", "data": "synthetic (seeded)", "config": config_of(wl, "n/a"),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "dtype": "f64", "data": "synthetic (seeded SplitMix64 generator)",
+            "config": config_of(wl, "n/a (CPU)"),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": workers, "kind": "oracle",
+                             "sample": sample, "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -190,8 +352,7 @@ def job_value(world, tokens_per_rank_step, steps, total_ms):
 
 
 # Kernels one step launches: transform_quant and pack_weights (one each), then the GEMM's own
-# launches as the library reports them for these sizes on the current device (operand
-# expansion and contraction, plus the split-K reduction when it splits the group range).
+# launches as the library reports them for these sizes on the current device.
 LAUNCHES_PER_STEP = 4
 
 
@@ -200,200 +361,20 @@ def launches_per_step(T, N, D):
     return 2 + pq.pq_w4a4_gemm_launch_count(T, N, D)
 
 
+def load_traffic(wl):
+    """DRAM bytes (read + write) per call from the committed ncu summary for this workload, if
+    it was captured from the current kernel sources; otherwise null."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None, "no capture"
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("sources") != sources_digest():
+        return None, "kernel sources changed since the capture"
+    return d.get("calls", {}).get(wl.name), d.get("note", "")
+
+
 # ------------------------------------------------------------------------ GPU arm
-def run_ours(args, wl, rank, world, local_rank):
-    import numpy as np
-    import torch
-    import torch.distributed as dist
-
-    from rotation_int4_w4a4_b200 import pq
-
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    stream = torch.cuda.current_stream()
-
-    def dev_bf16(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
-
-    kind = wl.kind
-    if kind == "givens":
-        pairs = pq.pq_select_pairs(wl.pair_seed, wl.D, wl.g, wl.K, wl.g // 2)
-        plan = pq.Plan("givens", wl.D, K=wl.K, pairs=pairs, angles=wl.angles, beta=wl.beta)
-    else:
-        plan = pq.Plan(kind, wl.D)
-    T, D, N, G = wl.T, wl.D, wl.N, wl.D // wl.g
-    X0, W0 = dev_bf16(wl.X), dev_bf16(wl.W)
-    smooth_w = torch.ones(D, dtype=torch.float32, device=dev) if kind == "smooth_hadamard" else None
-
-    def buffer_set(first):
-        return {"X": X0 if first else X0.clone(), "W": W0 if first else W0.clone(),
-                "ca": torch.empty((T, D // 2), dtype=torch.uint8, device=dev),
-                "sa": torch.empty((T, G), dtype=torch.float32, device=dev),
-                "cw": torch.empty((N, D // 2), dtype=torch.uint8, device=dev),
-                "sw": torch.empty((N, G), dtype=torch.float32, device=dev),
-                "Y": torch.empty((T, N), dtype=torch.float32, device=dev),
-                "sm": torch.empty(((T + 127) // 128, D), dtype=torch.float32, device=dev)
-                if kind == "smooth_hadamard" else None}
-
-    # Cold L2 between steps.  "flush" (default): one set of buffers, and a 256 MiB write + read
-    # between steps.  "rotate": enough complete sets of inputs and outputs that a step's buffers
-    # were last touched over 2 x L2 bytes ago and no other kernel runs between steps (the previous
-    # step's dirty outputs are then written back during the next step).
-    footprint = sum(t.numel() * t.element_size() for t in buffer_set(True).values() if t is not None)
-    nsets = 1 if args.l2 == "flush" else max(2, -(-2 * L2_BYTES // footprint))
-    sets = [buffer_set(i == 0) for i in range(nsets)]
-    flush = L2Flush(dev) if args.l2 == "flush" else (lambda: None)
-    l2_desc = (f"flushed between steps (256 MiB write, then 256 MiB read)" if args.l2 == "flush" else
-               f"cold: {nsets} rotating sets of inputs and outputs ({nsets * footprint / 1e6:.0f} MB "
-               f"working set, > 2 x the 126 MB L2); no other kernel between steps")
-
-    def run_step(bs):
-        pq.pq_transform_quant(plan, bs["X"], bs["ca"], bs["sa"], bs["sm"], stream=stream)
-        pq.pq_pack_weights(plan, bs["W"], bs["cw"], bs["sw"], smooth_w, stream=stream)
-        pq.pq_w4a4_gemm(bs["ca"], bs["sa"], bs["cw"], bs["sw"], bs["Y"], stream=stream)
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-
-    def timed_step(k):
-        bs = sets[(k + offset) % nsets]
-        e = ev[k]
-        e[0].record(stream)
-        pq.pq_transform_quant(plan, bs["X"], bs["ca"], bs["sa"], bs["sm"], stream=stream)
-        e[1].record(stream)
-        pq.pq_pack_weights(plan, bs["W"], bs["cw"], bs["sw"], smooth_w, stream=stream)
-        e[2].record(stream)
-        pq.pq_w4a4_gemm(bs["ca"], bs["sa"], bs["cw"], bs["sw"], bs["Y"], stream=stream)
-        e[3].record(stream)
-
-    for i in range(args.warmup):
-        flush()
-        run_step(sets[i % nsets])
-    torch.cuda.synchronize()
-    pq.pq_check_status(plan)
-
-    vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
-    clocks = ClockSampler(vis[local_rank] if local_rank < len(vis) else str(local_rank))
-    clocks.start()
-    t_roll = time.time()
-    i = 0
-    while time.time() - t_roll < 0.6:            # keep the GPU busy while sampling starts
-        flush()
-        run_step(sets[i % nsets])
-        i += 1
-        torch.cuda.synchronize()
-    offset = i                                   # the first timed step uses the least recent set
-
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    w0 = time.time()
-    for k in range(args.steps):
-        flush()
-        timed_step(k)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    w1 = time.time()
-    t_post = time.time()
-    while time.time() - t_post < 0.4:
-        flush()
-        run_step(sets[i % nsets])
-        i += 1
-        torch.cuda.synchronize()
-    clocks.stop()
-    pq.pq_check_status(plan)
-
-    per = [[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in ev]     # ms
-    step_ms = [sum(p) for p in per]
-    total_ms = max_over_ranks(sum(step_ms), world, dev)
-    tq_ms = statistics.mean(p[0] for p in per)
-    pw_ms = statistics.mean(p[1] for p in per)
-    gm_ms = statistics.mean(p[2] for p in per)
-
-    # ---------------------------------------------------------------- end to end
-    e2e_ms, h2d, d2h = e2e_run(args, wl, pq, plan, dev, stream, flush, sets[0]["sm"], smooth_w)
-    e2e_ms = max_over_ranks(e2e_ms, world, dev)
-
-    if rank != 0:
-        return
-    peaks, peak_src = load_peaks()
-    alg = algorithmic(wl)
-    hbm = peaks["hbm_gbs"]
-    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
-    comps = {
-        "transform_quant": {"us": 1e3 * tq_ms, "GB_s": alg["transform_quant_bytes"] / (tq_ms * 1e-3) / 1e9},
-        "pack_weights": {"us": 1e3 * pw_ms, "GB_s": alg["pack_weights_bytes"] / (pw_ms * 1e-3) / 1e9},
-        "w4a4_gemm": {"us": 1e3 * gm_ms, "TOPS": alg["gemm_ops"] / (gm_ms * 1e-3) / 1e12},
-    }
-    comps["transform_quant"]["frac_hbm"] = comps["transform_quant"]["GB_s"] / hbm
-    comps["pack_weights"]["frac_hbm"] = comps["pack_weights"]["GB_s"] / hbm
-    comps["w4a4_gemm"]["frac_int8"] = comps["w4a4_gemm"]["TOPS"] / int8_peak
-    dominant = max(("transform_quant", tq_ms), ("pack_weights", pw_ms), ("w4a4_gemm", gm_ms), key=lambda kv: kv[1])[0]
-    traffic = load_traffic(dominant, wl)
-    if dominant == "w4a4_gemm":
-        roof = {"bound": "tensor", "achieved": comps[dominant]["TOPS"], "peak": int8_peak, "unit": "TOPS",
-                "frac": comps[dominant]["TOPS"] / int8_peak, "traffic": traffic, "kernel": dominant,
-                "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {INT8_OVER_BF16} "
-                               "(nominal dense fp8 = int8 : bf16 ratio; the MMAs are E4M3)",
-                "algorithmic": f"2*T*N*D = {alg['gemm_ops']:.4g} ops per launch"}
-    else:
-        roof = {"bound": "hbm", "achieved": comps[dominant]["GB_s"], "peak": hbm, "unit": "GB/s",
-                "frac": comps[dominant]["GB_s"] / hbm, "traffic": traffic, "kernel": dominant,
-                "peak_source": f"{peak_src} copy bandwidth"}
-    value = job_value(world, wl.T, args.steps, total_ms)
-    cpu = None
-    if world == 1:
-        full, spent, sample = oracle_sample(wl)
-        cpu = {"value": wl.T / full, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample}
-    ck = clocks.summary(t_roll, time.time())
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in; f32 transform; e4m3 MMA -> f32; f32 out",
-            "data": "synthetic (seeded SplitMix64 generator)",
-            "config": config_of(wl, l2_desc),
-            "components": comps, "roofline": roof, "cpu_baseline": cpu,
-            "e2e": {"value": job_value(world, wl.T, 1, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": launches_per_step(wl.T, wl.N, wl.D) * args.steps, "clocks": ck, "wall_s_timed_region": w1 - w0}
-    print(json.dumps(line), flush=True)
-
-
-def e2e_run(args, wl, pq, plan, dev, stream, flush, sm, smooth_w):
-    """Same step through the public API from pinned host buffers: H2D of X and W, the three
-    calls, D2H of Y, all inside the CUDA-event-timed region."""
-    import numpy as np
-    import torch
-    T, D, N, G = wl.T, wl.D, wl.N, wl.D // wl.g
-    hX = torch.from_numpy(np.ascontiguousarray(wl.X).view(np.int16)).pin_memory()
-    hW = torch.from_numpy(np.ascontiguousarray(wl.W).view(np.int16)).pin_memory()
-    hY = torch.empty((T, N), dtype=torch.float32).pin_memory()
-    dX = torch.empty((T, D), dtype=torch.int16, device=dev)
-    dW = torch.empty((N, D), dtype=torch.int16, device=dev)
-    ca = torch.empty((T, D // 2), dtype=torch.uint8, device=dev)
-    sa = torch.empty((T, G), dtype=torch.float32, device=dev)
-    cw = torch.empty((N, D // 2), dtype=torch.uint8, device=dev)
-    sw = torch.empty((N, G), dtype=torch.float32, device=dev)
-    Y = torch.empty((T, N), dtype=torch.float32, device=dev)
-    total = 0.0
-    n = max(3, min(args.steps, 10))
-    for i in range(args.warmup + n):
-        flush()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        dX.copy_(hX, non_blocking=True)
-        dW.copy_(hW, non_blocking=True)
-        pq.pq_transform_quant(plan, dX, ca, sa, sm, T=T, ldx=D, stream=stream)
-        pq.pq_pack_weights(plan, dW, cw, sw, smooth_w, N=N, stream=stream)
-        pq.pq_w4a4_gemm(ca, sa, cw, sw, Y, stream=stream)
-        hY.copy_(Y, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        if i >= args.warmup:
-            total += e0.elapsed_time(e1)
-    pq.pq_check_status(plan)
-    return total / n, hX.numel() * 2 + hW.numel() * 2, hY.numel() * 4
-
-
 class L2Flush:
     """Evicts this GPU's L2 between timed steps: writes a 256 MiB buffer (twice the 126 MB L2),
     then reads another 256 MiB buffer so that the write's dirty lines are written back before
@@ -411,14 +392,264 @@ class L2Flush:
         torch.sum(self.r, dim=0, out=self.out)
 
 
-def load_traffic(kernel, wl):
-    """DRAM bytes per launch from the committed ncu summary for this kernel and workload, if any."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
-        return None
-    with open(p) as f:
-        d = json.load(f)
-    return d.get(f"{kernel}:{wl.name}")
+def dev_bf16(bits, dev):
+    import numpy as np
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+class Setup:
+    """A workload's plan and device buffers (one or several complete sets)."""
+
+    def __init__(self, wl, dev, l2):
+        import torch
+
+        from rotation_int4_w4a4_b200 import pq
+        self.wl, self.dev, self.pq = wl, dev, pq
+        if wl.kind == "givens":
+            pairs = pq.pq_select_pairs(wl.pair_seed, wl.D, wl.g, wl.K, wl.g // 2)
+            self.plan = pq.Plan("givens", wl.D, K=wl.K, pairs=pairs, angles=wl.angles, beta=wl.beta)
+        else:
+            self.plan = pq.Plan(wl.kind, wl.D)
+        T, D, N, G = wl.T, wl.D, wl.N, wl.D // wl.g
+        self.X0, self.W0 = dev_bf16(wl.X, dev), dev_bf16(wl.W, dev)
+        self.smooth_w = torch.ones(D, dtype=torch.float32, device=dev) if wl.kind == "smooth_hadamard" else None
+
+        def buffer_set(first):
+            return {"X": self.X0 if first else self.X0.clone(), "W": self.W0 if first else self.W0.clone(),
+                    "ca": torch.empty((T, D // 2), dtype=torch.uint8, device=dev),
+                    "sa": torch.empty((T, G), dtype=torch.float32, device=dev),
+                    "cw": torch.empty((N, D // 2), dtype=torch.uint8, device=dev),
+                    "sw": torch.empty((N, G), dtype=torch.float32, device=dev),
+                    "Y": torch.empty((T, N), dtype=torch.float32, device=dev),
+                    "sm": torch.empty(((T + 127) // 128, D), dtype=torch.float32, device=dev)
+                    if wl.kind == "smooth_hadamard" else None}
+
+        # Cold L2 between steps.  "flush" (default): one set of buffers, and a 256 MiB write +
+        # read between steps.  "rotate": enough complete sets of inputs and outputs that a step's
+        # buffers were last touched over 2 x L2 bytes ago and no other kernel runs between steps.
+        footprint = sum(t.numel() * t.element_size() for t in buffer_set(True).values() if t is not None)
+        self.nsets = 1 if l2 == "flush" else max(2, -(-2 * L2_BYTES // footprint))
+        self.sets = [buffer_set(i == 0) for i in range(self.nsets)]
+        self.flush = L2Flush(dev) if l2 == "flush" else (lambda: None)
+        self.l2_desc = ("flushed between steps (256 MiB write, then 256 MiB read)" if l2 == "flush" else
+                        f"cold: {self.nsets} rotating sets of inputs and outputs "
+                        f"({self.nsets * footprint / 1e6:.0f} MB working set, > 2 x the 126 MB L2); "
+                        "no other kernel between steps")
+
+    def calls(self, bs, stream):
+        pq, plan = self.pq, self.plan
+        return (lambda: pq.pq_transform_quant(plan, bs["X"], bs["ca"], bs["sa"], bs["sm"], stream=stream),
+                lambda: pq.pq_pack_weights(plan, bs["W"], bs["cw"], bs["sw"], self.smooth_w, stream=stream),
+                lambda: pq.pq_w4a4_gemm(bs["ca"], bs["sa"], bs["cw"], bs["sw"], bs["Y"], stream=stream))
+
+    def run_step(self, i, stream):
+        for c in self.calls(self.sets[i % self.nsets], stream):
+            c()
+
+    def timed_steps(self, steps, stream, offset=0):
+        """Per step and call, CUDA-event milliseconds on the launching stream (L2 cold first)."""
+        import torch
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+        for k in range(steps):
+            self.flush()
+            calls = self.calls(self.sets[(k + offset) % self.nsets], stream)
+            ev[k][0].record(stream)
+            for j, c in enumerate(calls):
+                c()
+                ev[k][j + 1].record(stream)
+        torch.cuda.synchronize()
+        return [[e[j].elapsed_time(e[j + 1]) for j in range(3)] for e in ev]
+
+    def close(self):
+        self.plan.close()
+
+
+def components(wl, per, peaks):
+    """Per-call times and rates from per-step event times [steps][3] (ms)."""
+    alg = algorithmic(wl)
+    hbm = peaks["hbm_gbs"]
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    tq, pw, gm = (statistics.mean(p[j] for p in per) for j in range(3))
+    comps = {
+        "transform_quant": {"us": 1e3 * tq, "GB_s": alg["transform_quant_bytes"] / (tq * 1e-3) / 1e9},
+        "pack_weights": {"us": 1e3 * pw, "GB_s": alg["pack_weights_bytes"] / (pw * 1e-3) / 1e9},
+        "w4a4_gemm": {"us": 1e3 * gm, "TOPS": alg["gemm_ops"] / (gm * 1e-3) / 1e12,
+                      "GB_s": alg["gemm_bytes"] / (gm * 1e-3) / 1e9},
+    }
+    for k in ("transform_quant", "pack_weights"):
+        comps[k]["frac_hbm"] = comps[k]["GB_s"] / hbm
+    comps["w4a4_gemm"]["frac_int8"] = comps["w4a4_gemm"]["TOPS"] / int8_peak
+    comps["w4a4_gemm"]["frac_hbm"] = comps["w4a4_gemm"]["GB_s"] / hbm
+    comps["w4a4_gemm"]["bound"] = "hbm" if wl.T <= DECODE_T_MAX else "tensor"
+    return comps
+
+
+def roofline_of(wl, comps, peaks, peak_src):
+    """The dominant call against its own bound."""
+    alg = algorithmic(wl)
+    dominant = max(comps, key=lambda k: comps[k]["us"])
+    traffic, tnote = load_traffic(wl)
+    if dominant == "w4a4_gemm" and wl.T > DECODE_T_MAX:
+        int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+        return {"bound": "tensor", "achieved": comps[dominant]["TOPS"], "peak": int8_peak, "unit": "TFLOP/s",
+                "frac": comps[dominant]["TOPS"] / int8_peak,
+                "traffic": traffic.get(dominant) if traffic else None, "traffic_note": tnote,
+                "kernel": "pq_w4a4_gemm (operand expansion + contraction launches)",
+                "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {INT8_OVER_BF16} "
+                               "(nominal dense fp8 = int8 : bf16 ratio; the MMAs are E4M3)",
+                "algorithmic": f"2*T*N*D = {alg['gemm_ops']:.4g} int ops per call"}
+    per_unit = {"transform_quant": alg["transform_quant_bytes"], "pack_weights": alg["pack_weights_bytes"],
+                "w4a4_gemm": alg["gemm_bytes"]}[dominant]
+    return {"bound": "hbm", "achieved": comps[dominant]["GB_s"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": comps[dominant]["GB_s"] / peaks["hbm_gbs"],
+            "traffic": traffic.get(dominant) if traffic else None, "traffic_note": tnote,
+            "kernel": dominant, "peak_source": f"{peak_src} copy bandwidth",
+            "algorithmic": f"{per_unit:.4g} bytes per call"}
+
+
+def e2e_run(args, setup, stream):
+    """Same step through the public API from pinned host buffers: H2D of X and W, the three
+    calls, D2H of Y, all inside the CUDA-event-timed region."""
+    import numpy as np
+    import torch
+    wl, pq, dev = setup.wl, setup.pq, setup.dev
+    T, D, N, G = wl.T, wl.D, wl.N, wl.D // wl.g
+    hX = torch.from_numpy(np.ascontiguousarray(wl.X).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hW = torch.from_numpy(np.ascontiguousarray(wl.W).view(np.int16)).view(torch.bfloat16).pin_memory()
+    hY = torch.empty((T, N), dtype=torch.float32).pin_memory()
+    bs = setup.sets[0]
+    dX, dW = bs["X"], bs["W"]
+    total = 0.0
+    n = max(3, min(args.steps, 10))
+    for i in range(args.warmup + n):
+        setup.flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        dX.copy_(hX, non_blocking=True)
+        dW.copy_(hW, non_blocking=True)
+        pq.pq_transform_quant(setup.plan, dX, bs["ca"], bs["sa"], bs["sm"], stream=stream)
+        pq.pq_pack_weights(setup.plan, dW, bs["cw"], bs["sw"], setup.smooth_w, stream=stream)
+        pq.pq_w4a4_gemm(bs["ca"], bs["sa"], bs["cw"], bs["sw"], bs["Y"], stream=stream)
+        hY.copy_(bs["Y"], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            total += e0.elapsed_time(e1)
+    pq.pq_check_status(setup.plan)
+    return total / n, hX.numel() * 2 + hW.numel() * 2, hY.numel() * 4
+
+
+def measure_also(name, args, dev, stream, peaks, peak_src):
+    """Components of another workload (fewer steps, same method), for the extra keys."""
+    import torch
+
+    from rotation_int4_w4a4_b200 import inputs
+    wl = inputs.workload(name)
+    setup = Setup(wl, dev, "flush")
+    for i in range(max(3, args.warmup)):
+        setup.flush()
+        setup.run_step(i, stream)
+    torch.cuda.synchronize()
+    per = setup.timed_steps(max(5, min(args.steps, 10)), stream)
+    setup.pq.pq_check_status(setup.plan)
+    comps = components(wl, per, peaks)
+    out = {"workload": config_of(wl, setup.l2_desc)["workload"], "T": wl.T, "D": wl.D, "N": wl.N,
+           "components": comps, "roofline": roofline_of(wl, comps, peaks, peak_src),
+           "ms_per_step": statistics.mean(sum(p) for p in per), "tokens_per_s": wl.T / (statistics.mean(sum(p) for p in per) * 1e-3)}
+    setup.close()
+    del setup
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    cpu = None
+    if world == 1 and not args.no_cpu:
+        # Before any CUDA call: the oracle's worker processes are spawned, never forked, but
+        # timing them before the GPU work also keeps the host quiet during the timed region.
+        cpu = cpu_baseline(wl)
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    setup = Setup(wl, dev, args.l2)
+    pq = setup.pq
+
+    for i in range(args.warmup):
+        setup.flush()
+        setup.run_step(i, stream)
+    torch.cuda.synchronize()
+    pq.pq_check_status(setup.plan)
+
+    vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    clocks = ClockSampler(vis[local_rank] if local_rank < len(vis) else str(local_rank))
+    clocks.start()
+    t_roll = time.time()
+    i = 0
+    while time.time() - t_roll < 0.6:            # keep the GPU busy while sampling starts
+        setup.flush()
+        setup.run_step(i, stream)
+        i += 1
+        torch.cuda.synchronize()
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    w0 = time.time()
+    per = setup.timed_steps(args.steps, stream, offset=i)   # the least recently used set first
+    if world > 1:
+        dist.barrier()
+    w1 = time.time()
+    t_post = time.time()
+    while time.time() - t_post < 0.4:
+        setup.flush()
+        setup.run_step(i, stream)
+        i += 1
+        torch.cuda.synchronize()
+    clocks.stop()
+    pq.pq_check_status(setup.plan)
+
+    step_ms = [sum(p) for p in per]
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
+    e2e_ms, h2d, d2h = e2e_run(args, setup, stream)
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
+    launches = launches_per_step(wl.T, wl.N, wl.D) * args.steps
+    setup.close()
+    del setup
+    torch.cuda.empty_cache()
+
+    peaks, peak_src = load_peaks()
+    also = {}
+    if world == 1 and not args.no_also and args.workload == DEFAULT_WORKLOAD and args.T is None:
+        for name in ("up_proj", "q_proj"):
+            also[name] = measure_also(name, args, dev, stream, peaks, peak_src)
+    if rank != 0:
+        return
+    comps = components(wl, per, peaks)
+    roof = roofline_of(wl, comps, peaks, peak_src)
+    ck = clocks.summary(t_roll, time.time())
+    line = {"metric": METRIC, "value": job_value(world, wl.T, args.steps, total_ms), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 in; f32 transform; e4m3 MMA -> f32; f32 out",
+            "data": "synthetic (seeded SplitMix64 generator)",
+            "config": config_of(wl, setup_l2_desc(args)), "components": comps, "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": job_value(world, wl.T, 1, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": launches, "clocks": ck, "wall_s_timed_region": w1 - w0}
+    if also:
+        line["also"] = also
+    print(json.dumps(line), flush=True)
+
+
+def setup_l2_desc(args):
+    return ("flushed between steps (256 MiB write, then 256 MiB read)" if args.l2 == "flush" else
+            "cold: rotating sets of inputs and outputs larger than twice the 126 MB L2")
 
 
 def main():
@@ -427,13 +658,15 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="q_proj")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--N", type=int, default=None, help="sweep workload: 4096 or 14336")
     ap.add_argument("--kind", default=None, help="sweep workload: hadamard or givens")
     ap.add_argument("--l2", choices=["flush", "rotate"], default="flush",
                     help="cold L2 between steps: a 256 MiB write + read (default), or rotating sets "
                          "of inputs and outputs larger than twice the L2")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-also", action="store_true", help="skip the extra workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -153,14 +153,18 @@ pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t N, const f
 
 /*
  * pq_w4a4_gemm — Y[t][n] = sum_G scales_A[t][G] * scales_W[n][G] * d_G[t][n], with
- * d_G = sum over the group's 128 channels of qa * qw computed exactly in int32 on the tensor
- * cores (tcgen05 kind::i8, accumulator in tensor memory), and the per-group scaling applied to
+ * d_G = sum over the group's 128 channels of qa * qw, and the per-group scaling applied to
  * each group's interim result in float32, groups summed in ascending order (RRS page main
  * equation, last line, and Fig. 4 step (3) with block size = group size).
+ *   How d_G is formed: the int4 codes are widened to E4M3 (every integer -8..7 is exact in
+ *   E4M3) and multiplied on the tensor cores by tcgen05.mma kind::f8f6f4 into a float32
+ *   accumulator in tensor memory, one accumulator per group.  Every product is an integer of
+ *   magnitude <= 64 and every partial sum an integer of magnitude <= 128 * 64 = 2^13, so each
+ *   is exact in float32 and d_G arrives exact (no int32 accumulator is involved).
  *   codes_A [T][D/2], scales_A [T][D/g], codes_W [N][D/2], scales_W [N][D/g]: device, dense.
  *   T >= 1, N >= 1 with N % 16 == 0, D % 128 == 0, g == 128.
  *   Y device [T][N] float32 (PQ_OUT_F32) or bf16 (PQ_OUT_BF16, RNE of the float32 result).
- *   Scales must be finite.  Every dot product fits int32 exactly (|d| <= 128*64).
+ *   Scales must be finite.
  *   Returns PQ_ERR_ALLOC if the stream-ordered scratch cannot be allocated.
  *   Output tiles are 256 channels x 256 tokens, one per pair of SMs.  Few tiles (at most half
  *   the SM pairs, e.g. decode shapes): the groups are split into ranges of a multiple of 4
@@ -181,8 +185,14 @@ pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A, const uint
  * reserved nearly all of it for its own caches, or a loop that needs a fixed footprint).  None
  * of the pages has a counterpart: it only changes where the GEMM's temporary int8 operands live.
  *   Scratch: a fixed device array of PQ_NOALLOC_SCRATCH_BYTES inside the library, one per
- *   device, reserved when the CUDA module holding it is loaded (at the latest by the first
- *   call on that device).  No call allocates or frees memory.  It needs no zeroing (each call writes all it reads).
+ *   device, reserved when the CUDA module holding it is loaded on that device and held by
+ *   every process that loads the library until it exits.  With CUDA's lazy module loading (the
+ *   default since CUDA 12.2) that happens at the first call of the library that touches the
+ *   module on the device, which may be this entry's first call: a caller that reserves nearly
+ *   all device memory for itself should make one call on each device before doing so, or run
+ *   with CUDA_MODULE_LOADING=EAGER.  No call allocates or frees memory.  It needs no zeroing:
+ *   each call writes every scratch byte it reads, and the tensor maps bound each operand to
+ *   its own rows, so bytes left by an earlier, larger call are never read.
  *   Limit: (T + N) * D <= PQ_NOALLOC_SCRATCH_BYTES, else PQ_ERR_INVALID_ARG before anything is
  *   launched.
  *   First call on each device: looks up the scratch address with that device current; make it

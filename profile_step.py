@@ -1,6 +1,6 @@
 """Run one workload's hot-path step a few times through the library, for profilers.
 
-    python -m rotation_int4_w4a4_b200.profile_step [--workload q_proj] [--repeat 3]
+    python profile_step.py [--workload q_proj] [--repeat 3]
 
 Each repetition launches, in order, the activation transform (pq_transform_quant), the weight
 transform (pq_pack_weights) and the W4A4 GEMM (pq_w4a4_gemm) on the named synthetic workload,
@@ -11,8 +11,14 @@ step).
 from __future__ import annotations
 
 import argparse
+import os
+import sys
 
 import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
 
 
 def main() -> None:

@@ -89,6 +89,29 @@ def _ptr(x, rows_strided=False):
     return x.data_ptr()
 
 
+def _arg(x, name, dtype, need, rows_strided=False):
+    """Pointer of a tensor argument after checking its dtype and that it holds at least `need`
+    elements (the C ABI only sees a pointer: a wrong dtype or a short buffer would make the
+    kernels read or write past its end).  Raw integer addresses pass unchecked."""
+    if x is None or isinstance(x, int):
+        return _ptr(x)
+    import torch
+    want = {"bf16": (torch.bfloat16,), "u8": (torch.uint8,), "f32": (torch.float32,),
+            "y": (torch.float32, torch.bfloat16)}[dtype]
+    if x.dtype not in want:
+        raise ValueError(f"{name}: dtype {x.dtype} is not accepted (expected {' or '.join(map(str, want))})")
+    p = _ptr(x, rows_strided)
+    if rows_strided:
+        if x.dim() != 2:
+            raise ValueError(f"{name}: expected a 2-D tensor")
+        extent = (x.shape[0] - 1) * x.stride(0) + x.shape[1] if x.shape[0] > 0 else 0
+    else:
+        extent = x.numel()
+    if extent < need:
+        raise ValueError(f"{name}: holds {extent} elements, the call needs {need}")
+    return p
+
+
 def _stream(stream):
     if stream is None:
         import torch
@@ -156,41 +179,60 @@ def pq_transform_quant(plan: Plan, X, codes, scales, smooth_out=None, T=None, ld
     """X bf16 [T, ldx] -> codes uint8 [T, D/2], scales float32 [T, D/g] (device tensors)."""
     T = X.shape[0] if T is None else T
     ldx = X.stride(0) if ldx is None else ldx
-    _check(lib.pq_transform_quant(plan.handle, _ptr(X, rows_strided=True), T, ldx, _ptr(codes), _ptr(scales),
-                                  _ptr(smooth_out), _stream(stream)), "pq_transform_quant")
+    D, G = plan.D, plan.D // plan.g
+    if not isinstance(X, int) and X.dim() == 2 and X.stride(0) != ldx:
+        raise ValueError(f"X: row stride {X.stride(0)} differs from ldx={ldx}")
+    xp = _arg(X, "X", "bf16", (T - 1) * ldx + D if T > 0 else 0, rows_strided=True)
+    _check(lib.pq_transform_quant(plan.handle, xp, T, ldx, _arg(codes, "codes", "u8", T * D // 2),
+                                  _arg(scales, "scales", "f32", T * G),
+                                  _arg(smooth_out, "smooth_out", "f32", -(-T // 128) * D),
+                                  _stream(stream)), "pq_transform_quant")
 
 
 def pq_pack_weights(plan: Plan, W, codes_W, scales_W, smooth_w=None, N=None, stream=None) -> None:
     """W bf16 [N, D] -> codes_W uint8 [N, D/2], scales_W float32 [N, D/g] (device tensors)."""
     N = W.shape[0] if N is None else N
-    _check(lib.pq_pack_weights(plan.handle, _ptr(W), N, _ptr(smooth_w), _ptr(codes_W),
-                               _ptr(scales_W), _stream(stream)), "pq_pack_weights")
+    D, G = plan.D, plan.D // plan.g
+    _check(lib.pq_pack_weights(plan.handle, _arg(W, "W", "bf16", N * D), N,
+                               _arg(smooth_w, "smooth_w", "f32", D),
+                               _arg(codes_W, "codes_W", "u8", N * D // 2),
+                               _arg(scales_W, "scales_W", "f32", N * G), _stream(stream)),
+           "pq_pack_weights")
 
 
 def pq_w4a4_gemm(codes_A, scales_A, codes_W, scales_W, Y, T=None, N=None, D=None, g=128,
                  out_dtype=None, stream=None) -> None:
     """Y [T, N] = per-group scaled int4 x int4 product (device tensors)."""
+    T, N, D, out_dtype, ptrs = _gemm_args(codes_A, scales_A, codes_W, scales_W, Y, T, N, D, g, out_dtype)
+    _check(lib.pq_w4a4_gemm(*ptrs[:4], T, N, D, g, ptrs[4], out_dtype, _stream(stream)), "pq_w4a4_gemm")
+
+
+def _gemm_args(codes_A, scales_A, codes_W, scales_W, Y, T, N, D, g, out_dtype):
+    """Sizes, output dtype and checked pointers shared by the two GEMM entry points."""
     T = codes_A.shape[0] if T is None else T
     N = codes_W.shape[0] if N is None else N
     D = codes_A.shape[1] * 2 if D is None else D
-    if out_dtype is None:
+    if not isinstance(Y, int):
         import torch
-        out_dtype = PQ_OUT_BF16 if Y.dtype == torch.bfloat16 else PQ_OUT_F32
-    _check(lib.pq_w4a4_gemm(_ptr(codes_A), _ptr(scales_A), _ptr(codes_W), _ptr(scales_W),
-                            T, N, D, g, _ptr(Y), out_dtype, _stream(stream)), "pq_w4a4_gemm")
+        y_kind = PQ_OUT_BF16 if Y.dtype == torch.bfloat16 else PQ_OUT_F32
+        if out_dtype is None:
+            out_dtype = y_kind
+        elif out_dtype != y_kind or Y.dtype not in (torch.float32, torch.bfloat16):
+            raise ValueError(f"Y: dtype {Y.dtype} does not match out_dtype={out_dtype}")
+    elif out_dtype is None:
+        out_dtype = PQ_OUT_F32
+    G = D // g if g else 0
+    ptrs = (_arg(codes_A, "codes_A", "u8", T * D // 2), _arg(scales_A, "scales_A", "f32", T * G),
+            _arg(codes_W, "codes_W", "u8", N * D // 2), _arg(scales_W, "scales_W", "f32", N * G),
+            _arg(Y, "Y", "y", T * N))
+    return T, N, D, out_dtype, ptrs
 
 
 def pq_w4a4_gemm_noalloc(codes_A, scales_A, codes_W, scales_W, Y, T=None, N=None, D=None, g=128,
                          out_dtype=None, stream=None) -> None:
     """:func:`pq_w4a4_gemm` with the library's fixed scratch; (T + N) * D <= NOALLOC_SCRATCH_BYTES."""
-    T = codes_A.shape[0] if T is None else T
-    N = codes_W.shape[0] if N is None else N
-    D = codes_A.shape[1] * 2 if D is None else D
-    if out_dtype is None:
-        import torch
-        out_dtype = PQ_OUT_BF16 if Y.dtype == torch.bfloat16 else PQ_OUT_F32
-    _check(lib.pq_w4a4_gemm_noalloc(_ptr(codes_A), _ptr(scales_A), _ptr(codes_W), _ptr(scales_W),
-                                    T, N, D, g, _ptr(Y), out_dtype, _stream(stream)),
+    T, N, D, out_dtype, ptrs = _gemm_args(codes_A, scales_A, codes_W, scales_W, Y, T, N, D, g, out_dtype)
+    _check(lib.pq_w4a4_gemm_noalloc(*ptrs[:4], T, N, D, g, ptrs[4], out_dtype, _stream(stream)),
            "pq_w4a4_gemm_noalloc")
 
 

@@ -45,7 +45,7 @@ def _rank_main(rank, world, port, out_dir):
         wl = inputs.workload("tiny")
         buf = io.StringIO()
         with redirect_stdout(buf):
-            bench.run_reference(args, wl, rank, world)
+            bench.run_reference(args, wl, rank, world, workers=2)
         dist.barrier()
         with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
             json.dump({"max": got, "value": value, "stdout": buf.getvalue()}, f)

@@ -56,6 +56,43 @@ def test_extreme_codes_bit_exact(pq):
     assert np.all(run_gemm(pq, m8, one_a, p7, one_w) == -7168.0)
 
 
+def adversarial_codes(rows, seed):
+    """Codes for one 128-element group whose dot products stress an accumulator of limited
+    alignment precision.  The contraction sees each group as four K32 slices: the low nibbles
+    of packed bytes 0..31 (even elements 0..62), of bytes 32..63 (even elements 64..126), then
+    the high nibbles of bytes 0..31 (odd elements 1..63) and of bytes 32..63 (odd 65..127).
+    Row pattern r % 7 puts large equal-sign codes (-8 or 7) in some slices, so that the running
+    sum reaches several thousand, and small codes (-5..5, odd and even) elsewhere, so that odd
+    products and odd slice sums meet a large partial sum at every slice boundary, in both
+    orders."""
+    rng = np.random.default_rng(seed)
+    slices = [np.arange(0, 64, 2), np.arange(64, 128, 2), np.arange(1, 64, 2), np.arange(65, 128, 2)]
+    big_sets = [(0, 1, 2), (1, 2, 3), (0, 2, 3), (0, 1, 3), (3,), (0,), (0, 1, 2, 3)]
+    q = np.zeros((rows, 128), dtype=np.int8)
+    for r in range(rows):
+        big = big_sets[r % len(big_sets)]
+        sign_big = -8 if (r // len(big_sets)) % 2 == 0 else 7
+        for k, idx in enumerate(slices):
+            if k in big:
+                q[r, idx] = sign_big
+            else:
+                q[r, idx] = rng.integers(-5, 6, idx.size).astype(np.int8)
+    return oracle.pack_nibbles(q)
+
+
+def test_adversarial_dots_bit_exact(pq):
+    """D = 128, unit scales: every output is one group's integer dot.  Row and column patterns
+    combine large slices (|partial sums| up to 96 * 64 = 6144 after three slices and up to
+    8192 in total) with odd products in the other slices; all results must be exact."""
+    T, N = 192, 384
+    ca = adversarial_codes(T, 71)
+    cw = adversarial_codes(N, 72)
+    Y = run_gemm(pq, ca, np.ones((T, 1), np.float32), cw, np.ones((N, 1), np.float32))
+    d = oracle.group_dots(ca, cw, 128)[0]
+    assert np.abs(d).max() == 8192 and np.any((d % 2) != 0) and np.any((np.abs(d) > 5000) & (d % 2 != 0))
+    assert np.array_equal(Y, d.astype(np.float32))
+
+
 @pytest.mark.parametrize("T,N,D", [(3, 16, 256), (200, 272, 384), (128, 256, 1024), (333, 1024, 512)])
 def test_random_codes_f32(pq, T, N, D):
     ca, sa = inputs.random_codes(7 + T, T, D)

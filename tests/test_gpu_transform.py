@@ -201,3 +201,42 @@ def test_full_size_sampled(pq, name):
         assert_scales_close(scales[rows], ref.scales, RTOL_G if wl.kind == "givens" else RTOL_H)
         if smooth:
             assert np.array_equal(sm[b], ref.smooth[0])
+
+
+# ------------------------------------- weights at the workloads' full sizes, sampled rows
+@pytest.mark.parametrize("name", ["q_proj", "up_proj", "down_proj"])
+def test_pack_weights_full_size_sampled(pq, name):
+    """pq_pack_weights on the whole W of each workload, in the launch configuration the
+    benchmark uses, compared with the oracle on sampled rows.
+
+    q_proj    Hadamard, W [4096, 4096] on the tensor cores.
+    up_proj   Givens K=16 (32 groups of weight-side matrices, exp(+beta)), W [14336, 4096].
+    down_proj smoothing + Hadamard, W [4096, 14336] with the register kernel's multi-task loop;
+              the channel multiplier is the oracle's own smoothing scale of X's first 128-row
+              block (the workload's pre-scaled weights), as float32.
+    """
+    import torch
+    wl = inputs.workload(name)
+    D, N = wl.D, wl.N
+    smooth_w = None
+    if wl.kind == "givens":
+        pairs, angles, beta = givens_inputs(wl)
+        plan = pq.Plan("givens", D, K=wl.K, pairs=pairs, angles=angles, beta=beta)
+        oplan = oracle_plan("givens", D, wl.K, pairs, angles, beta)
+    else:
+        plan = pq.Plan(wl.kind, D)
+        oplan = oracle_plan(wl.kind, D)
+        if wl.kind == "smooth_hadamard":
+            smooth_w = oracle.smooth_scales(oracle.bf16_to_f64(wl.X[:128]), 128)[0].astype(np.float32)
+    codes, scales = empty_outputs(N, D)
+    pq.pq_pack_weights(plan, to_dev_bf16(wl.W), codes, scales,
+                       to_dev(smooth_w) if smooth_w is not None else None)
+    pq.pq_check_status(plan)
+    rng = np.random.default_rng(17)
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, N // 2, N // 2 + 77, N - 1],
+                                     rng.integers(0, N, 9)]))
+    rt = torch.from_numpy(rows).cuda()
+    ref = oracle.pack_weights(wl.W[rows], oplan, smooth_w)
+    assert_codes_match(codes[rt].cpu().numpy(), ref)
+    assert_scales_close(scales[rt].cpu().numpy(), ref.scales,
+                        RTOL_G if wl.kind == "givens" else 2 * RTOL_H)

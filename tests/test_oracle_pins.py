@@ -141,6 +141,63 @@ def test_givens_layers_match_explicit_product_and_are_orthogonal():
     assert np.max(np.abs(back - x)) < 1e-12
 
 
+# ----------------------------------------------------- channel scale (ParoQuant §2.3)
+def _identity_pairs_plan(beta, K=2, G=2, g=128):
+    """A Givens plan whose every slot is empty: the rotations are the identity, so only the
+    channel scale acts."""
+    pairs = np.full((G, K, g // 2, 2), oracle.NONE, dtype=np.uint8)
+    angles = np.zeros((G, K, g // 2), dtype=np.float32)
+    return oracle.Plan("givens", G * g, g, K, pairs, angles, beta)
+
+
+def test_channel_scale_direction_closed_form():
+    """ParoQuant page §2.3 fixes W^ = diag(alpha) W with alpha = exp(beta), alpha one factor
+    per input channel: the weights are multiplied by exp(+beta) and, for the product to be
+    unchanged, the activations by exp(-beta).  With no rotation this is the whole transform."""
+    beta = (rng(12).standard_normal(256) * 0.7).astype(np.float32)
+    plan = _identity_pairs_plan(beta)
+    x = rng(13).standard_normal((5, 256))
+    w = rng(14).standard_normal((7, 256))
+    e = np.exp(beta.astype(np.float64))
+    y, s = oracle.activation_transform(x, plan)
+    assert s is None
+    assert np.allclose(y, x / e, rtol=1e-15, atol=0)
+    assert np.allclose(oracle.weight_transform(w, plan), w * e, rtol=1e-15, atol=0)
+    # A channel with beta = ln 2 exactly halves the activation and doubles the weight.
+    b2 = np.zeros(256, dtype=np.float32)
+    b2[9] = np.float32(math.log(2.0))
+    p2 = _identity_pairs_plan(b2)
+    one = np.ones((1, 256))
+    ya, _ = oracle.activation_transform(one, p2)
+    yw = oracle.weight_transform(one, p2)
+    assert ya[0, 9] == pytest.approx(0.5, rel=1e-7) and yw[0, 9] == pytest.approx(2.0, rel=1e-7)
+    assert np.all(np.delete(ya[0], 9) == 1.0) and np.all(np.delete(yw[0], 9) == 1.0)
+
+
+def test_channel_scale_follows_the_rotations():
+    """Reading: the channel scale is applied after the K layers (y = (x G_0 ... G_{K-1})
+    diag(exp(-beta))).  One pair (5, 77) rotated by theta and a scale on channel 77 only:
+    e_5 goes to (cos, sin) on (5, 77) and then channel 77 alone is divided by exp(beta_77)."""
+    g = 128
+    th = np.float32(0.9)
+    pairs, angles = one_pair_plan(5, 77, th)
+    beta = np.zeros(g, dtype=np.float32)
+    beta[77] = np.float32(0.5)
+    plan = oracle.Plan("givens", g, g, 1, pairs, angles, beta)
+    e5 = np.zeros((1, g))
+    e5[0, 5] = 1.0
+    y, _ = oracle.activation_transform(e5, plan)
+    c, s = math.cos(float(th)), math.sin(float(th))
+    assert y[0, 5] == pytest.approx(c, abs=1e-15)
+    assert y[0, 77] == pytest.approx(s * math.exp(-0.5), abs=1e-15)
+    # scale-then-rotate would have mixed the scaled channel 77 back into channel 5
+    e77 = np.zeros((1, g))
+    e77[0, 77] = 1.0
+    y77, _ = oracle.activation_transform(e77, plan)
+    assert y77[0, 5] == pytest.approx(-s, abs=1e-15)
+    assert y77[0, 77] == pytest.approx(c * math.exp(-0.5), abs=1e-15)
+
+
 # -------------------------------------------------------------- pair selection (A1)
 @pytest.mark.parametrize("K,N", [(8, 64), (16, 64), (4, 20)])
 def test_select_pairs_properties(K, N):
@@ -366,6 +423,27 @@ def _q8(orig):
     return f
 
 
+def _negated_beta(orig):
+    """Mutant: the same transform with beta replaced by -beta (flips the side that carries
+    exp(+beta); applied to both sides the product x w^T is unchanged)."""
+    def f(a, plan, *rest):
+        flipped = oracle.Plan(plan.kind, plan.D, plan.g, plan.K, plan.pairs, plan.angles,
+                              None if plan.beta is None else -plan.beta, plan.smooth_after_rotate)
+        return orig(a, flipped, *rest)
+    return f
+
+
+def _scale_first(orig, sign):
+    """Mutant: Givens applies exp(sign * beta) before the rotations instead of after them
+    (on both sides the product x w^T is again unchanged)."""
+    def f(a, plan, *rest):
+        if plan.kind != "givens" or plan.beta is None:
+            return orig(a, plan, *rest)
+        y = O.givens_rotate(a * np.exp(sign * plan.beta.astype(np.float64)), plan.pairs, plan.angles, plan.g)
+        return (y, None) if sign < 0 else y
+    return f
+
+
 MUTANTS = {
     "givens_sign_swapped": (
         "givens_rotate",
@@ -382,6 +460,16 @@ MUTANTS = {
             plan.kind, plan.D, plan.g, plan.K, plan.pairs, plan.angles,
             None if plan.beta is None else -plan.beta, plan.smooth_after_rotate), sw)),
         lambda: test_equivalence_before_quantisation(1)),
+    # exp(+beta) on the activations and exp(-beta) on the weights: the product is unchanged,
+    # so only the closed form of the page's W^ = diag(exp(beta)) W can catch it.
+    "channel_scale_both_sides_flipped": (
+        ("activation_transform", "weight_transform"),
+        (lambda orig: _negated_beta(orig), lambda orig: _negated_beta(orig)),
+        test_channel_scale_direction_closed_form),
+    "channel_scale_before_rotation": (
+        ("activation_transform", "weight_transform"),
+        (lambda orig: _scale_first(orig, -1.0), lambda orig: _scale_first(orig, +1.0)),
+        test_channel_scale_follows_the_rotations),
     "weight_rotation_transposed": (
         "weight_transform",
         lambda orig: (lambda w, plan, sw=None: orig(w, plan, sw) if plan.kind != "givens" else
@@ -406,8 +494,23 @@ MUTANTS = {
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_catch_planted_mistakes(name, monkeypatch):
-    attr, make, pin = MUTANTS[name]
-    orig = getattr(O, attr)
-    monkeypatch.setattr(O, attr, make(orig))
-    monkeypatch.setattr(oracle, attr, getattr(O, attr))
+    attrs, makes, pin = MUTANTS[name]
+    if isinstance(attrs, str):
+        attrs, makes = (attrs,), (makes,)
+    for attr, make in zip(attrs, makes):
+        orig = getattr(O, attr)
+        monkeypatch.setattr(O, attr, make(orig))
+        monkeypatch.setattr(oracle, attr, getattr(O, attr))
     assert _fails(pin), f"pin did not catch mutant {name}"
+
+
+@pytest.mark.parametrize("name", ["channel_scale_both_sides_flipped", "channel_scale_before_rotation"])
+def test_two_sided_mutants_keep_the_product(name, monkeypatch):
+    """The two-sided channel-scale mutants leave (x M)(w M^-T)^T = x w^T intact, so the
+    equivalence pin alone cannot see them: only the closed forms above can."""
+    attrs, makes, _ = MUTANTS[name]
+    for attr, make in zip(attrs, makes):
+        orig = getattr(O, attr)
+        monkeypatch.setattr(O, attr, make(orig))
+        monkeypatch.setattr(oracle, attr, getattr(O, attr))
+    test_equivalence_before_quantisation(1)

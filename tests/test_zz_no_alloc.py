@@ -1,9 +1,10 @@
 """pq_w4a4_gemm_noalloc: the W4A4 GEMM with the library's fixed device-array scratch.
 
 Collected last on purpose, so that it also runs after every other test has used the allocating
-entry point on the same device.  Two calls in a row on one stream (different shapes and data)
-must each match pq_w4a4_gemm on the same inputs within the GEMM's float32 tolerance; sizes
-beyond the fixed scratch are rejected before anything reaches the device.
+entry point on the same device.  Two calls in a row on one stream (a larger call, then a smaller
+one with ragged T and N) must each match pq_w4a4_gemm on the same inputs within the GEMM's
+float32 tolerance; sizes beyond the fixed scratch are rejected before anything reaches the
+device.
 """
 import ctypes
 
@@ -42,7 +43,12 @@ def test_rejects_sizes_beyond_the_fixed_scratch(pq):
 @pytest.mark.gpu
 def test_two_calls_match_the_allocating_entry(pq):
     import torch
-    cases = [(300, 256, 512, torch.float32, 11), (130, 768, 384, torch.bfloat16, 12)]
+    # The larger call runs first and leaves its operand bytes in the shared scratch; the second,
+    # smaller call has T and N that are not multiples of the 256-wide tile, so its last tiles
+    # reach past its own operands into bytes the first call wrote.  The tensor maps' bounds must
+    # keep those bytes out of its result.
+    cases = [(600, 1024, 1024, torch.float32, 11), (130, 272, 384, torch.bfloat16, 12)]
+    assert (cases[0][0] + cases[0][1]) * cases[0][2] > (cases[1][0] + cases[1][1]) * cases[1][2]
     data = []
     for T, N, D, dt, seed in cases:
         ca, sa = inputs.random_codes(seed, T, D)
