@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <string>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/pq.h"
@@ -82,11 +83,19 @@ inline int device_sm_count() {
   return c;
 }
 
-// Kernel launchers (transform.cu, gemm.cu).  Arguments are already validated.
-// y = ((x * pre) H) * post per row-group (pre/post per channel, either may be null).
-cudaError_t launch_hadamard_rows(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx,
-                                 const float* pre_scale, const float* post_scale,
-                                 uint8_t* codes, float* scales, cudaStream_t stream);
+// Kernel launchers (transform.cu, smooth_rows.cu, rotate_mma.cu, gemm.cu).  Arguments are
+// already validated.
+// Tensor map of a bf16 [rows][inner] matrix (row stride ld elements): 64 x 128 boxes, 128-byte
+// swizzle, zero fill outside (rotate_mma.cu).
+cudaError_t make_bf16_tile_map(CUtensorMap* map, const void* base, int64_t rows, int64_t inner, int64_t ld);
+// y = ((x * a) H) * b per row and group, one thread per row (smooth_rows.cu).  mode 0: a = 1/s with
+// s the per-channel max |x| over each 128-row block (to smooth_out if non-null); 1: a = vec;
+// 2: b = vec; 3: neither.
+enum { PQ_SR_COLMAX = 0, PQ_SR_PRE = 1, PQ_SR_POST = 2, PQ_SR_NONE = 3 };
+cudaError_t launch_smooth_rows(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int mode,
+                               const float* vec, uint8_t* codes, float* scales, float* smooth_out,
+                               cudaStream_t stream);
+// Runtime smoothing after the rotation (PQ_FLAG_SMOOTH_AFTER_ROTATE activations; transform.cu).
 cudaError_t launch_smooth_hadamard(const pq_plan* plan, const void* X, int64_t T, int64_t ldx,
                                    uint8_t* codes, float* scales, float* smooth_out,
                                    cudaStream_t stream);

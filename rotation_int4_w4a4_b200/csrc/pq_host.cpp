@@ -312,7 +312,10 @@ extern "C" pq_status pq_transform_quant(const pq_plan* plan, const void* X, int6
       e = launch_rotate_mma(plan, X, T, ldx, 0, codes, scales, s);
       break;
     case PQ_SMOOTH_HADAMARD:
-      e = launch_smooth_hadamard(plan, X, T, ldx, codes, scales, smooth_out, s);
+      if (plan->flags & PQ_FLAG_SMOOTH_AFTER_ROTATE)
+        e = launch_smooth_hadamard(plan, X, T, ldx, codes, scales, smooth_out, s);
+      else
+        e = launch_smooth_rows(plan, X, T, ldx, PQ_SR_COLMAX, nullptr, codes, scales, smooth_out, s);
       break;
   }
   return cuda_fail(e, "pq_transform_quant launch");
@@ -346,10 +349,12 @@ extern "C" pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t
       e = launch_rotate_mma(plan, W, N, plan->D, 1, codes_W, scales_W, s);
       break;
     case PQ_SMOOTH_HADAMARD:
-      if (plan->flags & PQ_FLAG_SMOOTH_AFTER_ROTATE)
-        e = launch_hadamard_rows(plan, W, N, plan->D, nullptr, smooth_w, codes_W, scales_W, s);
+      if (!smooth_w)
+        e = launch_smooth_rows(plan, W, N, plan->D, PQ_SR_NONE, nullptr, codes_W, scales_W, nullptr, s);
+      else if (plan->flags & PQ_FLAG_SMOOTH_AFTER_ROTATE)
+        e = launch_smooth_rows(plan, W, N, plan->D, PQ_SR_POST, smooth_w, codes_W, scales_W, nullptr, s);
       else
-        e = launch_hadamard_rows(plan, W, N, plan->D, smooth_w, nullptr, codes_W, scales_W, s);
+        e = launch_smooth_rows(plan, W, N, plan->D, PQ_SR_PRE, smooth_w, codes_W, scales_W, nullptr, s);
       break;
   }
   return cuda_fail(e, "pq_pack_weights launch");

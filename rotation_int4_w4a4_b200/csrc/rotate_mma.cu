@@ -278,8 +278,10 @@ EncodeTiledFnR encode_fn_r() {
   return fn;
 }
 
+}  // namespace
+
 // bf16 [rows][inner] (row stride ld elements) with a box of 64 x 128 and 128-byte swizzle.
-cudaError_t make_bf16_map(CUtensorMap* map, const void* base, int64_t rows, int64_t inner, int64_t ld) {
+cudaError_t make_bf16_tile_map(CUtensorMap* map, const void* base, int64_t rows, int64_t inner, int64_t ld) {
   EncodeTiledFnR enc = encode_fn_r();
   if (!enc) return cudaErrorNotSupported;
   cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
@@ -292,8 +294,6 @@ cudaError_t make_bf16_map(CUtensorMap* map, const void* base, int64_t rows, int6
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-}  // namespace
-
 cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
                               uint8_t* codes, float* scales, cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
@@ -301,10 +301,10 @@ cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, 
   const int terms = givens ? 2 : 1;
   const int r_groups = givens ? plan->G : 1;
   CUtensorMap tmX, tmR;
-  cudaError_t e = make_bf16_map(&tmX, X, rows, plan->D, ldx);
+  cudaError_t e = make_bf16_tile_map(&tmX, X, rows, plan->D, ldx);
   if (e != cudaSuccess) return e;
   const uint16_t* R = plan->d_rot + (size_t)(weights && givens ? 1 : 0) * r_groups * terms * RT_N * 128;
-  e = make_bf16_map(&tmR, R, (int64_t)r_groups * terms * RT_N, 128, 128);
+  e = make_bf16_tile_map(&tmR, R, (int64_t)r_groups * terms * RT_N, 128, 128);
   if (e != cudaSuccess) return e;
   const int row_blocks = (int)((rows + RT_M - 1) / RT_M);
   const int64_t tiles = (int64_t)row_blocks * plan->G;

@@ -1,14 +1,14 @@
-// Fused rotate / scale / smooth + per-group INT4 quantisation kernels (sm_100a).
-//
-// ParoQuant page §3.2: rotation, scaling and quantisation are one kernel, so each element is
-// read once from HBM (bf16, 2 B) and written once (a nibble), plus one float scale per group.
+// Runtime smoothing in the RRS page's order (rotate, then smooth the rotated channels) + per-group
+// INT4 quantisation, on a 128-row x 128-channel tile per CTA (sm_100a).  The other order and the
+// weight transforms run in smooth_rows.cu.
 //
 // Block Hadamard (Hadamard page §2.1/§4.2/§6.1, RRS page R = (1/sqrt(K))[s_ij]): a 128-channel
 // group is held by 4 lanes, 32 consecutive channels each (four 16-byte loads per lane).  H_128
 // = H_4 (x) H_32 in Sylvester order: channel bits 0..4 are transformed in registers (5 radix-2
 // stages), bits 5..6 across the 4 lanes with two xor-shuffle stages.  The 1/sqrt(128) factor
 // never touches the data: the codes do not depend on a uniform factor, so it is folded into the
-// stored scale.
+// stored scale.  The rotated channels' maxima over the tile's rows are combined across lanes
+// and warps, which needs every row of the tile in the CTA's registers at once.
 //
 // Quantisation (RRS page: alpha = max|X| / 7, codes in -8..7, RTN): m = max|y| over the group
 // (two xor-shuffles), inv = 7/m, q = RNE(y * inv) by one FMA with 1.5 * 2^23, whose low 4 bits
@@ -119,84 +119,6 @@ __device__ __forceinline__ uint32_t quant_pack8(const float* v, float inv) {
 __device__ __forceinline__ uint4 quant_pack32(const float (&v)[32], float inv) {
   return make_uint4(quant_pack8(v, inv), quant_pack8(v + 8, inv), quant_pack8(v + 16, inv),
                     quant_pack8(v + 24, inv));
-}
-
-__device__ __forceinline__ void scale32(float (&v)[32], const float* s) {
-  const float4* p = reinterpret_cast<const float4*>(s);
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float4 f = __ldg(p + k);
-    v[4 * k] *= f.x;
-    v[4 * k + 1] *= f.y;
-    v[4 * k + 2] *= f.z;
-    v[4 * k + 3] *= f.w;
-  }
-}
-
-// ---------------------------------------------------------------------------------------
-// Flat stream of row-groups (row t, group gi), 8 per warp-task, tasks strided over the grid.
-// y = ((x * pre) H) * post.  The next task's four 16-byte loads are issued before the current
-// task is transformed, so each warp keeps 2 KB in flight while it computes.
-__global__ void __launch_bounds__(256) hadamard_rows_kernel(
-    const __nv_bfloat16* __restrict__ X, int64_t rows, int64_t ldx, int G,
-    const float* __restrict__ pre, const float* __restrict__ post, uint8_t* __restrict__ codes,
-    float* __restrict__ scales) {
-  const int lane = threadIdx.x & 31;
-  const int q = lane & 3;
-  const int64_t R = rows * (int64_t)G;
-  const int64_t ntasks = (R + 7) / 8;
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (task >= ntasks) return;
-  const int64_t halfD = (int64_t)G * 64;
-  // This lane's row-group r = 8 task + lane/4, kept as (t, gi) and advanced incrementally.
-  const int64_t stride = nwarps * 8;
-  const int64_t st_t = stride / G;
-  const int st_g = (int)(stride - st_t * G);
-  int64_t r = task * 8 + (lane >> 2);
-  int64_t t = r / G;
-  int gi = (int)(r - t * G);
-  uint4 cur[4], nxt[4];
-  auto load = [&](int64_t rr, int64_t tt, int gg, uint4 (&dst)[4]) {
-    if (rr < R) {
-      const uint4* p = reinterpret_cast<const uint4*>(X + tt * ldx + gg * 128 + q * 32);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dst[j] = ld_stream(p + j);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dst[j] = make_uint4(0, 0, 0, 0);
-    }
-  };
-  load(r, t, gi, cur);
-  for (;;) {
-    const int64_t ntask = task + nwarps;
-    int64_t nr = r + stride, nt = t + st_t;
-    int ng = gi + st_g;
-    if (ng >= G) { ng -= G; ++nt; }
-    const bool more = ntask < ntasks;                  // warp-uniform
-    if (more) load(nr, nt, ng, nxt);
-    const int c0 = gi * 128 + q * 32;
-    float v[32];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) bf16x8_to_f32(cur[j], v + 8 * j);
-    if (pre) scale32(v, pre + c0);
-    fwht32(v);
-    fwht_across4(v, lane);
-    if (post) scale32(v, post + c0);
-    const float m = group_max4(absmax32(v));
-    const uint4 packed = quant_pack32(v, quant_inv(m));
-    if (r < R) {
-      *reinterpret_cast<uint4*>(codes + t * halfD + gi * 64 + q * 16) = packed;
-      if (q == 0) scales[r] = m * kScaleHadamard;
-    }
-    if (!more) break;
-    task = ntask;
-    r = nr;
-    t = nt;
-    gi = ng;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
-  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -324,30 +246,6 @@ __global__ void __launch_bounds__(128, 4) smooth_hadamard_kernel(
 }
 
 }  // namespace
-
-cudaError_t launch_hadamard_rows(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx,
-                                 const float* pre_scale, const float* post_scale, uint8_t* codes,
-                                 float* scales, cudaStream_t stream) {
-  const int64_t R = rows * plan->G;
-  const int64_t tasks = (R + 7) / 8;                // one warp-task = 8 row-groups
-  const int64_t want = (tasks + 7) / 8;             // 8 warps per block
-  static std::atomic<int> per_sm_cache{0};           // a property of the kernel binary
-  int per_sm = per_sm_cache.load(std::memory_order_relaxed);
-  if (per_sm < 1) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hadamard_rows_kernel, 256, 0) != cudaSuccess ||
-        per_sm < 1)
-      per_sm = 2;
-    per_sm_cache.store(per_sm, std::memory_order_relaxed);
-  }
-  const int64_t cap = (int64_t)device_sm_count() * per_sm;  // one resident wave, tasks strided over it
-  const int grid = (int)(want < cap ? want : cap);
-  static std::atomic<bool> attr_done[kMaxDevices];
-  cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(hadamard_rows_kernel), 0, attr_done);
-  if (e != cudaSuccess) return e;
-  hadamard_rows_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(X), rows,
-                                                 ldx, plan->G, pre_scale, post_scale, codes, scales);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_smooth_hadamard(const pq_plan* plan, const void* X, int64_t T, int64_t ldx,
                                    uint8_t* codes, float* scales, float* smooth_out,
