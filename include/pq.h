@@ -32,10 +32,10 @@
  *   16-byte aligned.  The library allocates no user-visible buffer.  A plan owns a few small
  *   device tables and a status word, allocated by pq_make_plan and freed by pq_destroy_plan;
  *   it is immutable after creation and may be used from several streams at once.
- *   pq_w4a4_gemm takes (T + N) * D bytes (more when split, see there) of temporary scratch per
- *   call from a library-owned, stream-ordered memory pool on the current device and returns it
- *   on the same stream; the pool keeps freed memory for reuse, so it holds about the largest
- *   single call's need.
+ *   pq_w4a4_gemm takes (T + N) * D bytes (T > 128; more when split, see there) of temporary
+ *   scratch per call from a library-owned, stream-ordered memory pool on the current device and
+ *   returns it on the same stream; the pool keeps freed memory for reuse, so it holds about the
+ *   largest single call's need.  Calls with T <= 128 take none unless they split.
  *
  * Errors
  *   Every call returns pq_status and never throws, aborts or exits.  Arguments are validated
@@ -166,11 +166,18 @@ pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t N, const f
  *   Y device [T][N] float32 (PQ_OUT_F32) or bf16 (PQ_OUT_BF16, RNE of the float32 result).
  *   Scales must be finite.
  *   Returns PQ_ERR_ALLOC if the stream-ordered scratch cannot be allocated.
- *   Output tiles are 256 channels x 256 tokens, one per pair of SMs.  Few tiles (at most half
- *   the SM pairs, e.g. decode shapes): the groups are split into ranges of a multiple of 4
- *   handled by different SM pairs, and the float32 partial results are
- *   added in ascending range order (4 * ranges * T * N extra scratch bytes); the result differs
- *   from the unsplit order only by float32 rounding.
+ *   T > 128: the codes are first widened to E4M3 into (T + N) * D bytes of scratch; output
+ *   tiles are 256 channels x 256 tokens, one per pair of SMs.  Few tiles (at most half the SM
+ *   pairs): the groups are split into ranges of a multiple of 4 handled by different SM pairs,
+ *   and the float32 partial results are added in ascending range order (4 * ranges * T * N
+ *   extra scratch bytes).
+ *   T <= 128 (decode): the packed codes are read directly (no operand scratch) and widened to
+ *   int8 q * 16 inside the kernel; tcgen05.mma kind::i8 forms 256 d_G exactly in int32 and the
+ *   epilogue applies sw / 256 (exact) and sa, giving the same per-group float32 values.  One
+ *   kernel writes Y, unless the 128-row weight tiles are too few to fill the device: then the
+ *   groups are split into ranges and their float32 partial tiles (4 * ranges * T * N scratch
+ *   bytes) are added in ascending range order by a second kernel.
+ *   A split result differs from the unsplit order only by float32 rounding.
  */
 pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                        const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
@@ -210,9 +217,10 @@ pq_status pq_w4a4_gemm_noalloc(const uint8_t* codes_A, const float* scales_A,
 /*
  * pq_w4a4_gemm_launch_count — host-only query, no counterpart in the pages.  Writes to
  * *launches the number of kernels one pq_w4a4_gemm call with these sizes launches on the
- * current device: 2 (operand expansion, contraction) or 3 (plus the split-K reduction, chosen
- * when the 256 x 256 output tiles fill at most half of the device's SM pairs).
- * pq_w4a4_gemm_noalloc never splits and always launches 2.  Sizes are validated as for
+ * current device.  T > 128: 2 (operand expansion, contraction) or 3 (plus the split-K
+ * reduction, chosen when the 256 x 256 output tiles fill at most half of the device's SM
+ * pairs).  T <= 128: 1, or 2 with the group-range reduction.  pq_w4a4_gemm_noalloc never
+ * splits: it launches 2 for T > 128 and 1 otherwise.  Sizes are validated as for
  * pq_w4a4_gemm (PQ_ERR_INVALID_ARG otherwise).  Without a usable device the count assumes 148 SMs.
  */
 pq_status pq_w4a4_gemm_launch_count(int64_t T, int64_t N, int64_t D, int* launches);

@@ -651,10 +651,14 @@ pq_status gemm_max_pairs(int sms, int* out) {
 
 }  // namespace
 
-size_t gemm_scratch_bytes(int64_t T, int64_t N, int64_t D) { return (size_t)(T + N) * (size_t)D; }
+size_t gemm_scratch_bytes(int64_t T, int64_t N, int64_t D) {
+  return T <= kGemmSmallT ? 0 : (size_t)(T + N) * (size_t)D;
+}
 
-// Split-K when the tiles fill at most half of the CTA pairs the device can run at once.
+// Few tokens: the few-token kernel's group ranges.  Otherwise split-K when the tiles fill at most
+// half of the CTA pairs the device can run at once.
 int gemm_ksplit(int64_t T, int64_t N, int64_t D, int* gs_out) {
+  if (T <= kGemmSmallT) return gemm_small_ranges(T, N, D, gs_out);
   const int G = (int)(D / 128);
   const int64_t tiles = ((N + PAIR_M - 1) / PAIR_M) * ((T + BN - 1) / BN);
   const int pairs = device_sm_count() / 2;
@@ -674,9 +678,21 @@ size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t D) {
   return ks > 1 ? (size_t)ks * (size_t)T * (size_t)N * sizeof(float) : 0;
 }
 
+pq_status launch_splitk_reduce(const float* ws, int ksplit, int64_t T, int64_t N, void* Y, int out_bf16,
+                               cudaStream_t stream) {
+  const int64_t n4 = T * N / 4;                              // N % 16 == 0
+  const int64_t rwant = (n4 + 255) / 256;
+  const int64_t cap = (int64_t)device_sm_count() * 8;
+  const int rgrid = (int)(rwant < cap ? rwant : cap);
+  splitk_reduce_kernel<<<rgrid, 256, 0, stream>>>(reinterpret_cast<const float4*>(ws), ksplit, n4, Y, out_bf16);
+  return cuda_fail(cudaGetLastError(), "splitk_reduce_kernel launch");
+}
+
 pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W, const float* scales_W,
                       int64_t T, int64_t N, int64_t D, void* Y, pq_out_dtype out_dtype, uint8_t* scratch,
                       float* ws, unsigned int* status, cudaStream_t stream) {
+  if (T <= kGemmSmallT)
+    return gemm_small_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype, ws, status, stream);
   uint8_t* A8 = scratch;
   uint8_t* W8 = scratch + (size_t)T * (size_t)D;
   // MMA operand A = weights (M = output channels), B = activations (N = tokens).
@@ -735,15 +751,7 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
                                                                m_tiles, n_tiles, ksplit, gs, ws, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel launch");
-  if (ksplit > 1) {
-    const int64_t n4 = T * N / 4;                              // N % 16 == 0
-    const int64_t rwant = (n4 + 255) / 256;
-    const int rgrid = (int)(rwant < (int64_t)sms * 8 ? rwant : (int64_t)sms * 8);
-    splitk_reduce_kernel<<<rgrid, 256, 0, stream>>>(reinterpret_cast<const float4*>(ws), ksplit, n4, Y,
-                                                    out_dtype == PQ_OUT_BF16 ? 1 : 0);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "splitk_reduce_kernel launch");
-  }
+  if (ksplit > 1) return launch_splitk_reduce(ws, ksplit, T, N, Y, out_dtype == PQ_OUT_BF16 ? 1 : 0, stream);
   return PQ_OK;
 }
 
@@ -760,6 +768,8 @@ pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t*
   // Operand scratch, then (small problems) the split-K partial tiles.
   const size_t op_bytes = (gemm_scratch_bytes(T, N, D) + 255) & ~(size_t)255;
   const size_t ws_bytes = gemm_workspace_bytes(T, N, D);
+  if (op_bytes + ws_bytes == 0)   // the few-token kernel without a split needs no scratch
+    return gemm_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype, nullptr, nullptr, status, stream);
   void* scratch = nullptr;
   e = cudaMallocFromPoolAsync(&scratch, op_bytes + ws_bytes, pool, stream);
   if (e != cudaSuccess) {

@@ -88,6 +88,10 @@ inline int device_sm_count() {
 // Tensor map of a bf16 [rows][inner] matrix (row stride ld elements): 64 x 128 boxes, 128-byte
 // swizzle, zero fill outside (rotate_mma.cu).
 cudaError_t make_bf16_tile_map(CUtensorMap* map, const void* base, int64_t rows, int64_t inner, int64_t ld);
+// Tensor map of a dense uint8 [rows][inner] matrix: box_inner bytes x box_rows, zero fill outside,
+// optionally the 128-byte swizzle (rotate_mma.cu).
+cudaError_t make_u8_tile_map(CUtensorMap* map, const void* base, int64_t rows, int64_t inner, int box_inner,
+                             int box_rows, bool swizzle128);
 // y = ((x * a) H) * b per row and group, one thread per row (smooth_rows.cu).  mode 0: a = 1/s with
 // s the per-channel max |x| over each 128-row block (to smooth_out if non-null); 1: a = vec;
 // 2: b = vec; 3: neither.
@@ -103,13 +107,26 @@ cudaError_t launch_smooth_hadamard(const pq_plan* plan, const void* X, int64_t T
 // weights = 0: activations, 1: weights.
 cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
                               uint8_t* codes, float* scales, cudaStream_t stream);
+// Calls with at most this many tokens take the few-token kernel (gemm_small.cu): packed codes
+// read directly, int8 tensor-core products, no operand scratch.
+constexpr int64_t kGemmSmallT = 128;
+// Group ranges per 128-row weight tile of the few-token kernel (1 = no split).
+int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int* gs_out);
+// The few-token GEMM (+ the split reduction when ws != nullptr and the sizes call for it).
+pq_status gemm_small_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
+                            const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
+                            pq_out_dtype out_dtype, float* ws, unsigned int* status, cudaStream_t stream);
+// Y = sum over ksplit float32 partial [T][N] tiles in ws, ascending (gemm.cu).
+pq_status launch_splitk_reduce(const float* ws, int ksplit, int64_t T, int64_t N, void* Y, int out_bf16,
+                               cudaStream_t stream);
 pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                    const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
                    pq_out_dtype out_dtype, cudaStream_t stream);
-// Bytes of int8 operand scratch the GEMM needs: (T + N) * D.
+// Bytes of operand scratch the GEMM needs: (T + N) * D for the expanded operands (none for the
+// few-token kernel).
 size_t gemm_scratch_bytes(int64_t T, int64_t N, int64_t D);
 // Split-K factor for a problem (1 = none) and the groups per range; the float32 partial-tile
-// workspace it needs (0 when unsplit).
+// workspace it needs (0 when unsplit), for whichever kernel the sizes select.
 int gemm_ksplit(int64_t T, int64_t N, int64_t D, int* gs_out);
 size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t D);
 // Expansion + contraction (+ split-K reduction) launches on `stream` using caller-provided

@@ -426,7 +426,8 @@ extern "C" pq_status pq_w4a4_gemm_launch_count(int64_t T, int64_t N, int64_t D, 
   }
   pq_status st = check_gemm_sizes(T, N, D);
   if (st != PQ_OK) return st;
-  *launches = gemm_ksplit(T, N, D, nullptr) > 1 ? 3 : 2;
+  const int split = gemm_ksplit(T, N, D, nullptr) > 1 ? 1 : 0;
+  *launches = (T <= kGemmSmallT ? 1 : 2) + split;
   return PQ_OK;
 }
 

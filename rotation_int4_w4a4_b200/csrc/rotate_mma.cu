@@ -294,6 +294,22 @@ cudaError_t make_bf16_tile_map(CUtensorMap* map, const void* base, int64_t rows,
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// uint8 [rows][inner] (row stride = inner bytes) with a box of box_inner bytes x box_rows, zero
+// fill outside; swizzle128: the 128-byte swizzle (box_inner must then be 128).
+cudaError_t make_u8_tile_map(CUtensorMap* map, const void* base, int64_t rows, int64_t inner, int box_inner,
+                             int box_rows, bool swizzle128) {
+  EncodeTiledFnR enc = encode_fn_r();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)inner};
+  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
                               uint8_t* codes, float* scales, cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;

@@ -177,3 +177,47 @@ def test_full_size_sampled_rows(pq, name):
     Ys = Y[torch.from_numpy(rows).cuda()].cpu().numpy()
     ref = oracle.gemm(ca[rows], sa[rows], cw, sw)
     assert rel_fro(Ys, ref.y64) < 1e-5
+
+
+# ------------------------------------------------------- few-token kernel (T <= 128)
+@pytest.mark.parametrize("T,N,D,out", [(1, 16, 128, "f32"), (2, 272, 384, "f32"), (15, 512, 1024, "bf16"),
+                                       (16, 4096, 4096, "f32"), (17, 144, 256, "f32"), (33, 1024, 512, "bf16"),
+                                       (64, 4096, 4096, "f32"), (65, 400, 640, "f32"), (100, 272, 1280, "bf16"),
+                                       (128, 1024, 2048, "f32"), (129, 256, 512, "f32")])
+def test_few_tokens(pq, T, N, D, out):
+    """T <= 128 runs the few-token kernel (packed codes widened in the kernel, int8 MMAs, N = T
+    rounded up to 16/32/64/128): token counts on both sides of each width, ragged N (past the
+    last 128-row weight tile), group-range splits (small T) and single launches (T = 64, 128).
+    T = 129 is the first call on the CTA-pair kernel."""
+    ca, sa = inputs.random_codes(5000 + T, T, D)
+    cw, sw = inputs.random_codes(6000 + N, N, D)
+    Y = run_gemm(pq, ca, sa, cw, sw, out=out)
+    r = oracle.gemm(ca, sa, cw, sw)
+    if out == "f32":
+        assert rel_fro(Y, r.y64) < 1e-5
+    else:
+        ref = oracle.bf16_round(r.y32)
+        ulp = np.maximum(np.abs(ref), 2.0 ** -126) * 2.0 ** -7
+        assert np.all(np.abs(Y - ref) <= ulp)
+
+
+def test_few_tokens_adversarial_dots_bit_exact(pq):
+    """Unit scales and D = 128 through the int8 path: each output is 256 d / 256, exact."""
+    T, N = 96, 384
+    ca = adversarial_codes(T, 81)
+    cw = adversarial_codes(N, 82)
+    Y = run_gemm(pq, ca, np.ones((T, 1), np.float32), cw, np.ones((N, 1), np.float32))
+    assert np.array_equal(Y, oracle.group_dots(ca, cw, 128)[0].astype(np.float32))
+
+
+@pytest.mark.parametrize("T", [1, 4, 16, 64])
+def test_few_tokens_match_unsplit_order(pq, T):
+    """The split group ranges (summed in ascending order) agree with the oracle's ascending
+    float32 accumulation to within float32 rounding, at the sweep's decode sizes."""
+    D, N = 4096, 14336
+    ca, sa = inputs.random_codes(7000 + T, T, D)
+    cw, sw = inputs.random_codes(7100, N, D)
+    Y = run_gemm(pq, ca, sa, cw, sw)
+    r = oracle.gemm(ca, sa, cw, sw)
+    assert rel_fro(Y, r.y64) < 1e-5
+    assert rel_fro(Y, r.y32) < 1e-5

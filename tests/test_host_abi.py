@@ -106,7 +106,8 @@ def test_selftest_wait_timeout_validation(pq):
 
 def test_gemm_launch_count_query(pq):
     """Host-only query (no GPU here, so 148 SMs are assumed): sizes are validated as for the
-    GEMM, and the count is 2 or 3 (with the split-K reduction)."""
+    GEMM.  More than 128 tokens: 2 or 3 launches (operand expansion, contraction, split-K
+    reduction).  At most 128 tokens: 1, or 2 with the group-range reduction."""
     import ctypes
     L = pq.lib
     n = ctypes.c_int(-1)
@@ -116,9 +117,15 @@ def test_gemm_launch_count_query(pq):
     assert L.pq_w4a4_gemm_launch_count(4, 16, 128, None) == pq.PQ_ERR_INVALID_ARG
     assert n.value == -1
     assert pq.pq_w4a4_gemm_launch_count(4096, 14336, 4096) == 2   # 896 pair tiles
-    assert pq.pq_w4a4_gemm_launch_count(1, 14336, 4096) == 2      # 56 pair tiles > 74 / 2
     assert pq.pq_w4a4_gemm_launch_count(256, 4096, 4096) == 3     # 16 pair tiles, 32 groups
-    assert pq.pq_w4a4_gemm_launch_count(1, 4096, 512) == 2        # 4 groups: never split
+    assert pq.pq_w4a4_gemm_launch_count(129, 4096, 4096) == 3     # 129 tokens: CTA-pair kernel
+    # few tokens: 32 weight tiles of 128 rows -> 4 group ranges in one wave over 148 SMs
+    assert pq.pq_w4a4_gemm_launch_count(1, 4096, 4096) == 2
+    assert pq.pq_w4a4_gemm_launch_count(1, 4096, 512) == 1        # 4 groups: one range (one stage)
+    assert pq.pq_w4a4_gemm_launch_count(1, 14336, 4096) == 1      # 112 tiles: one wave unsplit
+    # 64 and 128 tokens: partial tiles would outweigh the weights, so one launch writes Y
+    assert pq.pq_w4a4_gemm_launch_count(64, 4096, 4096) == 1
+    assert pq.pq_w4a4_gemm_launch_count(128, 14336, 4096) == 1
 
 
 def test_binding_rejects_host_and_strided_tensors(pq):
