@@ -426,3 +426,73 @@ def bf16_round(y32: np.ndarray) -> np.ndarray:
     b = np.ascontiguousarray(y32, dtype=np.float32).view(np.uint32).astype(np.uint64)
     r = (b + 0x7FFF + ((b >> 16) & 1)) >> 16
     return (r.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+# ------------------------------------------------ rotated runtime smoothing (RRS Fig. 4)
+@dataclasses.dataclass
+class RRSPrep:
+    chan_max: np.ndarray     # float64 [D]: max over all rows of |X_rot[:, j]| (original channel j)
+    perm: np.ndarray         # int64 [D]: reordered position k holds original channel perm[k]
+    group_scale: np.ndarray  # float64 [G]: s_G, the maximum over reordered group G (0 -> 1)
+
+
+def rrs_prepare(x_bits: np.ndarray, g: int = 128) -> RRSPrep:
+    """[RRS page] main equation: X_rot = X R and s_j = max |(X_rot)_j| over every row of the
+    column; Fig. 4 (1): the channels are reordered by their maxima; Fig. 4 (2): the reordered
+    channels are grouped by the GEMM's block size and each group's maximum is its runtime
+    smoothing scale.
+
+    Readings: R is the block Hadamard H_g / sqrt(g) (the page's R = (1/sqrt(K))[s_ij]); the order
+    is descending, ties broken by the lower original index; a group whose maximum is 0 gets 1.
+    """
+    xr = hadamard_rotate(bf16_to_f64(x_bits), g)
+    D = xr.shape[1]
+    m = np.max(np.abs(xr), axis=0)
+    perm = np.lexsort((np.arange(D), -m))          # primary key: -m ascending; then the index
+    s = m[perm].reshape(D // g, g).max(axis=1)
+    s[s == 0.0] = 1.0
+    return RRSPrep(m, perm.astype(np.int64), s)
+
+
+def rrs_transform_quant(x_bits: np.ndarray, prep: RRSPrep, g: int = 128) -> TQResult:
+    """The smoothed activations X_rot[:, perm] / s_G ([RRS page] main equation, fourth line:
+    Quantize(X_rot diag(s)^-1), with s constant over each reordered group as in Fig. 4 (2)),
+    quantised symmetrically per row over all D channels (the RRS page's setup quantises
+    activations per token): scale = max|.| / 7, codes = RNE(value / scale).  Returns codes
+    [rows, D/2] and the per-row scales [rows] (TQResult.scales)."""
+    xr = hadamard_rotate(bf16_to_f64(x_bits), g)
+    D = xr.shape[1]
+    xs = xr[:, prep.perm] / np.repeat(prep.group_scale, g)
+    q = quantize(xs, D)
+    return TQResult(pack_nibbles(q.codes), q.scales[:, 0].copy(), None, q, xs)
+
+
+def rrs_pack_weights(w_bits: np.ndarray, prep: RRSPrep, g: int = 128) -> TQResult:
+    """W_rot = W R^-T (the same block Hadamard, symmetric orthogonal) with its channels reordered
+    like the activations, quantised per group of g reordered channels.  The group's smoothing
+    scale is folded into the stored weight scale ([RRS page] Fig. 4 (3): the runtime smoothing
+    scales are applied to the interim block results):  F[n, G] = fl32(fl32(m / 7) * fl32(s_G))."""
+    wr = hadamard_rotate(bf16_to_f64(w_bits), g)[:, prep.perm]
+    q = quantize(wr, g)
+    F = (q.scales.astype(np.float32) * prep.group_scale.astype(np.float32)[None, :]).astype(np.float32)
+    return TQResult(pack_nibbles(q.codes), F, None, q, wr)
+
+
+def rrs_gemm(codes_a, token_scales, codes_w, F, g: int = 128) -> GemmResult:
+    """[RRS page] main equation, last line (Y = sum_j (X'_q)_j (W'_q)_j^T s_j) with Fig. 4 (3):
+    per block (= quantisation group) the interim integer product is scaled by the block's factor
+    F[n, G] (weight scale x smoothing scale), and the token's scale is applied once:
+    Y[t, n] = sa[t] * sum_G F[n, G] d_G[t, n].
+
+    Reading: float32 accumulation over G in ascending order, acc = fl(acc + fl(F d)), then
+    Y = fl(acc * sa); the float64 shadow is the exact sum."""
+    d = group_dots(codes_a, codes_w, g)
+    G, T, N = d.shape
+    sa = np.asarray(token_scales, dtype=np.float32)
+    Fw = np.asarray(F, dtype=np.float32)
+    acc = np.zeros((T, N), dtype=np.float32)
+    acc64 = np.zeros((T, N), dtype=np.float64)
+    for gi in range(G):
+        acc = (acc + (Fw[:, gi][None, :] * d[gi].astype(np.float32)).astype(np.float32)).astype(np.float32)
+        acc64 += Fw[:, gi].astype(np.float64)[None, :] * d[gi].astype(np.float64)
+    return GemmResult((acc * sa[:, None]).astype(np.float32), acc64 * sa.astype(np.float64)[:, None])
