@@ -48,8 +48,8 @@ L2_BYTES = 126 * 1000 * 1000                     # B200 L2
 DECODE_T_MAX = 128
 # Kernel sources whose DRAM counters profiles/traffic.json records; a change to any of them
 # makes the recorded traffic stale (reported as null).
-KERNEL_SOURCES = ("rotation_int4_w4a4_b200/csrc/gemm.cu", "rotation_int4_w4a4_b200/csrc/ptx.cuh",
-                  "rotation_int4_w4a4_b200/csrc/rotate_mma.cu", "rotation_int4_w4a4_b200/csrc/transform.cu")
+KERNEL_SOURCES = tuple("rotation_int4_w4a4_b200/csrc/" + f for f in (
+    "gemm.cu", "gemm_small.cu", "ptx.cuh", "rotate_mma.cu", "transform.cu", "smooth_rows.cu", "rows.cuh", "rrs.cu"))
 
 
 def load_peaks():
@@ -449,20 +449,29 @@ class Setup:
 
     def timed_steps(self, steps, stream, offset=0):
         """Per step and call, CUDA-event milliseconds on the launching stream (L2 cold first)."""
-        import torch
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
-        for k in range(steps):
-            self.flush()
-            calls = self.calls(self.sets[(k + offset) % self.nsets], stream)
-            ev[k][0].record(stream)
-            for j, c in enumerate(calls):
-                c()
-                ev[k][j + 1].record(stream)
-        torch.cuda.synchronize()
-        return [[e[j].elapsed_time(e[j + 1]) for j in range(3)] for e in ev]
+        return time_calls(lambda k: self.calls(self.sets[(k + offset) % self.nsets], stream), self.flush,
+                          steps, stream)
 
     def close(self):
         self.plan.close()
+
+
+def time_calls(calls_of, flush, steps, stream):
+    """Per step k and call j, the CUDA-event milliseconds of calls_of(k)[j] on the launching
+    stream, with flush() (L2 eviction) before each step."""
+    import torch
+    ev = []
+    for k in range(steps):
+        flush()
+        calls = calls_of(k)
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+        e[0].record(stream)
+        for j, c in enumerate(calls):
+            c()
+            e[j + 1].record(stream)
+        ev.append(e)
+    torch.cuda.synchronize()
+    return [[e[j].elapsed_time(e[j + 1]) for j in range(len(e) - 1)] for e in ev]
 
 
 def components(wl, per, peaks):
@@ -563,6 +572,68 @@ def measure_also(name, args, dev, stream, peaks, peak_src):
     return out
 
 
+def rrs_algorithmic(wl):
+    """Algorithmic bytes / ops per call of rotated runtime smoothing on a workload's shapes."""
+    T, D, N, G = wl.T, wl.D, wl.N, wl.D // wl.g
+    return {
+        # X in; channel maxima, order, inverse order out; group scales out
+        "rrs_prepare": T * D * 2 + D * 12 + G * 4,
+        # X, order and group scales in; codes and one float32 scale per token out
+        "rrs_transform_quant": T * D * 2.5 + T * 4 + D * 4 + G * 4,
+        # W, order and group scales in; codes and folded scales out
+        "rrs_pack_weights": N * D * 2.5 + N * G * 4 + D * 4 + G * 4,
+        "rrs_gemm_ops": 2.0 * T * N * D,
+        "rrs_gemm": T * D / 2 + N * D / 2 + T * 4 + N * G * 4 + T * N * 4,
+    }
+
+
+def measure_rrs(args, dev, stream, peaks, peak_src):
+    """Rotated runtime smoothing with channel reordering on the down_proj shapes: channel
+    maxima and order over all tokens, the smoothed per-token activation codes, the reordered
+    weights with the smoothing scale folded in, and the row-scale GEMM; timed like the main step
+    (L2 flushed before each step, CUDA events on the launching stream)."""
+    import torch
+
+    from rotation_int4_w4a4_b200 import inputs, pq
+    wl = inputs.workload("down_proj")
+    T, D, N, G = wl.T, wl.D, wl.N, wl.D // wl.g
+    plan = pq.Plan("hadamard", D)
+    X, W = dev_bf16(wl.X, dev), dev_bf16(wl.W, dev)
+    f32, i32, u8 = torch.float32, torch.int32, torch.uint8
+    b = {"cm": torch.empty(D, dtype=f32, device=dev), "perm": torch.empty(D, dtype=i32, device=dev),
+         "inv": torch.empty(D, dtype=i32, device=dev), "gs": torch.empty(G, dtype=f32, device=dev),
+         "ca": torch.empty((T, D // 2), dtype=u8, device=dev), "ts": torch.empty(T, dtype=f32, device=dev),
+         "cw": torch.empty((N, D // 2), dtype=u8, device=dev), "sw": torch.empty((N, G), dtype=f32, device=dev),
+         "Y": torch.empty((T, N), dtype=f32, device=dev)}
+    calls = (lambda: pq.pq_rrs_prepare(plan, X, b["cm"], b["perm"], b["inv"], b["gs"], stream=stream),
+             lambda: pq.pq_rrs_transform_quant(plan, X, b["perm"], b["gs"], b["ca"], b["ts"], stream=stream),
+             lambda: pq.pq_rrs_pack_weights(plan, W, b["perm"], b["gs"], b["cw"], b["sw"], stream=stream),
+             lambda: pq.pq_rrs_gemm(b["ca"], b["ts"], b["cw"], b["sw"], b["Y"], stream=stream))
+    flush = L2Flush(dev)
+    time_calls(lambda k: calls, flush, max(3, args.warmup), stream)
+    per = time_calls(lambda k: calls, flush, max(5, min(args.steps, 10)), stream)
+    pq.pq_check_status(plan)
+    alg = rrs_algorithmic(wl)
+    names = ("rrs_prepare", "rrs_transform_quant", "rrs_pack_weights", "rrs_gemm")
+    comps = {}
+    for j, nm in enumerate(names):
+        ms = statistics.mean(p[j] for p in per)
+        comps[nm] = {"us": 1e3 * ms, "GB_s": alg[nm] / (ms * 1e-3) / 1e9}
+        comps[nm]["frac_hbm"] = comps[nm]["GB_s"] / peaks["hbm_gbs"]
+    int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    comps["rrs_gemm"]["TOPS"] = alg["rrs_gemm_ops"] / (comps["rrs_gemm"]["us"] * 1e-6) / 1e12
+    comps["rrs_gemm"]["frac_int8"] = comps["rrs_gemm"]["TOPS"] / int8_peak
+    step_ms = statistics.mean(sum(p) for p in per)
+    plan.close()
+    del b, X, W, flush
+    torch.cuda.empty_cache()
+    return {"workload": f"rotated runtime smoothing, reordered channels: X[{T},{D}] (down_proj activations), "
+                        f"W[{N},{D}], g=128, per-token activation scales",
+            "T": T, "D": D, "N": N, "components": comps, "ms_per_step": step_ms,
+            "tokens_per_s": T / (step_ms * 1e-3), "peak_source": f"{peak_src} copy bandwidth; {peak_src} bf16 "
+                                                                 f"burst x {INT8_OVER_BF16}"}
+
+
 def run_ours(args, wl, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -627,6 +698,7 @@ def run_ours(args, wl, rank, world, local_rank):
     if world == 1 and not args.no_also and args.workload == DEFAULT_WORKLOAD and args.T is None:
         for name in ("up_proj", "q_proj"):
             also[name] = measure_also(name, args, dev, stream, peaks, peak_src)
+        also["rrs_down_proj"] = measure_rrs(args, dev, stream, peaks, peak_src)
     if rank != 0:
         return
     comps = components(wl, per, peaks)

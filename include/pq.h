@@ -183,6 +183,58 @@ pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A, const uint
                        const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
                        pq_out_dtype out_dtype, void* stream);
 
+/*
+ * Rotated runtime smoothing with channel reordering: the RRS page's main equation (X_rot = X R,
+ * s_j = max |(X_rot)_j|, Quantize(X_rot diag(s)^-1), Y = sum_j (X'_q)_j (W'_q)_j^T s_j) carried
+ * out as in its Fig. 4: (1) the channels are reordered by their maxima, (2) the reordered
+ * channels are grouped by 128 (the GEMM's block) and each group's maximum is its smoothing scale,
+ * (3) the GEMM applies each block's smoothing scale to the block's interim result.  Activations
+ * are quantised per token over the whole row (the page's setup); weights per group of 128
+ * reordered channels.  All four calls need a PQ_HADAMARD plan (R = block Hadamard H_128/sqrt(128))
+ * with D <= 16384 (else PQ_ERR_UNSUPPORTED); pointers are device pointers owned by the caller,
+ * 16-byte aligned; errors and launches behave as for the calls above.
+ *
+ * pq_rrs_prepare — from this call's activations X (bf16 [T][ldx], as pq_transform_quant):
+ *   chan_max     float32 [D]: max over all T rows of |(X R)[:, j]| (original channel order).
+ *   perm         int32 [D]: perm[k] = the original channel at reordered position k (descending
+ *                maximum; equal maxima keep the lower channel first).
+ *   inv_perm     int32 [D]: the inverse, inv_perm[perm[k]] = k.
+ *   group_scale  float32 [D/128]: s_G, the largest maximum of reordered group G (0 -> 1).
+ *   The four outputs are written in full (chan_max and inv_perm are cleared first on `stream`).
+ */
+pq_status pq_rrs_prepare(const pq_plan* plan, const void* X, int64_t T, int64_t ldx, float* chan_max,
+                         int32_t* perm, int32_t* inv_perm, float* group_scale, void* stream);
+
+/*
+ * pq_rrs_transform_quant — per row t: v_k = (X R)[t, perm[k]] / s_(k / 128), then one symmetric
+ * INT4 scale for the whole row, token_scales[t] = max_k |v_k| / 7, codes = RNE(v / scale) packed
+ * as elsewhere (codes [T][D/2] are in the reordered channel order).  perm and group_scale as
+ * written by pq_rrs_prepare (for the same or an earlier batch).
+ */
+pq_status pq_rrs_transform_quant(const pq_plan* plan, const void* X, int64_t T, int64_t ldx,
+                                 const int32_t* perm, const float* group_scale, uint8_t* codes,
+                                 float* token_scales, void* stream);
+
+/*
+ * pq_rrs_pack_weights — per weight row n (W bf16 [N][D] dense): v_k = (W R)[n, perm[k]] (the
+ * same rotation; H is symmetric orthogonal, so R^-T = R), quantised per group of 128 reordered
+ * channels; scales_W[n][G] = (max_(k in G) |v_k| / 7) * s_G, the group's weight scale with its
+ * smoothing scale folded in, which is the factor pq_rrs_gemm applies per block.
+ */
+pq_status pq_rrs_pack_weights(const pq_plan* plan, const void* W, int64_t N, const int32_t* perm,
+                              const float* group_scale, uint8_t* codes_W, float* scales_W, void* stream);
+
+/*
+ * pq_rrs_gemm — Y[t][n] = token_scales[t] * sum_G scales_W[n][G] * d_G[t][n], d_G the exact
+ * integer dot of group G as in pq_w4a4_gemm: per block one multiply-add per output element with
+ * the block's factor, then the token's scale once.  codes and scales as written by
+ * pq_rrs_transform_quant (token_scales float32 [T]) and pq_rrs_pack_weights.  Sizes, output,
+ * scratch, splitting and errors as for pq_w4a4_gemm.
+ */
+pq_status pq_rrs_gemm(const uint8_t* codes_A, const float* token_scales, const uint8_t* codes_W,
+                      const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
+                      pq_out_dtype out_dtype, void* stream);
+
 /* Bytes of the fixed device-array scratch behind pq_w4a4_gemm_noalloc (32 MiB). */
 #define PQ_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 

@@ -207,6 +207,9 @@ __device__ __forceinline__ void unit_coords(int u, const Work& wk, int& m0, int&
 }
 
 // -------------------------------------------------------------------------- control
+// kRow: scales_W holds per-(row, group) factors and scales_A one scale per token (applied in the
+// epilogue after the groups), so the loaders fetch only the weight rows' factors.
+template <bool kRow>
 __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA, const CUtensorMap& tmB,
                                             const float* __restrict__ scales_A, const float* __restrict__ scales_W,
                                             uint32_t tmem, int T, int N, int G, int scales_vec16, const Work& wk,
@@ -295,6 +298,7 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
         for (int i = 0; i < (BM + BN) / NUM_SCALE_THREADS; ++i) {
           const int r = j + NUM_SCALE_THREADS * i;       // 0..127 weight rows, 128..383 tokens
           const bool isw = r < BM;
+          if (kRow && !isw) continue;                    // token scales are not per group
           const int row = isw ? m0 + BM * wk.rank + r : n0 + (r - BM);
           const bool in = row < (isw ? N : T);
           const float* src = (isw ? scales_W : scales_A) + (int64_t)(in ? row : 0) * G + kg0;
@@ -319,9 +323,12 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
 // token half ch = ew / 4 (tokens 128 ch ..); lane L has g = L / 4, q = L % 4.  Its rows are
 // 32 sub + 16 h + g + 8 k and its tokens 128 ch + 16 c + 8 x + 2 q + e (h, k, x, e in {0, 1},
 // c in 0..7).  acc index: ((h * 2 + k) * 8 + c) * 4 + x * 2 + e.
+// kRow: per group acc += d * F (one packed FMA per element pair, F the row's factor for the
+// group), and each token's scale from token_scales multiplies the sum before it is stored.
+template <bool kRow>
 __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* __restrict__ Y, int T, int N,
                                              int G, int out_bf16, const Work& wk, float* __restrict__ ws,
-                                             unsigned int* status) {
+                                             const float* __restrict__ token_scales, unsigned int* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ew = warp - EPI_WARP0;
   const int sub = warp & 3;          // TMEM lane quarter this warp may access
@@ -367,9 +374,11 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
         ptx::tmem_ld_16x256b<EPI_NX>(tbase + EPI_LDC * cc, d0);
         ptx::tmem_ld_16x256b<EPI_NX>(tbase + (16u << 16) + EPI_LDC * cc, d1);
         uint64_t sa2[EPI_NX];                        // token scales of columns LDC cc + 8x + 2q + {0, 1}
+        if (!kRow) {
 #pragma unroll
-        for (int x = 0; x < EPI_NX; ++x)
-          sa2[x] = ptx::lds_pair<4 * SC_GROUPS>(sab + 4 * SC_GROUPS * (EPI_LDC * cc + 8 * x));
+          for (int x = 0; x < EPI_NX; ++x)
+            sa2[x] = ptx::lds_pair<4 * SC_GROUPS>(sab + 4 * SC_GROUPS * (EPI_LDC * cc + 8 * x));
+        }
         const uint32_t after = ptx::tmem_ld_wait_token();
         if (cc == EPI_COLS / EPI_LDC - 1) {
           // The whole group's tile is read: hand the buffer back to the MMA before the math.
@@ -385,8 +394,13 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
             const int c = xx >> 1;                          // 16-token chunk of the accumulator layout
             const int i0 = ((0 * 2 + k) * EPI_CHUNKS + c) * 2 + (xx & 1);
             const int i1 = ((1 * 2 + k) * EPI_CHUNKS + c) * 2 + (xx & 1);
-            ptx::mul_fma2(acc2[i0], d0[4 * x + 2 * k], d0[4 * x + 2 * k + 1], sw2[0 * 2 + k], sa2[x], after);
-            ptx::mul_fma2(acc2[i1], d1[4 * x + 2 * k], d1[4 * x + 2 * k + 1], sw2[1 * 2 + k], sa2[x], after);
+            if (kRow) {
+              ptx::fma2(acc2[i0], d0[4 * x + 2 * k], d0[4 * x + 2 * k + 1], sw2[0 * 2 + k], after);
+              ptx::fma2(acc2[i1], d1[4 * x + 2 * k], d1[4 * x + 2 * k + 1], sw2[1 * 2 + k], after);
+            } else {
+              ptx::mul_fma2(acc2[i0], d0[4 * x + 2 * k], d0[4 * x + 2 * k + 1], sw2[0 * 2 + k], sa2[x], after);
+              ptx::mul_fma2(acc2[i1], d1[4 * x + 2 * k], d1[4 * x + 2 * k + 1], sw2[1 * 2 + k], sa2[x], after);
+            }
           }
       }
       if (gi == SC_GROUPS - 1 || kg == k1 - 1) {
@@ -417,12 +431,13 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
         const int dt = 8 * (xe >> 1) + (xe & 1);
         if (tb + 16 * c + dt < T) {
           char* p = row + dt * row_step;
+          const float ts = kRow ? __ldg(token_scales + tb + 16 * c + dt) : 1.0f;
 #pragma unroll
           for (int hk = 0; hk < 4; ++hk) {
             if (!nin[hk]) continue;
             float lo, hi;                                            // rows 16 h + 8 k = 8 hk
             ptx::unpack2(acc2[(hk * EPI_CHUNKS + c) * 2 + (xe >> 1)], lo, hi);
-            const float v = (xe & 1) ? hi : lo;
+            const float v = kRow ? ((xe & 1) ? hi : lo) * ts : ((xe & 1) ? hi : lo);
             if (!bf16_out) reinterpret_cast<float*>(p)[8 * hk] = v;
             else reinterpret_cast<__nv_bfloat16*>(p)[8 * hk] = __float2bfloat16_rn(v);
           }
@@ -433,6 +448,7 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
   }
 }
 
+template <bool kRow>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const float* __restrict__ scales_A, const float* __restrict__ scales_W, void* __restrict__ Y,
@@ -487,10 +503,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1) w4a4
 
   if (warp < EPI_WARP0) {
     ptx::setmaxnreg_dec<REG_CTRL>();
-    cta_control(S, tmA, tmB, scales_A, scales_W, tmem, T, N, G, scales_vec16, wk, status);
+    cta_control<kRow>(S, tmA, tmB, scales_A, scales_W, tmem, T, N, G, scales_vec16, wk, status);
   } else {
     ptx::setmaxnreg_inc<REG_EPI>();
-    cta_epilogue(S, tmem, Y, T, N, G, out_bf16, wk, ws, status);
+    cta_epilogue<kRow>(S, tmem, Y, T, N, G, out_bf16, wk, ws, scales_A, status);
   }
 
   __syncwarp();
@@ -637,7 +653,7 @@ pq_status gemm_max_pairs(int sms, int* out) {
     attr.val.clusterDim.z = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    e = cudaOccupancyMaxActiveClusters(&n, w4a4_gemm_kernel, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, w4a4_gemm_kernel<false>, &cfg);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(gemm)");
     if (n < 1) {
       set_error("w4a4_gemm_kernel: no CTA pair fits on this device");
@@ -690,9 +706,10 @@ pq_status launch_splitk_reduce(const float* ws, int ksplit, int64_t T, int64_t N
 
 pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W, const float* scales_W,
                       int64_t T, int64_t N, int64_t D, void* Y, pq_out_dtype out_dtype, uint8_t* scratch,
-                      float* ws, unsigned int* status, cudaStream_t stream) {
+                      float* ws, unsigned int* status, cudaStream_t stream, bool row_scale) {
   if (T <= kGemmSmallT)
-    return gemm_small_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype, ws, status, stream);
+    return gemm_small_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype, ws, status, stream,
+                             row_scale);
   uint8_t* A8 = scratch;
   uint8_t* W8 = scratch + (size_t)T * (size_t)D;
   // MMA operand A = weights (M = output channels), B = activations (N = tokens).
@@ -712,11 +729,15 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   const int64_t chunksA = T * (D / 32), chunksW = N * (D / 32);   // 16 packed bytes each
   const int64_t want = (chunksA + chunksW + 255) / 256;
   const int egrid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
-  static std::atomic<bool> attr_expand[kMaxDevices], attr_gemm[kMaxDevices];
+  static std::atomic<bool> attr_expand[kMaxDevices], attr_gemm[kMaxDevices], attr_gemm_row[kMaxDevices];
   cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(expand_codes_kernel), 0, attr_expand);
   if (e != cudaSuccess) return cuda_fail(e, "expand_codes_kernel attributes");
-  e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_kernel), (int)kSmemBytes, attr_gemm);
+  e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_kernel<false>), (int)kSmemBytes, attr_gemm);
   if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel attributes");
+  if (row_scale) {
+    e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_kernel<true>), (int)kSmemBytes, attr_gemm_row);
+    if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel attributes");
+  }
   expand_codes_kernel<<<egrid, 256, 0, stream>>>(codes_A, chunksA, codes_W, chunksW, A8, W8);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "expand_codes_kernel launch");
@@ -731,14 +752,14 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   // The warp roles re-divide the launch's registers with setmaxnreg; that only works when the
   // kernel was compiled with exactly the budgeted count (otherwise an increase would never be
   // granted), so refuse to launch anything else.
-  static std::atomic<int> num_regs_cache{-1};       // a property of the kernel binary
-  int num_regs = num_regs_cache.load(std::memory_order_relaxed);
+  static std::atomic<int> num_regs_cache[2] = {-1, -1};   // a property of each kernel binary
+  int num_regs = num_regs_cache[row_scale].load(std::memory_order_relaxed);
   if (num_regs < 0) {
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, w4a4_gemm_kernel);
+    e = row_scale ? cudaFuncGetAttributes(&fa, w4a4_gemm_kernel<true>) : cudaFuncGetAttributes(&fa, w4a4_gemm_kernel<false>);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(gemm)");
     num_regs = fa.numRegs;
-    num_regs_cache.store(num_regs, std::memory_order_relaxed);
+    num_regs_cache[row_scale].store(num_regs, std::memory_order_relaxed);
   }
   if (num_regs != (int)REG_LAUNCH) {
     set_error("w4a4_gemm_kernel compiled with %d registers per thread, %u expected", num_regs, REG_LAUNCH);
@@ -746,9 +767,14 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   }
   const int G = (int)(D / 128);
   const int scales_vec16 = (G % SC_GROUPS == 0) ? 1 : 0;   // rows of 16-byte multiples
-  w4a4_gemm_kernel<<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB, scales_A, scales_W, Y, (int)T, (int)N,
-                                                               G, scales_vec16, out_dtype == PQ_OUT_BF16 ? 1 : 0,
-                                                               m_tiles, n_tiles, ksplit, gs, ws, status);
+  if (row_scale)
+    w4a4_gemm_kernel<true><<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB, scales_A, scales_W, Y, (int)T, (int)N,
+                                                                      G, scales_vec16, out_dtype == PQ_OUT_BF16 ? 1 : 0,
+                                                                      m_tiles, n_tiles, ksplit, gs, ws, status);
+  else
+    w4a4_gemm_kernel<false><<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB, scales_A, scales_W, Y, (int)T, (int)N,
+                                                                       G, scales_vec16, out_dtype == PQ_OUT_BF16 ? 1 : 0,
+                                                                       m_tiles, n_tiles, ksplit, gs, ws, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel launch");
   if (ksplit > 1) return launch_splitk_reduce(ws, ksplit, T, N, Y, out_dtype == PQ_OUT_BF16 ? 1 : 0, stream);
@@ -756,7 +782,8 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
 }
 
 pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W, const float* scales_W,
-                   int64_t T, int64_t N, int64_t D, void* Y, pq_out_dtype out_dtype, cudaStream_t stream) {
+                   int64_t T, int64_t N, int64_t D, void* Y, pq_out_dtype out_dtype, cudaStream_t stream,
+                   bool row_scale) {
   unsigned int* status = nullptr;
   cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_gemm_status);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(gemm status)");
@@ -769,7 +796,8 @@ pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t*
   const size_t op_bytes = (gemm_scratch_bytes(T, N, D) + 255) & ~(size_t)255;
   const size_t ws_bytes = gemm_workspace_bytes(T, N, D);
   if (op_bytes + ws_bytes == 0)   // the few-token kernel without a split needs no scratch
-    return gemm_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype, nullptr, nullptr, status, stream);
+    return gemm_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype, nullptr, nullptr, status, stream,
+                       row_scale);
   void* scratch = nullptr;
   e = cudaMallocFromPoolAsync(&scratch, op_bytes + ws_bytes, pool, stream);
   if (e != cudaSuccess) {
@@ -778,7 +806,7 @@ pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t*
   }
   float* ws = ws_bytes ? reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + op_bytes) : nullptr;
   pq_status st = gemm_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype,
-                             static_cast<uint8_t*>(scratch), ws, status, stream);
+                             static_cast<uint8_t*>(scratch), ws, status, stream, row_scale);
   e = cudaFreeAsync(scratch, stream);
   if (st == PQ_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(gemm scratch)");
   return st;

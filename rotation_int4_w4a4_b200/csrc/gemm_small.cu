@@ -154,7 +154,9 @@ __device__ __forceinline__ Unit unit_of(int u, int ranges, int gs, int G) {
   return w;
 }
 
-template <int NT>
+// kRow: scales_W holds per-(row, group) factors and scales_A one scale per token: per group
+// acc += float(256 d) * (F / 256), and the token's scale multiplies the sum at the end.
+template <int NT, bool kRow>
 __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
     const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
     const float* __restrict__ scales_A, const float* __restrict__ scales_W, void* __restrict__ Y,
@@ -303,11 +305,11 @@ __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
 #pragma unroll
       for (int t = 0; t < NT; ++t) acc[t] = 0.0f;
       __syncwarp();                  // the previous unit's reads of the staged scales are done
-      stage(w.k0, w.k1, 0);
+      if (!kRow) stage(w.k0, w.k1, 0);
       for (int kg = w.k0; kg < w.k1; ++kg, ++step) {
         const int g = (kg - w.k0) % GS_SC;
         const int buf = ((kg - w.k0) / GS_SC) & 1;
-        if (g == 0) {
+        if (!kRow && g == 0) {
           // This batch's scales have landed; start copying the next batch into the other buffer.
           ptx::cp_async_wait_all();
           __syncwarp();
@@ -331,17 +333,27 @@ __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&S.acc_empty[b]);
           }
+          if (kRow) {
 #pragma unroll
-          for (int j = 0; j < 16; j += 4) {
-            const float4 s4 = *reinterpret_cast<const float4*>(sag + 16 * c + j);
-            acc[16 * c + j] = fmaf(__int2float_rn((int)d[j]) * swv, s4.x, acc[16 * c + j]);
-            acc[16 * c + j + 1] = fmaf(__int2float_rn((int)d[j + 1]) * swv, s4.y, acc[16 * c + j + 1]);
-            acc[16 * c + j + 2] = fmaf(__int2float_rn((int)d[j + 2]) * swv, s4.z, acc[16 * c + j + 2]);
-            acc[16 * c + j + 3] = fmaf(__int2float_rn((int)d[j + 3]) * swv, s4.w, acc[16 * c + j + 3]);
+            for (int j = 0; j < 16; ++j) acc[16 * c + j] = fmaf(__int2float_rn((int)d[j]), swv, acc[16 * c + j]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; j += 4) {
+              const float4 s4 = *reinterpret_cast<const float4*>(sag + 16 * c + j);
+              acc[16 * c + j] = fmaf(__int2float_rn((int)d[j]) * swv, s4.x, acc[16 * c + j]);
+              acc[16 * c + j + 1] = fmaf(__int2float_rn((int)d[j + 1]) * swv, s4.y, acc[16 * c + j + 1]);
+              acc[16 * c + j + 2] = fmaf(__int2float_rn((int)d[j + 2]) * swv, s4.z, acc[16 * c + j + 2]);
+              acc[16 * c + j + 3] = fmaf(__int2float_rn((int)d[j + 3]) * swv, s4.w, acc[16 * c + j + 3]);
+            }
           }
         }
       }
       if (!ok) break;
+      if (kRow) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+          if (t < T) acc[t] *= __ldg(scales_A + t);
+      }
       if (n < N) {
         // Token t of row n: consecutive threads write consecutive channels.
         if (ranges > 1) {
@@ -374,12 +386,12 @@ __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
   }
 }
 
-template <int NT>
+template <int NT, bool kRow>
 pq_status launch_small(const CUtensorMap& tmW, const CUtensorMap& tmA, const float* scales_A, const float* scales_W,
                        void* Y, float* ws, int T, int N, int G, int ranges, int gs, int units, int out_bf16,
                        unsigned int* status, cudaStream_t stream) {
   static std::atomic<bool> attr_done[kMaxDevices];
-  cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_small_kernel<NT>),
+  cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_small_kernel<NT, kRow>),
                                         (int)small_smem_bytes<NT>(), attr_done);
   if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_small_kernel attributes");
   // The warpgroups' setmaxnreg shares are drawn from the launch allocation (compiled registers x
@@ -388,7 +400,7 @@ pq_status launch_small(const CUtensorMap& tmW, const CUtensorMap& tmA, const flo
   int regs = regs_cache.load(std::memory_order_relaxed);
   if (regs < 0) {
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, w4a4_gemm_small_kernel<NT>);
+    e = cudaFuncGetAttributes(&fa, w4a4_gemm_small_kernel<NT, kRow>);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(w4a4_gemm_small_kernel)");
     regs = fa.numRegs;
     regs_cache.store(regs, std::memory_order_relaxed);
@@ -399,7 +411,7 @@ pq_status launch_small(const CUtensorMap& tmW, const CUtensorMap& tmA, const flo
     return PQ_ERR_CUDA;
   }
   const int grid = std::min(units, device_sm_count());
-  w4a4_gemm_small_kernel<NT><<<grid, GS_THREADS, small_smem_bytes<NT>(), stream>>>(
+  w4a4_gemm_small_kernel<NT, kRow><<<grid, GS_THREADS, small_smem_bytes<NT>(), stream>>>(
       tmW, tmA, scales_A, scales_W, Y, ws, T, N, G, ranges, gs, units, out_bf16, status);
   return cuda_fail(cudaGetLastError(), "w4a4_gemm_small_kernel launch");
 }
@@ -430,7 +442,8 @@ int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int* gs_out) {
 
 pq_status gemm_small_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                             const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
-                            pq_out_dtype out_dtype, float* ws, unsigned int* status, cudaStream_t stream) {
+                            pq_out_dtype out_dtype, float* ws, unsigned int* status, cudaStream_t stream,
+                            bool row_scale) {
   const int NT = T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128;
   const int G = (int)(D / 128);
   int gs = G;
@@ -451,12 +464,18 @@ pq_status gemm_small_launch(const uint8_t* codes_A, const float* scales_A, const
   if (e != cudaSuccess) return cuda_fail(e, "tensor map (packed activations)");
   const int bf16 = out_dtype == PQ_OUT_BF16 ? 1 : 0;
   pq_status st;
+#define PQ_SMALL_CASE(W)                                                                                      \
+  st = row_scale ? launch_small<W, true>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, ranges, gs,  \
+                                         (int)units, bf16, status, stream)                                    \
+                 : launch_small<W, false>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, ranges, gs, \
+                                          (int)units, bf16, status, stream)
   switch (NT) {
-    case 16: st = launch_small<16>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, ranges, gs, (int)units, bf16, status, stream); break;
-    case 32: st = launch_small<32>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, ranges, gs, (int)units, bf16, status, stream); break;
-    case 64: st = launch_small<64>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, ranges, gs, (int)units, bf16, status, stream); break;
-    default: st = launch_small<128>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, ranges, gs, (int)units, bf16, status, stream); break;
+    case 16: PQ_SMALL_CASE(16); break;
+    case 32: PQ_SMALL_CASE(32); break;
+    case 64: PQ_SMALL_CASE(64); break;
+    default: PQ_SMALL_CASE(128); break;
   }
+#undef PQ_SMALL_CASE
   if (st != PQ_OK || ranges == 1) return st;
   return launch_splitk_reduce(ws, ranges, T, N, Y, bf16, stream);
 }

@@ -80,7 +80,7 @@ pq_status gemm_run_static_scratch(const uint8_t* codes_A, const float* scales_A,
   pq_status st = device_setup(dev, &s);
   if (st != PQ_OK) return st;
   return gemm_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype, s.scratch,
-                     /*ws=*/nullptr, s.status, stream);
+                     /*ws=*/nullptr, s.status, stream, /*row_scale=*/false);
 }
 
 }  // namespace pq

@@ -69,6 +69,25 @@ inline cudaError_t set_kernel_attributes(const void* func, int dyn_smem, std::at
   return cudaSuccess;
 }
 
+// For kernels whose dynamic shared memory depends on the call's sizes: raises the kernel's limit
+// whenever a call needs more than the largest value set so far on this device (`largest` is the
+// caller's per-kernel table; the limit only grows, so a larger earlier call keeps later ones valid).
+inline cudaError_t raise_dynamic_smem(const void* func, int dyn_smem, std::atomic<int> (&largest)[kMaxDevices]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool slot = dev >= 0 && dev < kMaxDevices;
+  if (slot && largest[dev].load(std::memory_order_acquire) >= dyn_smem) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_smem);
+  if (e != cudaSuccess) return e;
+  if (slot) {
+    int cur = largest[dev].load(std::memory_order_relaxed);
+    while (cur < dyn_smem && !largest[dev].compare_exchange_weak(cur, dyn_smem, std::memory_order_acq_rel)) {
+    }
+  }
+  return cudaSuccess;
+}
+
 // Multiprocessor count of the current device (148 if it cannot be read).
 inline int device_sm_count() {
   static std::atomic<int> cache[kMaxDevices];
@@ -92,6 +111,10 @@ cudaError_t make_bf16_tile_map(CUtensorMap* map, const void* base, int64_t rows,
 // optionally the 128-byte swizzle (rotate_mma.cu).
 cudaError_t make_u8_tile_map(CUtensorMap* map, const void* base, int64_t rows, int64_t inner, int box_inner,
                              int box_rows, bool swizzle128);
+// bf16 rows [rows][D] as lines of 128 bytes: a box of box_rows whole rows, 128-byte swizzle,
+// rows past the end zero-filled (D / 64 <= 256).
+cudaError_t make_bf16_row_lines_map(CUtensorMap* map, const void* base, int64_t rows, int64_t D, int64_t ld,
+                                    int box_rows);
 // y = ((x * a) H) * b per row and group, one thread per row (smooth_rows.cu).  mode 0: a = 1/s with
 // s the per-channel max |x| over each 128-row block (to smooth_out if non-null); 1: a = vec;
 // 2: b = vec; 3: neither.
@@ -99,14 +122,25 @@ enum { PQ_SR_COLMAX = 0, PQ_SR_PRE = 1, PQ_SR_POST = 2, PQ_SR_NONE = 3 };
 cudaError_t launch_smooth_rows(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int mode,
                                const float* vec, uint8_t* codes, float* scales, float* smooth_out,
                                cudaStream_t stream);
+// Rotated runtime smoothing with channel reordering (rrs.cu): chan_max (float, [D]), perm and
+// inv_perm (int32, [D]) and group_scale ([G]) from the activations; then the row transforms
+// (weights = 0: per-token activation codes and scales [rows]; 1: per-group weight codes and
+// scales with the group's smoothing scale folded in).  rrs_rows_smem_bytes: shared memory per CTA.
+cudaError_t launch_rrs_prepare(const pq_plan* plan, const void* X, int64_t T, int64_t ldx, float* chan_max,
+                               int* perm, int* inv_perm, float* group_scale, cudaStream_t stream);
+cudaError_t launch_rrs_rows(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
+                            const int* perm, const float* group_scale, uint8_t* codes, float* scales,
+                            cudaStream_t stream);
+size_t rrs_rows_smem_bytes(int D);
 // Runtime smoothing after the rotation (PQ_FLAG_SMOOTH_AFTER_ROTATE activations; transform.cu).
 cudaError_t launch_smooth_hadamard(const pq_plan* plan, const void* X, int64_t T, int64_t ldx,
                                    uint8_t* codes, float* scales, float* smooth_out,
                                    cudaStream_t stream);
 // y = x R per group on the tensor cores (rotate_mma.cu) for PQ_GIVENS and PQ_HADAMARD plans;
-// weights = 0: activations, 1: weights.
+// weights = 0: activations, 1: weights.  With chan_max (float bits, [D], zeroed by the caller)
+// nothing is quantised: chan_max[j] becomes max over the rows of |y[:, j]| (normalised rotation).
 cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
-                              uint8_t* codes, float* scales, cudaStream_t stream);
+                              uint8_t* codes, float* scales, cudaStream_t stream, unsigned int* chan_max = nullptr);
 // Calls with at most this many tokens take the few-token kernel (gemm_small.cu): packed codes
 // read directly, int8 tensor-core products, no operand scratch.
 constexpr int64_t kGemmSmallT = 128;
@@ -115,13 +149,16 @@ int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int* gs_out);
 // The few-token GEMM (+ the split reduction when ws != nullptr and the sizes call for it).
 pq_status gemm_small_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                             const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
-                            pq_out_dtype out_dtype, float* ws, unsigned int* status, cudaStream_t stream);
+                            pq_out_dtype out_dtype, float* ws, unsigned int* status, cudaStream_t stream,
+                            bool row_scale);
 // Y = sum over ksplit float32 partial [T][N] tiles in ws, ascending (gemm.cu).
 pq_status launch_splitk_reduce(const float* ws, int ksplit, int64_t T, int64_t N, void* Y, int out_bf16,
                                cudaStream_t stream);
+// row_scale: scales_W holds per-(row, group) factors and scales_A one scale per token, applied
+// after the groups (the rotated-runtime-smoothing GEMM); otherwise both are per (row, group).
 pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                    const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
-                   pq_out_dtype out_dtype, cudaStream_t stream);
+                   pq_out_dtype out_dtype, cudaStream_t stream, bool row_scale = false);
 // Bytes of operand scratch the GEMM needs: (T + N) * D for the expanded operands (none for the
 // few-token kernel).
 size_t gemm_scratch_bytes(int64_t T, int64_t N, int64_t D);
@@ -134,7 +171,7 @@ size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t D);
 pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                       const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
                       pq_out_dtype out_dtype, uint8_t* scratch, float* ws, unsigned int* status,
-                      cudaStream_t stream);
+                      cudaStream_t stream, bool row_scale);
 pq_status gemm_read_and_clear_status(unsigned int* bits);
 // Launches the bounded-wait diagnostic (a wait that cannot complete, limited to limit_ns).
 pq_status gemm_wait_timeout_selftest(uint64_t limit_ns, cudaStream_t stream);

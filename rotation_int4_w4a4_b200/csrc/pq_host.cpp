@@ -418,6 +418,95 @@ extern "C" pq_status pq_w4a4_gemm_noalloc(const uint8_t* codes_A, const float* s
                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
+// --------------------------------------- rotated runtime smoothing (RRS page, Fig. 4)
+namespace {
+
+pq_status check_rrs_plan(const pq_plan* plan) {
+  if (!plan) { set_error("plan is NULL"); return PQ_ERR_INVALID_ARG; }
+  if (plan->kind != PQ_HADAMARD) {
+    set_error("rotated runtime smoothing needs a PQ_HADAMARD plan");
+    return PQ_ERR_UNSUPPORTED;
+  }
+  if (plan->D > 16384 || rrs_rows_smem_bytes(plan->D) > 232448) {
+    set_error("D=%d: rotated runtime smoothing supports D <= 16384", plan->D);
+    return PQ_ERR_UNSUPPORTED;
+  }
+  return check_plan(plan);
+}
+
+pq_status check_rows_arg(const void* X, int64_t rows, int64_t ldx, int D, const char* what) {
+  if (!X) { set_error("%s is NULL", what); return PQ_ERR_INVALID_ARG; }
+  if (rows < 1 || rows >= ((int64_t)1 << 31)) { set_error("%s: rows=%lld out of range", what, (long long)rows); return PQ_ERR_INVALID_ARG; }
+  if (ldx < D || ldx % 8 != 0) { set_error("ldx=%lld must be >= D=%d and a multiple of 8", (long long)ldx, D); return PQ_ERR_INVALID_ARG; }
+  if (!aligned16(X)) { set_error("device pointers must be 16-byte aligned"); return PQ_ERR_INVALID_ARG; }
+  return PQ_OK;
+}
+
+}  // namespace
+
+extern "C" pq_status pq_rrs_prepare(const pq_plan* plan, const void* X, int64_t T, int64_t ldx, float* chan_max,
+                                    int32_t* perm, int32_t* inv_perm, float* group_scale, void* stream) {
+  clear_error();
+  pq_status st = check_rrs_plan(plan);
+  if (st != PQ_OK) return st;
+  st = check_rows_arg(X, T, ldx, plan->D, "X");
+  if (st != PQ_OK) return st;
+  if (!chan_max || !perm || !inv_perm || !group_scale || !aligned16(chan_max) || !aligned16(perm) ||
+      !aligned16(inv_perm) || !aligned16(group_scale)) {
+    set_error("chan_max, perm, inv_perm and group_scale must be non-NULL and 16-byte aligned");
+    return PQ_ERR_INVALID_ARG;
+  }
+  return cuda_fail(launch_rrs_prepare(plan, X, T, ldx, chan_max, perm, inv_perm, group_scale,
+                                      reinterpret_cast<cudaStream_t>(stream)),
+                   "pq_rrs_prepare launch");
+}
+
+extern "C" pq_status pq_rrs_transform_quant(const pq_plan* plan, const void* X, int64_t T, int64_t ldx,
+                                            const int32_t* perm, const float* group_scale, uint8_t* codes,
+                                            float* token_scales, void* stream) {
+  clear_error();
+  pq_status st = check_rrs_plan(plan);
+  if (st != PQ_OK) return st;
+  st = check_rows_arg(X, T, ldx, plan->D, "X");
+  if (st != PQ_OK) return st;
+  if (!perm || !group_scale || !codes || !token_scales || !aligned16(perm) || !aligned16(group_scale) ||
+      !aligned16(codes) || !aligned16(token_scales)) {
+    set_error("perm, group_scale, codes and token_scales must be non-NULL and 16-byte aligned");
+    return PQ_ERR_INVALID_ARG;
+  }
+  return cuda_fail(launch_rrs_rows(plan, X, T, ldx, 0, perm, group_scale, codes, token_scales,
+                                   reinterpret_cast<cudaStream_t>(stream)),
+                   "pq_rrs_transform_quant launch");
+}
+
+extern "C" pq_status pq_rrs_pack_weights(const pq_plan* plan, const void* W, int64_t N, const int32_t* perm,
+                                         const float* group_scale, uint8_t* codes_W, float* scales_W,
+                                         void* stream) {
+  clear_error();
+  pq_status st = check_rrs_plan(plan);
+  if (st != PQ_OK) return st;
+  st = check_rows_arg(W, N, plan->D, plan->D, "W");
+  if (st != PQ_OK) return st;
+  if (!perm || !group_scale || !codes_W || !scales_W || !aligned16(perm) || !aligned16(group_scale) ||
+      !aligned16(codes_W) || !aligned16(scales_W)) {
+    set_error("perm, group_scale, codes_W and scales_W must be non-NULL and 16-byte aligned");
+    return PQ_ERR_INVALID_ARG;
+  }
+  return cuda_fail(launch_rrs_rows(plan, W, N, plan->D, 1, perm, group_scale, codes_W, scales_W,
+                                   reinterpret_cast<cudaStream_t>(stream)),
+                   "pq_rrs_pack_weights launch");
+}
+
+extern "C" pq_status pq_rrs_gemm(const uint8_t* codes_A, const float* token_scales, const uint8_t* codes_W,
+                                 const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
+                                 pq_out_dtype out_dtype, void* stream) {
+  clear_error();
+  pq_status st = check_gemm_args(codes_A, token_scales, codes_W, scales_W, T, N, D, g, Y, out_dtype);
+  if (st != PQ_OK) return st;
+  return gemm_run(codes_A, token_scales, codes_W, scales_W, T, N, D, Y, out_dtype,
+                  reinterpret_cast<cudaStream_t>(stream), /*row_scale=*/true);
+}
+
 extern "C" pq_status pq_w4a4_gemm_launch_count(int64_t T, int64_t N, int64_t D, int* launches) {
   clear_error();
   if (!launches) {

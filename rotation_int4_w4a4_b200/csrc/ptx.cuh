@@ -154,6 +154,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_
       : "memory");
 }
 
+// 3-D tiled load into this CTA's shared memory (no multicast); x innermost.
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_t* bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+
 // Same load for a CTA pair (tcgen05 cta_group::2): the tile lands in this CTA's shared memory
 // and its bytes complete on `bar_cluster`, an mbarrier of this CTA or of its peer given by its
 // shared::cluster address.  No multicast.
@@ -412,6 +421,14 @@ __device__ __forceinline__ void mul_fma2(uint64_t& acc2, uint32_t d0, uint32_t d
   asm("{ .reg .b64 d; mov.b64 d, {%1, %2}; mul.rn.f32x2 d, d, %3; fma.rn.f32x2 %0, d, %4, %0; }"
       : "+l"(acc2)
       : "r"(d0), "r"(d1), "l"(s2), "l"(t2), "r"(after));
+}
+
+// acc2 += (d0, d1) * s2 on a float32 pair (one packed FMA).  `after` orders it after the wait
+// for d0, d1, as in mul_fma2.
+__device__ __forceinline__ void fma2(uint64_t& acc2, uint32_t d0, uint32_t d1, uint64_t s2, uint32_t after) {
+  asm("{ .reg .b64 d; mov.b64 d, {%1, %2}; fma.rn.f32x2 %0, d, %3, %0; }"
+      : "+l"(acc2)
+      : "r"(d0), "r"(d1), "l"(s2), "r"(after));
 }
 
 // Two float32 values from shared memory (byte addresses a and a + stride) as one pair.

@@ -96,10 +96,17 @@ __device__ __forceinline__ uint32_t rt_pack8(const float* v, float inv) {
 // Tiles are numbered group-major: tile = gi * row_blocks + rb.  CTA c owns [begin, end).
 // terms: 1 (R exact in bf16) or 2 (R_hi + R_lo).  r_groups: number of distinct matrices (G, or 1
 // when every group uses the same one).  scale_mult: stored scale = max|y| * scale_mult.
+// kColMax: instead of quantising, the per-channel maximum of |y| over all rows (RRS page, main
+// equation: s_j = max |(X_rot)_j|).  The operands are swapped (D = R^T X^T: tensor-memory lanes
+// are output channels, columns are rows), so each epilogue thread owns one channel and takes
+// its maximum over the tile's 128 rows in registers; the result (times scale_mult) is merged
+// into chan_max[channel] with an unsigned atomic maximum on the float's bits (all values are
+// non-negative, for which the bit order is the numeric order).  Rows past the end read as zeros.
+template <bool kColMax>
 __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
     const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmR, int64_t rows, int G,
     int row_blocks, int64_t num_tiles, int terms, int r_groups, float scale_mult, uint8_t* __restrict__ codes,
-    float* __restrict__ scales, unsigned int* status) {
+    float* __restrict__ scales, unsigned int* __restrict__ chan_max, unsigned int* status) {
   extern __shared__ unsigned char smem_raw[];
   RotSmem& S = *reinterpret_cast<RotSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -197,9 +204,11 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
             const uint32_t a0 = ptx::smem_addr(S.x[s][kb]);
             const uint32_t b0 = ptx::smem_addr(S.r[term][kb]);
 #pragma unroll
-            for (int k = 0; k < 4; ++k, ++n)   // K16 per MMA = 32 bytes along the swizzled row
-              ptx::umma_f16(d, ptx::smem_desc_sw128(a0 + 32 * k), ptx::smem_desc_sw128(b0 + 32 * k), kIdescBf16,
-                            n > 0 ? 1u : 0u);
+            for (int k = 0; k < 4; ++k, ++n) {   // K16 per MMA = 32 bytes along the swizzled row
+              const uint64_t da = ptx::smem_desc_sw128(a0 + 32 * k), db = ptx::smem_desc_sw128(b0 + 32 * k);
+              if (kColMax) ptx::umma_f16(d, db, da, kIdescBf16, n > 0 ? 1u : 0u);   // D = R^T X^T
+              else ptx::umma_f16(d, da, db, kIdescBf16, n > 0 ? 1u : 0u);           // D = X R
+            }
           }
         ptx::umma_commit(&S.x_empty[s]);
         ptx::umma_commit(&S.acc_full[b]);
@@ -237,6 +246,11 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
       float m = 0.0f;
 #pragma unroll
       for (int i = 0; i < 128; ++i) m = fmaxf(m, fabsf(y[i]));
+      if constexpr (kColMax) {
+        // this thread's lane is output channel rl of group gi; its columns are the tile's rows
+        atomicMax(chan_max + (int64_t)gi * 128 + rl, __float_as_uint(m * scale_mult));
+        continue;
+      }
       const float inv = m > 0.0f ? 7.0f * __frcp_rn(m) : 0.0f;
       if (t < rows) {
         uint4* dst = reinterpret_cast<uint4*>(codes + t * (int64_t)G * 64 + gi * 64);
@@ -310,8 +324,25 @@ cudaError_t make_u8_tile_map(CUtensorMap* map, const void* base, int64_t rows, i
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// bf16 rows [rows][D] (row stride ld elements) seen as [rows][D/64][64]: a box of box_rows whole
+// rows lands as D/64 * box_rows lines of 128 bytes with the 128-byte swizzle (line L's 16-byte
+// chunk c at L * 128 + ((c ^ (L mod 8)) * 16)); rows past the end read as zero.  D / 64 <= 256.
+cudaError_t make_bf16_row_lines_map(CUtensorMap* map, const void* base, int64_t rows, int64_t D, int64_t ld,
+                                    int box_rows) {
+  EncodeTiledFnR enc = encode_fn_r();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[3] = {64, (cuuint64_t)(D / 64), (cuuint64_t)rows};
+  cuuint64_t strides[2] = {128, (cuuint64_t)ld * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)(D / 64), (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
-                              uint8_t* codes, float* scales, cudaStream_t stream) {
+                              uint8_t* codes, float* scales, cudaStream_t stream, unsigned int* chan_max) {
   if (rows <= 0) return cudaSuccess;
   const bool givens = plan->kind == PQ_GIVENS;
   const int terms = givens ? 2 : 1;
@@ -329,11 +360,22 @@ cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, 
   // Givens: scale = m / 7.  Hadamard: R = H unnormalised, so y is sqrt(128) times the
   // orthonormal rotation and scale = m / (7 sqrt(128)).
   const float scale_mult = givens ? (1.0f / 7.0f) : 0.012626906806902634f;
+  if (chan_max) {
+    // column maxima of the normalised rotation: max |x R| (Hadamard: R unnormalised, so / sqrt(128))
+    static std::atomic<bool> attr_cm[kMaxDevices];
+    e = set_kernel_attributes(reinterpret_cast<const void*>(rotate_mma_kernel<true>), (int)kRotSmemBytes, attr_cm);
+    if (e != cudaSuccess) return e;
+    rotate_mma_kernel<true><<<grid, RT_THREADS, kRotSmemBytes, stream>>>(
+        tmX, tmR, rows, plan->G, row_blocks, tiles, terms, r_groups, givens ? 1.0f : 0.088388347648318440550f,
+        nullptr, nullptr, chan_max, plan->d_status);
+    return cudaGetLastError();
+  }
   static std::atomic<bool> attr_done[kMaxDevices];
-  e = set_kernel_attributes(reinterpret_cast<const void*>(rotate_mma_kernel), (int)kRotSmemBytes, attr_done);
+  e = set_kernel_attributes(reinterpret_cast<const void*>(rotate_mma_kernel<false>), (int)kRotSmemBytes, attr_done);
   if (e != cudaSuccess) return e;
-  rotate_mma_kernel<<<grid, RT_THREADS, kRotSmemBytes, stream>>>(tmX, tmR, rows, plan->G, row_blocks, tiles, terms,
-                                                                r_groups, scale_mult, codes, scales, plan->d_status);
+  rotate_mma_kernel<false><<<grid, RT_THREADS, kRotSmemBytes, stream>>>(tmX, tmR, rows, plan->G, row_blocks, tiles,
+                                                                       terms, r_groups, scale_mult, codes, scales,
+                                                                       nullptr, plan->d_status);
   return cudaGetLastError();
 }
 

@@ -27,6 +27,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "rows.cuh"
 
 namespace pq {
 namespace {
@@ -35,7 +36,6 @@ constexpr int SR_ROWS = 128;                          // rows per tile = threads
 constexpr int SR_STAGES = 2;
 constexpr uint32_t kSrTileBytes = SR_ROWS * 128 * 2;  // one tile: 32 KB of bf16
 constexpr uint64_t kSrWaitNs = 2000000000ull;         // 2 s
-constexpr float kSrRoundMagic = 12582912.0f;          // 1.5 * 2^23
 constexpr float kSrScaleHadamard = 0.012626906806902634f;   // 1/(7*sqrt(128)), float-rounded
 
 enum : int { SR_COLMAX = PQ_SR_COLMAX, SR_PRE = PQ_SR_PRE, SR_POST = PQ_SR_POST, SR_NONE = PQ_SR_NONE };
@@ -52,51 +52,6 @@ constexpr size_t kSrSmemBytes = sizeof(SrSmem) + 1024;
 // Byte offset of the 16-byte chunk j (channels 8j..8j+7 of a K-block) of row r in a tile
 // loaded with the 128-byte swizzle: chunk index XOR (row mod 8).
 __device__ __forceinline__ uint32_t sr_chunk(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
-
-__device__ __forceinline__ void sr_bf16x8(const uint4& w, float* v) {
-  v[0] = __uint_as_float(w.x << 16);
-  v[1] = __uint_as_float(w.x & 0xFFFF0000u);
-  v[2] = __uint_as_float(w.y << 16);
-  v[3] = __uint_as_float(w.y & 0xFFFF0000u);
-  v[4] = __uint_as_float(w.z << 16);
-  v[5] = __uint_as_float(w.z & 0xFFFF0000u);
-  v[6] = __uint_as_float(w.w << 16);
-  v[7] = __uint_as_float(w.w & 0xFFFF0000u);
-}
-
-// Unnormalised Walsh-Hadamard transform of 128 register values, Sylvester order (Hadamard page
-// §4.2 butterflies): stage h maps (v[i], v[i + h]) to (v[i] + v[i + h], v[i] - v[i + h]).  The
-// first stage pairs neighbours; the others run on packed float pairs.
-__device__ __forceinline__ void sr_fwht128(float (&v)[128]) {
-#pragma unroll
-  for (int i = 0; i < 128; i += 2) {
-    const float a = v[i], b = v[i + 1];
-    v[i] = a + b;
-    v[i + 1] = a - b;
-  }
-#pragma unroll
-  for (int h = 2; h < 128; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 128; i += 2) {
-      if ((i & h) == 0) {
-        const uint64_t P = ptx::f2_pack(v[i], v[i + 1]), Q = ptx::f2_pack(v[i + h], v[i + h + 1]);
-        ptx::f2_unpack(ptx::f2_add(P, Q), v[i], v[i + 1]);
-        ptx::f2_unpack(ptx::f2_sub(P, Q), v[i + h], v[i + h + 1]);
-      }
-    }
-  }
-}
-
-// 8 values -> 8 nibbles: byte k = q[2k] | q[2k+1] << 4, q = RNE(v * inv) (|q| <= 7); the FMA with
-// 1.5 * 2^23 leaves q's two's-complement low bits in the low byte.
-__device__ __forceinline__ uint32_t sr_pack8(const float* v, float inv) {
-  uint32_t b[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) b[k] = __float_as_uint(fmaf(v[k], inv, kSrRoundMagic));
-  const uint32_t even = __byte_perm(__byte_perm(b[0], b[2], 0x0040), __byte_perm(b[4], b[6], 0x0040), 0x5410);
-  const uint32_t odd = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
-  return (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
-}
 
 __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
     const __grid_constant__ CUtensorMap tmX, int64_t rows, int G, int64_t num_tiles, int mode,
@@ -184,7 +139,7 @@ __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
     for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        sr_bf16x8(*reinterpret_cast<const uint4*>(S.x[s][kb] + sr_chunk(t, j)), v + 64 * kb + 8 * j);
+        row_bf16x8(*reinterpret_cast<const uint4*>(S.x[s][kb] + sr_chunk(t, j)), v + 64 * kb + 8 * j);
     __syncthreads();   // every row (and column) of stage s is read; S.mul is complete
     if (t == 0 && tile + 2 * stride < num_tiles) issue(tile + 2 * stride, s);
 
@@ -198,7 +153,7 @@ __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
         v[i + 3] *= f.w;
       }
     }
-    sr_fwht128(v);
+    row_fwht128(v);
     if (mode == SR_POST) {
 #pragma unroll
       for (int i = 0; i < 128; i += 4) {
@@ -218,8 +173,8 @@ __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
       uint4* dst = reinterpret_cast<uint4*>(codes + row * (D / 2) + gi * 64);
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        dst[q] = make_uint4(sr_pack8(v + 32 * q, inv), sr_pack8(v + 32 * q + 8, inv),
-                            sr_pack8(v + 32 * q + 16, inv), sr_pack8(v + 32 * q + 24, inv));
+        dst[q] = make_uint4(row_pack8(v + 32 * q, inv), row_pack8(v + 32 * q + 8, inv),
+                            row_pack8(v + 32 * q + 16, inv), row_pack8(v + 32 * q + 24, inv));
       scales[row * G + gi] = m * kSrScaleHadamard;
     }
   }

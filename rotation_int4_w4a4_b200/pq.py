@@ -27,6 +27,7 @@ KINDS = {"hadamard": PQ_HADAMARD, "givens": PQ_GIVENS, "smooth_hadamard": PQ_SMO
 # Every symbol the header declares.
 EXPORTS = ("pq_select_pairs", "pq_make_plan", "pq_destroy_plan", "pq_transform_quant",
            "pq_pack_weights", "pq_w4a4_gemm", "pq_w4a4_gemm_noalloc", "pq_w4a4_gemm_launch_count",
+           "pq_rrs_prepare", "pq_rrs_transform_quant", "pq_rrs_pack_weights", "pq_rrs_gemm",
            "pq_check_status",
            "pq_selftest_wait_timeout", "pq_status_string", "pq_last_error")
 
@@ -48,6 +49,14 @@ lib.pq_w4a4_gemm_noalloc.argtypes = lib.pq_w4a4_gemm.argtypes
 lib.pq_w4a4_gemm_noalloc.restype = _i32
 lib.pq_w4a4_gemm_launch_count.argtypes = [_i64, _i64, _i64, _c.POINTER(_i32)]
 lib.pq_w4a4_gemm_launch_count.restype = _i32
+lib.pq_rrs_prepare.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]
+lib.pq_rrs_prepare.restype = _i32
+lib.pq_rrs_transform_quant.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]
+lib.pq_rrs_transform_quant.restype = _i32
+lib.pq_rrs_pack_weights.argtypes = [_vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp]
+lib.pq_rrs_pack_weights.restype = _i32
+lib.pq_rrs_gemm.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _i32, _vp]
+lib.pq_rrs_gemm.restype = _i32
 lib.pq_selftest_wait_timeout.argtypes = [_u64, _vp]
 lib.pq_selftest_wait_timeout.restype = _i32
 lib.pq_check_status.argtypes = [_vp, _vp]
@@ -97,7 +106,7 @@ def _arg(x, name, dtype, need, rows_strided=False):
         return _ptr(x)
     import torch
     want = {"bf16": (torch.bfloat16,), "u8": (torch.uint8,), "f32": (torch.float32,),
-            "y": (torch.float32, torch.bfloat16)}[dtype]
+            "i32": (torch.int32,), "y": (torch.float32, torch.bfloat16)}[dtype]
     if x.dtype not in want:
         raise ValueError(f"{name}: dtype {x.dtype} is not accepted (expected {' or '.join(map(str, want))})")
     p = _ptr(x, rows_strided)
@@ -207,7 +216,7 @@ def pq_w4a4_gemm(codes_A, scales_A, codes_W, scales_W, Y, T=None, N=None, D=None
     _check(lib.pq_w4a4_gemm(*ptrs[:4], T, N, D, g, ptrs[4], out_dtype, _stream(stream)), "pq_w4a4_gemm")
 
 
-def _gemm_args(codes_A, scales_A, codes_W, scales_W, Y, T, N, D, g, out_dtype):
+def _gemm_args(codes_A, scales_A, codes_W, scales_W, Y, T, N, D, g, out_dtype, sa_per_token=False):
     """Sizes, output dtype and checked pointers shared by the two GEMM entry points."""
     T = codes_A.shape[0] if T is None else T
     N = codes_W.shape[0] if N is None else N
@@ -222,7 +231,8 @@ def _gemm_args(codes_A, scales_A, codes_W, scales_W, Y, T, N, D, g, out_dtype):
     elif out_dtype is None:
         out_dtype = PQ_OUT_F32
     G = D // g if g else 0
-    ptrs = (_arg(codes_A, "codes_A", "u8", T * D // 2), _arg(scales_A, "scales_A", "f32", T * G),
+    ptrs = (_arg(codes_A, "codes_A", "u8", T * D // 2),
+            _arg(scales_A, "token_scales" if sa_per_token else "scales_A", "f32", T if sa_per_token else T * G),
             _arg(codes_W, "codes_W", "u8", N * D // 2), _arg(scales_W, "scales_W", "f32", N * G),
             _arg(Y, "Y", "y", T * N))
     return T, N, D, out_dtype, ptrs
@@ -234,6 +244,54 @@ def pq_w4a4_gemm_noalloc(codes_A, scales_A, codes_W, scales_W, Y, T=None, N=None
     T, N, D, out_dtype, ptrs = _gemm_args(codes_A, scales_A, codes_W, scales_W, Y, T, N, D, g, out_dtype)
     _check(lib.pq_w4a4_gemm_noalloc(*ptrs[:4], T, N, D, g, ptrs[4], out_dtype, _stream(stream)),
            "pq_w4a4_gemm_noalloc")
+
+
+def pq_rrs_prepare(plan: Plan, X, chan_max, perm, inv_perm, group_scale, T=None, ldx=None, stream=None) -> None:
+    """Channel maxima of the rotated activations, their descending order and the smoothing scale
+    of each reordered group of 128 (device tensors: float32 [D], int32 [D], int32 [D], float32 [G])."""
+    T = X.shape[0] if T is None else T
+    ldx = X.stride(0) if ldx is None else ldx
+    D, G = plan.D, plan.D // plan.g
+    xp = _arg(X, "X", "bf16", (T - 1) * ldx + D if T > 0 else 0, rows_strided=True)
+    _check(lib.pq_rrs_prepare(plan.handle, xp, T, ldx, _arg(chan_max, "chan_max", "f32", D),
+                              _arg(perm, "perm", "i32", D), _arg(inv_perm, "inv_perm", "i32", D),
+                              _arg(group_scale, "group_scale", "f32", G), _stream(stream)), "pq_rrs_prepare")
+
+
+def pq_rrs_transform_quant(plan: Plan, X, perm, group_scale, codes, token_scales, T=None, ldx=None,
+                           stream=None) -> None:
+    """Smoothed, reordered activations quantised per token: codes uint8 [T, D/2], float32 [T]."""
+    T = X.shape[0] if T is None else T
+    ldx = X.stride(0) if ldx is None else ldx
+    D, G = plan.D, plan.D // plan.g
+    xp = _arg(X, "X", "bf16", (T - 1) * ldx + D if T > 0 else 0, rows_strided=True)
+    _check(lib.pq_rrs_transform_quant(plan.handle, xp, T, ldx, _arg(perm, "perm", "i32", D),
+                                      _arg(group_scale, "group_scale", "f32", G),
+                                      _arg(codes, "codes", "u8", T * D // 2),
+                                      _arg(token_scales, "token_scales", "f32", T), _stream(stream)),
+           "pq_rrs_transform_quant")
+
+
+def pq_rrs_pack_weights(plan: Plan, W, perm, group_scale, codes_W, scales_W, N=None, stream=None) -> None:
+    """Reordered weights quantised per group, smoothing scales folded into scales_W [N, G]."""
+    N = W.shape[0] if N is None else N
+    D, G = plan.D, plan.D // plan.g
+    _check(lib.pq_rrs_pack_weights(plan.handle, _arg(W, "W", "bf16", N * D), N, _arg(perm, "perm", "i32", D),
+                                   _arg(group_scale, "group_scale", "f32", G),
+                                   _arg(codes_W, "codes_W", "u8", N * D // 2),
+                                   _arg(scales_W, "scales_W", "f32", N * G), _stream(stream)),
+           "pq_rrs_pack_weights")
+
+
+def pq_rrs_gemm(codes_A, token_scales, codes_W, scales_W, Y, T=None, N=None, D=None, g=128, out_dtype=None,
+                stream=None) -> None:
+    """Y [T, N] = token_scales[t] * sum_G scales_W[n, G] d_G (device tensors)."""
+    T = codes_A.shape[0] if T is None else T
+    N = codes_W.shape[0] if N is None else N
+    D = codes_A.shape[1] * 2 if D is None else D
+    T, N, D, out_dtype, ptrs = _gemm_args(codes_A, token_scales, codes_W, scales_W, Y, T, N, D, g, out_dtype,
+                                          sa_per_token=True)
+    _check(lib.pq_rrs_gemm(*ptrs[:4], T, N, D, g, ptrs[4], out_dtype, _stream(stream)), "pq_rrs_gemm")
 
 
 def pq_w4a4_gemm_launch_count(T: int, N: int, D: int) -> int:
