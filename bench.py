@@ -410,7 +410,7 @@ class Setup:
             pairs = pq.pq_select_pairs(wl.pair_seed, wl.D, wl.g, wl.K, wl.g // 2)
             self.plan = pq.Plan("givens", wl.D, K=wl.K, pairs=pairs, angles=wl.angles, beta=wl.beta)
         else:
-            self.plan = pq.Plan(wl.kind, wl.D)
+            self.plan = pq.Plan(wl.kind, wl.D, g=wl.g)
         T, D, N, G = wl.T, wl.D, wl.N, wl.D // wl.g
         self.X0, self.W0 = dev_bf16(wl.X, dev), dev_bf16(wl.W, dev)
         self.smooth_w = torch.ones(D, dtype=torch.float32, device=dev) if wl.kind == "smooth_hadamard" else None
@@ -441,7 +441,7 @@ class Setup:
         pq, plan = self.pq, self.plan
         return (lambda: pq.pq_transform_quant(plan, bs["X"], bs["ca"], bs["sa"], bs["sm"], stream=stream),
                 lambda: pq.pq_pack_weights(plan, bs["W"], bs["cw"], bs["sw"], self.smooth_w, stream=stream),
-                lambda: pq.pq_w4a4_gemm(bs["ca"], bs["sa"], bs["cw"], bs["sw"], bs["Y"], stream=stream))
+                lambda: pq.pq_w4a4_gemm(bs["ca"], bs["sa"], bs["cw"], bs["sw"], bs["Y"], g=self.wl.g, stream=stream))
 
     def run_step(self, i, stream):
         for c in self.calls(self.sets[i % self.nsets], stream):
@@ -549,12 +549,17 @@ def e2e_run(args, setup, stream):
     return total / n, hX.numel() * 2 + hW.numel() * 2, hY.numel() * 4
 
 
-def measure_also(name, args, dev, stream, peaks, peak_src):
-    """Components of another workload (fewer steps, same method), for the extra keys."""
+def measure_also(name, args, dev, stream, peaks, peak_src, g=None):
+    """Components of another workload (fewer steps, same method), for the extra keys; g: the same
+    workload at another group size (block-Hadamard workloads)."""
+    import dataclasses
+
     import torch
 
     from rotation_int4_w4a4_b200 import inputs
     wl = inputs.workload(name)
+    if g is not None:
+        wl = dataclasses.replace(wl, g=g, name=f"{name}_g{g}")
     setup = Setup(wl, dev, "flush")
     for i in range(max(3, args.warmup)):
         setup.flush()
@@ -698,6 +703,8 @@ def run_ours(args, wl, rank, world, local_rank):
     if world == 1 and not args.no_also and args.workload == DEFAULT_WORKLOAD and args.T is None:
         for name in ("up_proj", "q_proj"):
             also[name] = measure_also(name, args, dev, stream, peaks, peak_src)
+        for g in (64, 256):
+            also[f"q_proj_g{g}"] = measure_also("q_proj", args, dev, stream, peaks, peak_src, g=g)
         also["rrs_down_proj"] = measure_rrs(args, dev, stream, peaks, peak_src)
     if rank != 0:
         return

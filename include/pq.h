@@ -20,7 +20,7 @@
  * Conventions
  *   X  bf16 [T][D] row-major, row stride ldx elements (activations, one row per token).
  *   W  bf16 [N][D] row-major (Y = X W^T).
- *   g  group size; only g = 128 is supported.  G = D / g groups per row.
+ *   g  group size: 128, 64 (Hadamard, Givens) or 256 (Hadamard); G = D / g groups per row.
  *   codes  uint8 [rows][D/2]: byte k holds element 2k in the low nibble and element 2k+1 in
  *          the high nibble, both two's complement in -8..7.
  *   scales float32 [rows][G]: per-group scale m/7, m = max |transformed value| in the group
@@ -56,7 +56,7 @@ extern "C" {
 typedef enum pq_status {
   PQ_OK = 0,
   PQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, stride, alignment or plan */
-  PQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. g != 128) */
+  PQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. a group size a kind lacks) */
   PQ_ERR_CUDA = 3,          /* a CUDA runtime call failed (message in pq_last_error) */
   PQ_ERR_ALLOC = 4,         /* a device allocation (plan tables, GEMM scratch) failed */
   PQ_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up (see pq_check_status) */
@@ -91,14 +91,18 @@ typedef struct pq_plan pq_plan;
  *   Then K layers: scan the shuffled list, take a pair when both channels are still free in
  *   this layer and the pair was not taken by an earlier layer; stop a layer at N pairs.
  *   pairs_out: host uint8 [D/g][K][g/2][2], caller-owned; slots past a layer's last pair are
- *   PQ_NO_PAIR.  Requires g = 128, D % g = 0, 1 <= K <= 64, 1 <= N <= g/2.
+ *   PQ_NO_PAIR.  Requires g = 64 or 128, D % g = 0, 1 <= K <= 64, 1 <= N <= g/2.
  */
 pq_status pq_select_pairs(uint64_t seed, int D, int g, int K, int N, uint8_t* pairs_out);
 
 /*
  * pq_make_plan — build the device tables for one transform.
  *   kind    PQ_HADAMARD | PQ_GIVENS | PQ_SMOOTH_HADAMARD.
- *   D, g    channels and group size (g must be 128, D % g == 0, D >= g).
+ *   D, g    channels and group size: D % 128 == 0, D % g == 0, and g = 128 for every kind,
+ *           64 for PQ_HADAMARD and PQ_GIVENS (ParoQuant page §4.1: smaller groups for layers
+ *           with many outliers), 256 for PQ_HADAMARD (§6: larger groups on mobile parts);
+ *           other combinations return PQ_ERR_UNSUPPORTED.  (Givens at g = 256 would need
+ *           256 x 256 matrices, which do not fit the rotation kernel's shared memory.)
  *   K       Givens layers (1..64); ignored otherwise.
  *   pairs   host uint8 [D/g][K][g/2][2] (Givens; NULL otherwise).  Within a layer of a group
  *           the valid pairs (i < j < g) must be disjoint; PQ_NO_PAIR slots are skipped.
@@ -109,8 +113,9 @@ pq_status pq_select_pairs(uint64_t seed, int D, int g, int K, int N, uint8_t* pa
  *           exp(+beta), so that the product is unchanged before quantisation.
  *   flags   PQ_FLAG_* bits.
  *   Givens: per group the K layers and exp(-+beta) are composed on the host in double precision
- *   into one 128 x 128 matrix (one for activations, one for weights), stored as a bf16 pair
- *   hi + lo (about 2^-17 relative); the transform is then a tensor-core product y = x R.
+ *   into one g x g matrix (one for activations, one for weights; at g = 64 two groups share a
+ *   128 x 128 block-diagonal matrix), stored as a bf16 pair hi + lo (about 2^-17 relative);
+ *   the transform is then a tensor-core product y = x R.
  *   The plan is created on the current device.  *out is set only on success.
  */
 pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int K, const uint8_t* pairs,
@@ -153,16 +158,18 @@ pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t N, const f
 
 /*
  * pq_w4a4_gemm — Y[t][n] = sum_G scales_A[t][G] * scales_W[n][G] * d_G[t][n], with
- * d_G = sum over the group's 128 channels of qa * qw, and the per-group scaling applied to
+ * d_G = sum over the group's g channels of qa * qw, and the per-group scaling applied to
  * each group's interim result in float32, groups summed in ascending order (RRS page main
  * equation, last line, and Fig. 4 step (3) with block size = group size).
  *   How d_G is formed: the int4 codes are widened to E4M3 (every integer -8..7 is exact in
  *   E4M3) and multiplied on the tensor cores by tcgen05.mma kind::f8f6f4 into a float32
  *   accumulator in tensor memory, one accumulator per group.  Every product is an integer of
- *   magnitude <= 64 and every partial sum an integer of magnitude <= 128 * 64 = 2^13, so each
+ *   magnitude <= 64 and every partial sum an integer of magnitude <= 256 * 64 = 2^14, so each
  *   is exact in float32 and d_G arrives exact (no int32 accumulator is involved).
  *   codes_A [T][D/2], scales_A [T][D/g], codes_W [N][D/2], scales_W [N][D/g]: device, dense.
- *   T >= 1, N >= 1 with N % 16 == 0, D % 128 == 0, g == 128.
+ *   T >= 1, N >= 1 with N % 16 == 0, D % 128 == 0, g in {64, 128, 256} with D % g == 0
+ *   (PQ_ERR_UNSUPPORTED for another g).  A group is g / 32 tensor-core K32 steps into its own
+ *   accumulator: two groups per 128-code K-block at g = 64, two K-blocks per group at g = 256.
  *   Y device [T][N] float32 (PQ_OUT_F32) or bf16 (PQ_OUT_BF16, RNE of the float32 result).
  *   Scales must be finite.
  *   Returns PQ_ERR_ALLOC if the stream-ordered scratch cannot be allocated.
@@ -268,14 +275,15 @@ pq_status pq_w4a4_gemm_noalloc(const uint8_t* codes_A, const float* scales_A,
 
 /*
  * pq_w4a4_gemm_launch_count — host-only query, no counterpart in the pages.  Writes to
- * *launches the number of kernels one pq_w4a4_gemm call with these sizes launches on the
- * current device.  T > 128: 2 (operand expansion, contraction) or 3 (plus the split-K
+ * *launches the number of kernels one pq_w4a4_gemm call with these sizes and g = 128 launches
+ * on the current device (pq_w4a4_gemm_launch_count_g: the same for group size g).  T > 128: 2 (operand expansion, contraction) or 3 (plus the split-K
  * reduction, chosen when the 256 x 256 output tiles fill at most half of the device's SM
  * pairs).  T <= 128: 1, or 2 with the group-range reduction.  pq_w4a4_gemm_noalloc never
  * splits: it launches 2 for T > 128 and 1 otherwise.  Sizes are validated as for
  * pq_w4a4_gemm (PQ_ERR_INVALID_ARG otherwise).  Without a usable device the count assumes 148 SMs.
  */
 pq_status pq_w4a4_gemm_launch_count(int64_t T, int64_t N, int64_t D, int* launches);
+pq_status pq_w4a4_gemm_launch_count_g(int64_t T, int64_t N, int64_t D, int g, int* launches);
 
 /*
  * pq_check_status — synchronises `stream`, then reads and clears the device status words

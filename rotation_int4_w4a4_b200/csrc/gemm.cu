@@ -156,23 +156,28 @@ __device__ __forceinline__ uint32_t codes_to_e4m3(uint32_t x) {
   return (pos & ~m) | (neg & m);
 }
 
-// One thread per 16 packed bytes (32 codes of one group): writes the 16 low-nibble codes at K
-// offset 16p and the 16 high-nibble codes at 64 + 16p of the group's 128-byte row.
+// One thread per 16 packed bytes (32 codes): K-block kb (128 codes, 64 packed bytes) holds the
+// chunk's 16 low-nibble codes and 16 high-nibble codes.  g >= 128: at K offsets 16p and 64 + 16p
+// of the block (the permutation stays inside each 128-code block, so inside each group);
+// g = 64: inside each 64-code half h = p / 2, at 64 h + 16 (p % 2) and 64 h + 32 + 16 (p % 2).
 __global__ void __launch_bounds__(256) expand_codes_kernel(const uint8_t* __restrict__ A, int64_t chunksA,
                                                            const uint8_t* __restrict__ W, int64_t chunksW,
-                                                           uint8_t* __restrict__ A8, uint8_t* __restrict__ W8) {
+                                                           uint8_t* __restrict__ A8, uint8_t* __restrict__ W8,
+                                                           int g64) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunksA + chunksW; i += stride) {
     const bool isA = i < chunksA;
     const int64_t c = isA ? i : i - chunksA;
     const uint4 w = __ldg(reinterpret_cast<const uint4*>(isA ? A : W) + c);
-    const int64_t group = c >> 2;          // 4 chunks of 16 bytes per 64-byte packed group
+    const int64_t kb = c >> 2;             // 4 chunks of 16 bytes per 64-byte packed K-block
     const int p = (int)(c & 3);
-    uint8_t* dst = (isA ? A8 : W8) + group * 128 + 16 * p;
-    *reinterpret_cast<uint4*>(dst) =
+    const int lo = g64 ? 64 * (p >> 1) + 16 * (p & 1) : 16 * p;
+    const int hi = lo + (g64 ? 32 : 64);
+    uint8_t* base = (isA ? A8 : W8) + kb * 128;
+    *reinterpret_cast<uint4*>(base + lo) =
         make_uint4(codes_to_e4m3(w.x & 0x0F0F0F0Fu), codes_to_e4m3(w.y & 0x0F0F0F0Fu),
                    codes_to_e4m3(w.z & 0x0F0F0F0Fu), codes_to_e4m3(w.w & 0x0F0F0F0Fu));
-    *reinterpret_cast<uint4*>(dst + 64) =
+    *reinterpret_cast<uint4*>(base + hi) =
         make_uint4(codes_to_e4m3((w.x >> 4) & 0x0F0F0F0Fu), codes_to_e4m3((w.y >> 4) & 0x0F0F0F0Fu),
                    codes_to_e4m3((w.z >> 4) & 0x0F0F0F0Fu), codes_to_e4m3((w.w >> 4) & 0x0F0F0F0Fu));
   }
@@ -193,6 +198,7 @@ __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, 
 struct Work {
   int m_tiles, n_tiles, num_tiles;
   int ksplit, gs, G;
+  int gsl;               // K32 slices per group (g / 32): 2, 4 or 8; a K-block holds 4
   int units;
   int first, stride;     // this CTA pair's first unit and the number of pairs in the grid
   int rank;              // 0 = even CTA (issues the pair's MMAs), 1 = odd CTA
@@ -226,13 +232,15 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
       for (int u = wk.first; u < wk.units && ok; u += wk.stride) {
         int m0, n0, kr, k0, k1;
         unit_coords(u, wk, m0, n0, kr, k0, k1);
-        for (int kg = k0; kg < k1; ++kg, ++step) {
+        // the unit's K-blocks (its groups start on a K-block boundary: ranges are 4 groups)
+        const int kb0 = k0 * wk.gsl / 4, kb1 = k1 * wk.gsl / 4;
+        for (int kb = kb0; kb < kb1; ++kb, ++step) {
           const int s = step % OP_STAGES;
           const uint32_t ph = (uint32_t)(step / OP_STAGES) & 1u;
           if (!wait_or_abort(S, &S.op_empty[s], ph ^ 1u, status)) { ok = false; break; }
           if (wk.rank == 0) ptx::mbar_arrive_expect_tx(&S.op_full[s], kTxBytes);
-          ptx::tma_load_2d_pair(S.opA[s], &tmA, full0 + 8u * s, kg * BK, m0 + BM * wk.rank);
-          ptx::tma_load_2d_pair(S.opB[s], &tmB, full0 + 8u * s, kg * BK, n0 + BN_HALF * wk.rank);
+          ptx::tma_load_2d_pair(S.opA[s], &tmA, full0 + 8u * s, kb * BK, m0 + BM * wk.rank);
+          ptx::tma_load_2d_pair(S.opB[s], &tmB, full0 + 8u * s, kb * BK, n0 + BN_HALF * wk.rank);
         }
       }
       // Drain: every stage's last use is released by the pair's MMAs (so every load issued has
@@ -250,28 +258,38 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
     // are released by one multicast commit.
     if (lane == 0 && wk.rank == 0) {
       constexpr uint32_t idesc = ptx::idesc_e4m3_f32(PAIR_M, BN);
-      int step = 0;
+      int step = 0;    // groups
+      int kstep = 0;   // K-blocks (operand stages) consumed
       bool ok = true;
       for (int u = wk.first; u < wk.units && ok; u += wk.stride) {
         int m0, n0, kr, k0, k1;
         unit_coords(u, wk, m0, n0, kr, k0, k1);
-        for (int kg = k0; kg < k1; ++kg, ++step) {
-          const int s = step % OP_STAGES;
-          const uint32_t ph = (uint32_t)(step / OP_STAGES) & 1u;
+        for (int kg = k0; kg < k1 && ok; ++kg, ++step) {
           const int b = step & 1;
           const uint32_t u = (uint32_t)(step >> 1);
           // the first use of each buffer passes at once (parity of the phase before the first)
           if (!wait_or_abort(S, &S.acc_empty[b], (u & 1u) ^ 1u, status)) { ok = false; break; }
-          if (!wait_or_abort(S, &S.op_full[s], ph, status)) { ok = false; break; }
           ptx::tc_fence_after();
-          const uint32_t a0 = ptx::smem_addr(S.opA[s]);
-          const uint32_t b0 = ptx::smem_addr(S.opB[s]);
           const uint32_t d = tmem + (uint32_t)b * BN;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)   // k = 0 overwrites the buffer: each group starts from 0
-            ptx::umma_e4m3_pair(d, ptx::smem_desc_sw128(a0 + 32 * k), ptx::smem_desc_sw128(b0 + 32 * k), idesc,
-                                k > 0 ? 1u : 0u);
-          ptx::umma_commit_pair(&S.op_empty[s], 0x3);
+          // The group's K32 slices (2, 4 or 8): a K-block's stage is awaited at its first slice
+          // and released after its fourth; slice 0 of the group overwrites the buffer.
+          for (int sl = 0; sl < wk.gsl; ++sl) {
+            const int sub = ((kg - k0) * wk.gsl + sl) & 3;
+            const int s = kstep % OP_STAGES;
+            if (sub == 0) {
+              if (!wait_or_abort(S, &S.op_full[s], (uint32_t)(kstep / OP_STAGES) & 1u, status)) { ok = false; break; }
+              ptx::tc_fence_after();
+            }
+            const uint32_t a0 = ptx::smem_addr(S.opA[s]);
+            const uint32_t b0 = ptx::smem_addr(S.opB[s]);
+            ptx::umma_e4m3_pair(d, ptx::smem_desc_sw128(a0 + 32 * sub), ptx::smem_desc_sw128(b0 + 32 * sub), idesc,
+                                sl > 0 ? 1u : 0u);
+            if (sub == 3) {
+              ptx::umma_commit_pair(&S.op_empty[s], 0x3);
+              ++kstep;
+            }
+          }
+          if (!ok) break;
           ptx::umma_commit_pair(&S.acc_full[b], 0x3);
         }
       }
@@ -452,7 +470,7 @@ template <bool kRow>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const float* __restrict__ scales_A, const float* __restrict__ scales_W, void* __restrict__ Y,
-    int T, int N, int G, int scales_vec16, int out_bf16, int m_tiles, int n_tiles, int ksplit, int gs,
+    int T, int N, int G, int gsl, int scales_vec16, int out_bf16, int m_tiles, int n_tiles, int ksplit, int gs,
     float* __restrict__ ws, unsigned int* status) {
   extern __shared__ unsigned char smem_raw[];
   GemmSmem& S = *reinterpret_cast<GemmSmem*>(
@@ -465,6 +483,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1) w4a4
   wk.ksplit = ksplit;
   wk.gs = gs;
   wk.G = G;
+  wk.gsl = gsl;
   wk.units = wk.num_tiles * ksplit;
   wk.rank = (int)ptx::cluster_ctarank();
   wk.first = (int)(blockIdx.x >> 1);
@@ -673,9 +692,9 @@ size_t gemm_scratch_bytes(int64_t T, int64_t N, int64_t D) {
 
 // Few tokens: the few-token kernel's group ranges.  Otherwise split-K when the tiles fill at most
 // half of the CTA pairs the device can run at once.
-int gemm_ksplit(int64_t T, int64_t N, int64_t D, int* gs_out) {
-  if (T <= kGemmSmallT) return gemm_small_ranges(T, N, D, gs_out);
-  const int G = (int)(D / 128);
+int gemm_ksplit(int64_t T, int64_t N, int64_t D, int g, int* gs_out) {
+  if (T <= kGemmSmallT) return gemm_small_ranges(T, N, D, g, gs_out);
+  const int G = (int)(D / g);
   const int64_t tiles = ((N + PAIR_M - 1) / PAIR_M) * ((T + BN - 1) / BN);
   const int pairs = device_sm_count() / 2;
   int ks = 1, gs = G;
@@ -689,8 +708,8 @@ int gemm_ksplit(int64_t T, int64_t N, int64_t D, int* gs_out) {
   return ks;
 }
 
-size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t D) {
-  const int ks = gemm_ksplit(T, N, D, nullptr);
+size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t D, int g) {
+  const int ks = gemm_ksplit(T, N, D, g, nullptr);
   return ks > 1 ? (size_t)ks * (size_t)T * (size_t)N * sizeof(float) : 0;
 }
 
@@ -705,10 +724,10 @@ pq_status launch_splitk_reduce(const float* ws, int ksplit, int64_t T, int64_t N
 }
 
 pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W, const float* scales_W,
-                      int64_t T, int64_t N, int64_t D, void* Y, pq_out_dtype out_dtype, uint8_t* scratch,
+                      int64_t T, int64_t N, int64_t D, int g, void* Y, pq_out_dtype out_dtype, uint8_t* scratch,
                       float* ws, unsigned int* status, cudaStream_t stream, bool row_scale) {
   if (T <= kGemmSmallT)
-    return gemm_small_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype, ws, status, stream,
+    return gemm_small_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype, ws, status, stream,
                              row_scale);
   uint8_t* A8 = scratch;
   uint8_t* W8 = scratch + (size_t)T * (size_t)D;
@@ -738,11 +757,11 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
     e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_kernel<true>), (int)kSmemBytes, attr_gemm_row);
     if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel attributes");
   }
-  expand_codes_kernel<<<egrid, 256, 0, stream>>>(codes_A, chunksA, codes_W, chunksW, A8, W8);
+  expand_codes_kernel<<<egrid, 256, 0, stream>>>(codes_A, chunksA, codes_W, chunksW, A8, W8, g == 64 ? 1 : 0);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "expand_codes_kernel launch");
-  int gs = (int)(D / 128);
-  const int ksplit = ws ? gemm_ksplit(T, N, D, &gs) : 1;
+  int gs = (int)(D / g);
+  const int ksplit = ws ? gemm_ksplit(T, N, D, g, &gs) : 1;
   const int64_t units = tiles * ksplit;
   int max_pairs = 0;
   st = gemm_max_pairs(sms, &max_pairs);
@@ -765,15 +784,15 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
     set_error("w4a4_gemm_kernel compiled with %d registers per thread, %u expected", num_regs, REG_LAUNCH);
     return PQ_ERR_CUDA;
   }
-  const int G = (int)(D / 128);
+  const int G = (int)(D / g), gsl = g / 32;
   const int scales_vec16 = (G % SC_GROUPS == 0) ? 1 : 0;   // rows of 16-byte multiples
   if (row_scale)
     w4a4_gemm_kernel<true><<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB, scales_A, scales_W, Y, (int)T, (int)N,
-                                                                      G, scales_vec16, out_dtype == PQ_OUT_BF16 ? 1 : 0,
+                                                                      G, gsl, scales_vec16, out_dtype == PQ_OUT_BF16 ? 1 : 0,
                                                                       m_tiles, n_tiles, ksplit, gs, ws, status);
   else
     w4a4_gemm_kernel<false><<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB, scales_A, scales_W, Y, (int)T, (int)N,
-                                                                       G, scales_vec16, out_dtype == PQ_OUT_BF16 ? 1 : 0,
+                                                                       G, gsl, scales_vec16, out_dtype == PQ_OUT_BF16 ? 1 : 0,
                                                                        m_tiles, n_tiles, ksplit, gs, ws, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel launch");
@@ -782,7 +801,7 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
 }
 
 pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W, const float* scales_W,
-                   int64_t T, int64_t N, int64_t D, void* Y, pq_out_dtype out_dtype, cudaStream_t stream,
+                   int64_t T, int64_t N, int64_t D, int g, void* Y, pq_out_dtype out_dtype, cudaStream_t stream,
                    bool row_scale) {
   unsigned int* status = nullptr;
   cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_gemm_status);
@@ -794,9 +813,9 @@ pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t*
   if (e != cudaSuccess) return cuda_fail(e, "scratch memory pool");
   // Operand scratch, then (small problems) the split-K partial tiles.
   const size_t op_bytes = (gemm_scratch_bytes(T, N, D) + 255) & ~(size_t)255;
-  const size_t ws_bytes = gemm_workspace_bytes(T, N, D);
+  const size_t ws_bytes = gemm_workspace_bytes(T, N, D, g);
   if (op_bytes + ws_bytes == 0)   // the few-token kernel without a split needs no scratch
-    return gemm_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype, nullptr, nullptr, status, stream,
+    return gemm_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype, nullptr, nullptr, status, stream,
                        row_scale);
   void* scratch = nullptr;
   e = cudaMallocFromPoolAsync(&scratch, op_bytes + ws_bytes, pool, stream);
@@ -805,7 +824,7 @@ pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t*
     return PQ_ERR_ALLOC;
   }
   float* ws = ws_bytes ? reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + op_bytes) : nullptr;
-  pq_status st = gemm_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype,
+  pq_status st = gemm_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype,
                              static_cast<uint8_t*>(scratch), ws, status, stream, row_scale);
   e = cudaFreeAsync(scratch, stream);
   if (st == PQ_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(gemm scratch)");

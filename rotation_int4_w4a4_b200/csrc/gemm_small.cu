@@ -5,21 +5,24 @@
 // packed weights: W is read from HBM once, as int4, and nothing is written back but Y.
 //
 // A work unit is 128 weight rows x a range of groups; persistent CTAs take the units in turn.
-//   warp 0      TMA: four groups per stage, as two boxes of two groups (128 contiguous bytes of
+// Codes move in K-blocks of 128 (64 packed bytes per row); a group is g / 128 of a block (g = 64),
+// one block (g = 128) or two (g = 256).
+//   warp 0      TMA: four K-blocks per stage, as two boxes of two blocks (128 contiguous bytes of
 //               each row, 128-byte swizzle) for the unit's 128 weight rows and for the NT token
 //               rows (rows past T read as zeros), into a ring of 2..4 stages.  Row segments of
-//               128 bytes rather than one group's 64 keep the L2 and DRAM requests large.
-//   warp 1      TMEM allocator and MMA issuer: 4 x tcgen05.mma kind::i8 (M128, N = NT, K32) per
-//               group into a ring of int32 accumulators (the first of the four overwrites).
-//   warps 4..7  widening (one warp per scheduler), one group at a time into a ring of operand
+//               128 bytes keep the L2 and DRAM requests large.
+//   warp 1      TMEM allocator and MMA issuer: g / 32 tcgen05.mma kind::i8 (M128, N = NT, K32) per
+//               group into a ring of int32 accumulators (the first of them overwrites).
+//   warps 4..7  widening (one warp per scheduler), one K-block at a time into a ring of operand
 //               stages deep enough to cover the MMA's completion latency: each packed byte's two
-//               nibbles become two int8
-//               values q * 16 (the nibble moved to the byte's top: one shift and one mask per four
-//               bytes, exact), written in the 128-byte-swizzled K-major operand layout.  Within each
-//               group the low nibbles land at K positions 0..63 and the high nibbles at 64..127, on
-//               both operands alike, so every dot product is unchanged; it comes out as 256 d_G,
-//               exact in int32 (|256 d_G| <= 2^21).  Eight consecutive threads take eight
-//               consecutive rows of one 16-byte column, which the swizzle spreads over all banks.
+//               nibbles become two int8 values q * 16 (the nibble moved to the byte's top: one
+//               shift and one mask per four bytes, exact), written in the 128-byte-swizzled
+//               K-major operand layout.  Within each 128-code block the low nibbles land at K
+//               positions 0..63 and the high nibbles at 64..127 (g = 64: within each 64-code
+//               half, 0..31 and 32..63), on both operands alike, so every group's dot product is
+//               unchanged; it comes out as 256 d_G, exact in int32 (|256 d_G| <= 2^22).  Eight
+//               consecutive threads take eight consecutive rows of one 16-byte column, which the
+//               swizzle spreads over all banks.
 //   warps 8..11 epilogue: one thread per weight row (TMEM lane), NT tokens; per group
 //               acc += float(256 d_G) * (sw / 256) * sa, the same float32 value and rounding as
 //               fl(d_G * sw) * sa, groups in ascending order.
@@ -44,7 +47,8 @@ namespace pq {
 namespace {
 
 constexpr int GS_M = 128;           // weight rows per unit (MMA M = TMEM lanes)
-constexpr int GS_GPS = 4;           // groups per packed-code stage (two 128-byte boxes)
+constexpr int GS_GPS = 4;           // group ranges are multiples of 4 groups
+constexpr int GS_KPS = 4;           // K-blocks (128 codes, 64 packed bytes) per packed-code stage
 constexpr int GS_SC = 8;            // groups of token scales staged per epilogue warp at a time
 constexpr int GS_THREADS = 384;     // warp 0 TMA, 1 MMA, 4..7 widening, 8..11 epilogue
 constexpr int GS_WIDEN0 = 4;        // first widening warp
@@ -107,13 +111,15 @@ __device__ __forceinline__ void gs_drain(uint64_t* bar, uint32_t parity) {
   (void)ptx::mbar_wait_bounded(bar, parity, &never, kGsWaitNs);
 }
 
-// One group of ROWS rows: the 64 packed bytes of row r sit in the `half` 64-byte half of the
-// row's 128-byte swizzled segment in `raw`; they become 128 int8 values in the row's 128-byte
-// swizzled operand row in `op` (16-byte chunk c stored at c XOR (row mod 8) in both).  Task i:
-// row i % ROWS, 16-byte column p = i / ROWS (low nibbles -> chunk p, high -> chunk p + 4).  All
-// loads are issued before any store.
+// One K-block (128 codes) of ROWS rows: the 64 packed bytes of row r sit in the `half` 64-byte
+// half of the row's 128-byte swizzled segment in `raw`; they become 128 int8 values in the row's
+// 128-byte swizzled operand row in `op` (16-byte chunk c stored at c XOR (row mod 8) in both).
+// Task i: row i % ROWS, 16-byte column p = i / ROWS.  g >= 128: low nibbles -> chunk p, high ->
+// chunk p + 4; g = 64 (two groups per block): low -> chunk 4 (p / 2) + p % 2, high -> that + 2,
+// so that each group's codes stay within its own 64 K positions.  All loads are issued before
+// any store.
 template <int ROWS>
-__device__ __forceinline__ void widen_group(const uint8_t* raw, uint8_t* op, int half, int ct) {
+__device__ __forceinline__ void widen_block(const uint8_t* raw, uint8_t* op, int half, int ct, int g64) {
   constexpr int TASKS = ROWS * 4, NTH = 32 * GS_WIDEN, PER = (TASKS + NTH - 1) / NTH;
   uint4 v[PER];
 #pragma unroll
@@ -129,12 +135,13 @@ __device__ __forceinline__ void widen_group(const uint8_t* raw, uint8_t* op, int
     const int i = ct + NTH * q;
     if (TASKS % NTH == 0 || i < TASKS) {
       const int row = i % ROWS, p = i / ROWS;
+      const int lo = g64 ? (((p & 2) << 1) | (p & 1)) : p, hi = lo + (g64 ? 2 : 4);
       const uint4 w = v[q];
       uint8_t* base = op + row * 128;
-      *reinterpret_cast<uint4*>(base + ((p ^ (row & 7)) << 4)) =
+      *reinterpret_cast<uint4*>(base + ((lo ^ (row & 7)) << 4)) =
           make_uint4((w.x << 4) & 0xF0F0F0F0u, (w.y << 4) & 0xF0F0F0F0u, (w.z << 4) & 0xF0F0F0F0u,
                      (w.w << 4) & 0xF0F0F0F0u);
-      *reinterpret_cast<uint4*>(base + (((p + 4) ^ (row & 7)) << 4)) =
+      *reinterpret_cast<uint4*>(base + ((hi ^ (row & 7)) << 4)) =
           make_uint4(w.x & 0xF0F0F0F0u, w.y & 0xF0F0F0F0u, w.z & 0xF0F0F0F0u, w.w & 0xF0F0F0F0u);
     }
   }
@@ -160,9 +167,12 @@ template <int NT, bool kRow>
 __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
     const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
     const float* __restrict__ scales_A, const float* __restrict__ scales_W, void* __restrict__ Y,
-    float* __restrict__ ws, int T, int N, int G, int ranges, int gs, int units, int out_bf16,
+    float* __restrict__ ws, int T, int N, int G, int gsl, int ranges, int gs, int units, int out_bf16,
     unsigned int* status) {
+  // gsl: K32 slices per group (g / 32 = 2, 4 or 8); a K-block of 128 codes holds 4, an operand
+  // stage is one K-block and a packed-code stage four.  Group ranges start on K-block boundaries.
   using Smem = SmallSmem<NT>;
+  const int g64 = gsl == 2 ? 1 : 0;
   constexpr int RAW = Smem::RAW, GS_OPS = Smem::OPS, GS_NACC = Smem::NACC;
   constexpr uint32_t kTmemCols = GS_NACC * NT < 32 ? 32 : GS_NACC * NT;
   constexpr uint32_t kRawBytes = 2 * GS_M * 128 + 2 * NT * 128;
@@ -211,13 +221,14 @@ __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const Unit w = unit_of(u, ranges, gs, G);
-        for (int kg0 = w.k0; kg0 < w.k1; kg0 += GS_GPS, ++ss) {
+        const int kb1 = w.k1 * gsl / 4;
+        for (int kq = w.k0 * gsl / 4; kq < kb1; kq += GS_KPS, ++ss) {
           const int s = ss % RAW;
           if (!gs_wait(S, &S.raw_empty[s], ((uint32_t)(ss / RAW) & 1u) ^ 1u, status)) { ok = false; break; }
           ptx::mbar_arrive_expect_tx(&S.raw_full[s], kRawBytes);
-          for (int b = 0; b < 2; ++b) {   // groups kg0 + 2b, kg0 + 2b + 1 (bytes past a row read as zeros)
-            ptx::tma_load_2d(S.rawW[s][b], &tmW, &S.raw_full[s], (kg0 + 2 * b) * 64, w.m0);
-            ptx::tma_load_2d(S.rawA[s][b], &tmA, &S.raw_full[s], (kg0 + 2 * b) * 64, 0);
+          for (int b = 0; b < 2; ++b) {   // K-blocks kq + 2b, kq + 2b + 1 (bytes past a row read as zeros)
+            ptx::tma_load_2d(S.rawW[s][b], &tmW, &S.raw_full[s], (kq + 2 * b) * 64, w.m0);
+            ptx::tma_load_2d(S.rawA[s][b], &tmA, &S.raw_full[s], (kq + 2 * b) * 64, 0);
           }
         }
       }
@@ -229,22 +240,34 @@ __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
     // ------------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = ptx::idesc_s8_s32(GS_M, NT);
-      int step = 0;
+      int step = 0;    // groups
+      int kstep = 0;   // operand stages (K-blocks) consumed
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const Unit w = unit_of(u, ranges, gs, G);
-        for (int kg = w.k0; kg < w.k1; ++kg, ++step) {
-          const int o = step % GS_OPS, b = step % GS_NACC;
+        for (int kg = w.k0; kg < w.k1 && ok; ++kg, ++step) {
+          const int b = step % GS_NACC;
           if (!gs_wait(S, &S.acc_empty[b], ((uint32_t)(step / GS_NACC) & 1u) ^ 1u, status)) { ok = false; break; }
-          if (!gs_wait(S, &S.op_full[o], (uint32_t)(step / GS_OPS) & 1u, status)) { ok = false; break; }
           ptx::tc_fence_after();
-          const uint32_t a0 = ptx::smem_addr(S.opW[o]), b0 = ptx::smem_addr(S.opA[o]);
           const uint32_t d = tmem + (uint32_t)(b * NT);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)   // K32 per MMA = 32 bytes along the swizzled row
-            ptx::umma_s8(d, ptx::smem_desc_sw128(a0 + 32 * k), ptx::smem_desc_sw128(b0 + 32 * k), idesc,
-                         k > 0 ? 1u : 0u);
-          ptx::umma_commit(&S.op_empty[o]);
+          // K32 per MMA = 32 bytes along the swizzled row; a stage is awaited at its first slice
+          // and released after its fourth; slice 0 of the group overwrites the buffer.
+          for (int sl = 0; sl < gsl; ++sl) {
+            const int sub = ((kg - w.k0) * gsl + sl) & 3;
+            const int o = kstep % GS_OPS;
+            if (sub == 0) {
+              if (!gs_wait(S, &S.op_full[o], (uint32_t)(kstep / GS_OPS) & 1u, status)) { ok = false; break; }
+              ptx::tc_fence_after();
+            }
+            const uint32_t a0 = ptx::smem_addr(S.opW[o]), b0 = ptx::smem_addr(S.opA[o]);
+            ptx::umma_s8(d, ptx::smem_desc_sw128(a0 + 32 * sub), ptx::smem_desc_sw128(b0 + 32 * sub), idesc,
+                         sl > 0 ? 1u : 0u);
+            if (sub == 3) {
+              ptx::umma_commit(&S.op_empty[o]);
+              ++kstep;
+            }
+          }
+          if (!ok) break;
           ptx::umma_commit(&S.acc_full[b]);
         }
       }
@@ -260,15 +283,16 @@ __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
     bool ok = true;
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       const Unit w = unit_of(u, ranges, gs, G);
-      for (int kg0 = w.k0; kg0 < w.k1 && ok; kg0 += GS_GPS, ++ss) {
+      const int kb1 = w.k1 * gsl / 4;
+      for (int kq = w.k0 * gsl / 4; kq < kb1 && ok; kq += GS_KPS, ++ss) {
         const int s = ss % RAW;
         if (!gs_warp_wait(S, &S.raw_full[s], (uint32_t)(ss / RAW) & 1u, status)) { ok = false; break; }
-        const int ng = min(GS_GPS, w.k1 - kg0);
-        for (int j = 0; j < ng; ++j, ++step) {
+        const int nk = min(GS_KPS, kb1 - kq);
+        for (int j = 0; j < nk; ++j, ++step) {
           const int o = step % GS_OPS;
           if (!gs_warp_wait(S, &S.op_empty[o], ((uint32_t)(step / GS_OPS) & 1u) ^ 1u, status)) { ok = false; break; }
-          widen_group<GS_M>(S.rawW[s][j >> 1], S.opW[o], j & 1, ct);
-          widen_group<NT>(S.rawA[s][j >> 1], S.opA[o], j & 1, ct);
+          widen_block<GS_M>(S.rawW[s][j >> 1], S.opW[o], j & 1, ct, g64);
+          widen_block<NT>(S.rawA[s][j >> 1], S.opA[o], j & 1, ct, g64);
           ptx::fence_proxy_async_smem();   // the tensor core reads these bytes through the async proxy
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&S.op_full[o]);
@@ -388,7 +412,7 @@ __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
 
 template <int NT, bool kRow>
 pq_status launch_small(const CUtensorMap& tmW, const CUtensorMap& tmA, const float* scales_A, const float* scales_W,
-                       void* Y, float* ws, int T, int N, int G, int ranges, int gs, int units, int out_bf16,
+                       void* Y, float* ws, int T, int N, int G, int gsl, int ranges, int gs, int units, int out_bf16,
                        unsigned int* status, cudaStream_t stream) {
   static std::atomic<bool> attr_done[kMaxDevices];
   cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_small_kernel<NT, kRow>),
@@ -412,7 +436,7 @@ pq_status launch_small(const CUtensorMap& tmW, const CUtensorMap& tmA, const flo
   }
   const int grid = std::min(units, device_sm_count());
   w4a4_gemm_small_kernel<NT, kRow><<<grid, GS_THREADS, small_smem_bytes<NT>(), stream>>>(
-      tmW, tmA, scales_A, scales_W, Y, ws, T, N, G, ranges, gs, units, out_bf16, status);
+      tmW, tmA, scales_A, scales_W, Y, ws, T, N, G, gsl, ranges, gs, units, out_bf16, status);
   return cuda_fail(cudaGetLastError(), "w4a4_gemm_small_kernel launch");
 }
 
@@ -426,8 +450,8 @@ static_assert(small_smem_bytes<16>() <= 232448 && small_smem_bytes<32>() <= 2324
 // second, partial wave would double the time of the CTAs that run it), and only while the
 // float32 partial tiles (written and read back, 8 T N bytes per range) stay within a quarter of
 // the packed weight bytes (N D / 2).  A range is a multiple of 4 groups (one packed-code stage).
-int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int* gs_out) {
-  const int G = (int)(D / 128);
+int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int g, int* gs_out) {
+  const int G = (int)(D / g);
   const int64_t m_tiles = (N + GS_M - 1) / GS_M;
   const int64_t fill = device_sm_count() / m_tiles;
   const int64_t traffic = std::max<int64_t>(1, D / (64 * T));
@@ -441,13 +465,13 @@ int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int* gs_out) {
 }
 
 pq_status gemm_small_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
-                            const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
+                            const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
                             pq_out_dtype out_dtype, float* ws, unsigned int* status, cudaStream_t stream,
                             bool row_scale) {
   const int NT = T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128;
-  const int G = (int)(D / 128);
+  const int G = (int)(D / g), gsl = g / 32;
   int gs = G;
-  const int ranges = ws ? gemm_small_ranges(T, N, D, &gs) : 1;
+  const int ranges = ws ? gemm_small_ranges(T, N, D, g, &gs) : 1;
   if (ranges == 1) gs = G;
   const int64_t m_tiles = (N + GS_M - 1) / GS_M;
   const int64_t units = m_tiles * ranges;
@@ -465,10 +489,10 @@ pq_status gemm_small_launch(const uint8_t* codes_A, const float* scales_A, const
   const int bf16 = out_dtype == PQ_OUT_BF16 ? 1 : 0;
   pq_status st;
 #define PQ_SMALL_CASE(W)                                                                                      \
-  st = row_scale ? launch_small<W, true>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, ranges, gs,  \
-                                         (int)units, bf16, status, stream)                                    \
-                 : launch_small<W, false>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, ranges, gs, \
-                                          (int)units, bf16, status, stream)
+  st = row_scale ? launch_small<W, true>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, gsl, ranges,  \
+                                         gs, (int)units, bf16, status, stream)                                    \
+                 : launch_small<W, false>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, gsl, ranges, \
+                                          gs, (int)units, bf16, status, stream)
   switch (NT) {
     case 16: PQ_SMALL_CASE(16); break;
     case 32: PQ_SMALL_CASE(32); break;

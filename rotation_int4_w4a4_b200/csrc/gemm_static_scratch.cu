@@ -60,7 +60,7 @@ pq_status device_setup(int dev, DeviceSetup* out) {
 
 pq_status gemm_run_static_scratch(const uint8_t* codes_A, const float* scales_A,
                                   const uint8_t* codes_W, const float* scales_W, int64_t T,
-                                  int64_t N, int64_t D, void* Y, pq_out_dtype out_dtype,
+                                  int64_t N, int64_t D, int g, void* Y, pq_out_dtype out_dtype,
                                   cudaStream_t stream) {
   const size_t need = gemm_scratch_bytes(T, N, D);
   if (need > (size_t)PQ_NOALLOC_SCRATCH_BYTES) {
@@ -79,7 +79,7 @@ pq_status gemm_run_static_scratch(const uint8_t* codes_A, const float* scales_A,
   DeviceSetup s;
   pq_status st = device_setup(dev, &s);
   if (st != PQ_OK) return st;
-  return gemm_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype, s.scratch,
+  return gemm_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype, s.scratch,
                      /*ws=*/nullptr, s.status, stream, /*row_scale=*/false);
 }
 

@@ -144,11 +144,11 @@ cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, 
 // Calls with at most this many tokens take the few-token kernel (gemm_small.cu): packed codes
 // read directly, int8 tensor-core products, no operand scratch.
 constexpr int64_t kGemmSmallT = 128;
-// Group ranges per 128-row weight tile of the few-token kernel (1 = no split).
-int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int* gs_out);
+// Group ranges per 128-row weight tile of the few-token kernel (1 = no split); g = group size.
+int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int g, int* gs_out);
 // The few-token GEMM (+ the split reduction when ws != nullptr and the sizes call for it).
 pq_status gemm_small_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
-                            const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
+                            const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
                             pq_out_dtype out_dtype, float* ws, unsigned int* status, cudaStream_t stream,
                             bool row_scale);
 // Y = sum over ksplit float32 partial [T][N] tiles in ws, ascending (gemm.cu).
@@ -157,19 +157,19 @@ pq_status launch_splitk_reduce(const float* ws, int ksplit, int64_t T, int64_t N
 // row_scale: scales_W holds per-(row, group) factors and scales_A one scale per token, applied
 // after the groups (the rotated-runtime-smoothing GEMM); otherwise both are per (row, group).
 pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
-                   const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
+                   const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
                    pq_out_dtype out_dtype, cudaStream_t stream, bool row_scale = false);
 // Bytes of operand scratch the GEMM needs: (T + N) * D for the expanded operands (none for the
 // few-token kernel).
 size_t gemm_scratch_bytes(int64_t T, int64_t N, int64_t D);
 // Split-K factor for a problem (1 = none) and the groups per range; the float32 partial-tile
 // workspace it needs (0 when unsplit), for whichever kernel the sizes select.
-int gemm_ksplit(int64_t T, int64_t N, int64_t D, int* gs_out);
-size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t D);
+int gemm_ksplit(int64_t T, int64_t N, int64_t D, int g, int* gs_out);
+size_t gemm_workspace_bytes(int64_t T, int64_t N, int64_t D, int g);
 // Expansion + contraction (+ split-K reduction) launches on `stream` using caller-provided
 // scratch; ws = nullptr disables split-K.
 pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
-                      const float* scales_W, int64_t T, int64_t N, int64_t D, void* Y,
+                      const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
                       pq_out_dtype out_dtype, uint8_t* scratch, float* ws, unsigned int* status,
                       cudaStream_t stream, bool row_scale);
 pq_status gemm_read_and_clear_status(unsigned int* bits);
@@ -180,7 +180,7 @@ cudaError_t gemm_status_address(unsigned int** status);
 // gemm_launch with the fixed device-array scratch of gemm_static_scratch.cu (no allocation).
 pq_status gemm_run_static_scratch(const uint8_t* codes_A, const float* scales_A,
                                   const uint8_t* codes_W, const float* scales_W, int64_t T,
-                                  int64_t N, int64_t D, void* Y, pq_out_dtype out_dtype,
+                                  int64_t N, int64_t D, int g, void* Y, pq_out_dtype out_dtype,
                                   cudaStream_t stream);
 
 }  // namespace pq

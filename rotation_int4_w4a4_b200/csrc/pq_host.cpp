@@ -62,7 +62,7 @@ extern "C" pq_status pq_select_pairs(uint64_t seed, int D, int g, int K, int N,
                                      uint8_t* pairs_out) {
   clear_error();
   if (!pairs_out) { set_error("pairs_out is NULL"); return PQ_ERR_INVALID_ARG; }
-  if (g != kGroup) { set_error("g=%d: only g=128 is supported", g); return PQ_ERR_UNSUPPORTED; }
+  if (g != 64 && g != 128) { set_error("g=%d: Givens pairs are drawn for g = 64 or 128", g); return PQ_ERR_UNSUPPORTED; }
   if (D < g || D % g != 0) { set_error("D=%d must be a positive multiple of g", D); return PQ_ERR_INVALID_ARG; }
   if (K < 1 || K > 64) { set_error("K=%d out of range 1..64", K); return PQ_ERR_INVALID_ARG; }
   if (N < 1 || N > g / 2) { set_error("N=%d out of range 1..g/2", N); return PQ_ERR_INVALID_ARG; }
@@ -140,15 +140,18 @@ static float bf16_value(uint16_t h) {
   return f;
 }
 
-// Givens, tensor-core operands.  Per group, R = G_0 G_1 ... G_{K-1} in float64 for the row-vector
-// convention y = x R: layer l's pair (i, j, theta) replaces columns (i, j) of R by
-// (c col_i - s col_j, s col_i + c col_j).  Column n is then scaled by exp(-beta_n) for the
+// Givens, tensor-core operands.  Per group of g channels, R = G_0 G_1 ... G_{K-1} in float64
+// for the row-vector convention y = x R: layer l's pair (i, j, theta) replaces columns (i, j) of
+// R by (c col_i - s col_j, s col_i + c col_j).  Column n is then scaled by exp(-beta_n) for the
 // activations and exp(+beta_n) for the weights (R diag(exp(beta)) = M^-T, the rotations being
-// orthogonal).  Stored transposed (entry [n][k] = R[k][n]) as bf16 R_hi + R_lo.
-static void build_rotation_operands(int G, int K, const uint8_t* pairs, const float* angles, const float* beta,
+// orthogonal).  The kernels take one 128 x 128 matrix per 128-channel tile: the group's R for
+// g = 128, the two groups' matrices on the diagonal for g = 64.  Stored transposed (entry
+// [n][k] = R[k][n]) as bf16 R_hi + R_lo, laid out [activations / weights][tile][term][n][k].
+static void build_rotation_operands(int D, int g, int K, const uint8_t* pairs, const float* angles, const float* beta,
                                     std::vector<uint16_t>& out) {
-  constexpr int g = kGroup, half = kGroup / 2;
-  out.assign((size_t)2 * G * 2 * g * g, 0);
+  constexpr int TW = 128;
+  const int G = D / g, tiles = D / TW, half = g / 2;
+  out.assign((size_t)2 * tiles * 2 * TW * TW, 0);
   std::vector<double> R((size_t)g * g);
   for (int gi = 0; gi < G; ++gi) {
     std::fill(R.begin(), R.end(), 0.0);
@@ -166,16 +169,17 @@ static void build_rotation_operands(int G, int K, const uint8_t* pairs, const fl
         }
       }
     }
+    const int ti = gi * g / TW, off = gi * g % TW;   // tile and the group's offset on its diagonal
     for (int which = 0; which < 2; ++which) {
-      uint16_t* hi = out.data() + ((size_t)(which * G + gi) * 2 + 0) * g * g;
-      uint16_t* lo = out.data() + ((size_t)(which * G + gi) * 2 + 1) * g * g;
+      uint16_t* hi = out.data() + ((size_t)(which * tiles + ti) * 2 + 0) * TW * TW;
+      uint16_t* lo = out.data() + ((size_t)(which * tiles + ti) * 2 + 1) * TW * TW;
       for (int n = 0; n < g; ++n) {
         const double cs = beta ? std::exp((which == 0 ? -1.0 : 1.0) * (double)beta[gi * g + n]) : 1.0;
         for (int k = 0; k < g; ++k) {
           const double v = R[(size_t)k * g + n] * cs;
           const uint16_t h = bf16_bits((float)v);
-          hi[(size_t)n * g + k] = h;
-          lo[(size_t)n * g + k] = bf16_bits((float)(v - (double)bf16_value(h)));
+          hi[(size_t)(off + n) * TW + off + k] = h;
+          lo[(size_t)(off + n) * TW + off + k] = bf16_bits((float)(v - (double)bf16_value(h)));
         }
       }
     }
@@ -191,8 +195,17 @@ extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int
     set_error("unknown kind %d", (int)kind);
     return PQ_ERR_INVALID_ARG;
   }
-  if (g != kGroup) { set_error("g=%d: only g=128 is supported", g); return PQ_ERR_UNSUPPORTED; }
-  if (D < g || D % g != 0) { set_error("D=%d must be a positive multiple of 128", D); return PQ_ERR_INVALID_ARG; }
+  // Group sizes: 128 everywhere; 64 for Givens and Hadamard; 256 for Hadamard (its uint8 pair
+  // slots and the 128 x 128 tensor-core tiles bound the Givens groups to 128 channels).
+  const bool g_ok = g == kGroup || (g == 64 && kind != PQ_SMOOTH_HADAMARD) || (g == 256 && kind == PQ_HADAMARD);
+  if (!g_ok) {
+    set_error("g=%d is not supported for this plan kind (Hadamard: 64, 128, 256; Givens: 64, 128; smoothing: 128)", g);
+    return PQ_ERR_UNSUPPORTED;
+  }
+  if (D < 128 || D % 128 != 0 || D % g != 0) {
+    set_error("D=%d must be a positive multiple of 128 and of g=%d", D, g);
+    return PQ_ERR_INVALID_ARG;
+  }
   if (flags & ~PQ_FLAG_SMOOTH_AFTER_ROTATE) { set_error("unknown flags 0x%x", flags); return PQ_ERR_INVALID_ARG; }
   if ((flags & PQ_FLAG_SMOOTH_AFTER_ROTATE) && kind != PQ_SMOOTH_HADAMARD) {
     set_error("PQ_FLAG_SMOOTH_AFTER_ROTATE needs PQ_SMOOTH_HADAMARD");
@@ -242,15 +255,25 @@ extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int
   pq_status st = cuda_fail(cudaGetDevice(&p->device), "cudaGetDevice");
   if (st == PQ_OK && kind == PQ_GIVENS) {
     std::vector<uint16_t> rot;
-    build_rotation_operands(G, K, pairs, angles, beta, rot);
+    build_rotation_operands(D, g, K, pairs, angles, beta, rot);
     st = upload(&p->d_rot, rot.data(), rot.size(), "givens tensor-core operands");
   }
   if (st == PQ_OK && kind == PQ_HADAMARD) {
-    // Unnormalised Sylvester H_128: entry (k, n) = (-1)^popcount(k & n) (Hadamard page §2.1),
-    // symmetric, so [n][k] = [k][n]; +-1 in bf16 is 0x3F80 / 0xBF80.
-    std::vector<uint16_t> h((size_t)g * g);
-    for (int k = 0; k < g; ++k)
-      for (int n = 0; n < g; ++n) h[(size_t)n * g + k] = (__builtin_popcount(k & n) & 1) ? 0xBF80 : 0x3F80;
+    // Unnormalised Sylvester H_b: entry (k, n) = (-1)^popcount(k & n) (Hadamard page §2.1),
+    // symmetric, so [n][k] = [k][n]; +-1 in bf16 is 0x3F80 / 0xBF80, 0 is 0.  g = 128: H_128;
+    // g = 64: diag(H_64, H_64) (zero where k and n lie in different halves); g = 256: H_128 then
+    // -H_128 (H_256 = [[H, H], [H, -H]] is applied as products with these two).
+    constexpr int TW = 128;
+    const int mats = g == 256 ? 2 : 1;
+    std::vector<uint16_t> h((size_t)mats * TW * TW);
+    for (int m = 0; m < mats; ++m)
+      for (int k = 0; k < TW; ++k)
+        for (int n = 0; n < TW; ++n) {
+          uint16_t v;
+          if (g == 64 && ((k ^ n) & 64)) v = 0;
+          else v = ((__builtin_popcount(k & n & (g == 64 ? 63 : 127)) + m) & 1) ? 0xBF80 : 0x3F80;
+          h[((size_t)m * TW + n) * TW + k] = v;
+        }
     st = upload(&p->d_rot, h.data(), h.size(), "hadamard tensor-core operand");
   }
   if (st == PQ_OK) st = upload<unsigned int>(&p->d_status, nullptr, 1, "status word");
@@ -382,9 +405,10 @@ pq_status check_gemm_args(const uint8_t* codes_A, const float* scales_A, const u
     set_error("all tensor pointers must be non-NULL");
     return PQ_ERR_INVALID_ARG;
   }
-  if (g != kGroup) { set_error("g=%d: only g=128 is supported", g); return PQ_ERR_UNSUPPORTED; }
+  if (g != 64 && g != 128 && g != 256) { set_error("g=%d: the GEMM supports g = 64, 128, 256", g); return PQ_ERR_UNSUPPORTED; }
   pq_status st = check_gemm_sizes(T, N, D);
   if (st != PQ_OK) return st;
+  if (D % g != 0) { set_error("D=%lld must be a multiple of g=%d", (long long)D, g); return PQ_ERR_INVALID_ARG; }
   if (out_dtype != PQ_OUT_F32 && out_dtype != PQ_OUT_BF16) { set_error("bad out_dtype"); return PQ_ERR_INVALID_ARG; }
   if (!aligned16(codes_A) || !aligned16(scales_A) || !aligned16(codes_W) ||
       !aligned16(scales_W) || !aligned16(Y)) {
@@ -403,7 +427,7 @@ extern "C" pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A,
   clear_error();
   pq_status st = check_gemm_args(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype);
   if (st != PQ_OK) return st;
-  return gemm_run(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype,
+  return gemm_run(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype,
                   reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -414,7 +438,7 @@ extern "C" pq_status pq_w4a4_gemm_noalloc(const uint8_t* codes_A, const float* s
   clear_error();
   pq_status st = check_gemm_args(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype);
   if (st != PQ_OK) return st;
-  return gemm_run_static_scratch(codes_A, scales_A, codes_W, scales_W, T, N, D, Y, out_dtype,
+  return gemm_run_static_scratch(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype,
                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -423,8 +447,8 @@ namespace {
 
 pq_status check_rrs_plan(const pq_plan* plan) {
   if (!plan) { set_error("plan is NULL"); return PQ_ERR_INVALID_ARG; }
-  if (plan->kind != PQ_HADAMARD) {
-    set_error("rotated runtime smoothing needs a PQ_HADAMARD plan");
+  if (plan->kind != PQ_HADAMARD || plan->g != kGroup) {
+    set_error("rotated runtime smoothing needs a PQ_HADAMARD plan with g = 128");
     return PQ_ERR_UNSUPPORTED;
   }
   if (plan->D > 16384 || rrs_rows_smem_bytes(plan->D) > 232448) {
@@ -503,21 +527,28 @@ extern "C" pq_status pq_rrs_gemm(const uint8_t* codes_A, const float* token_scal
   clear_error();
   pq_status st = check_gemm_args(codes_A, token_scales, codes_W, scales_W, T, N, D, g, Y, out_dtype);
   if (st != PQ_OK) return st;
-  return gemm_run(codes_A, token_scales, codes_W, scales_W, T, N, D, Y, out_dtype,
+  if (g != kGroup) { set_error("g=%d: rotated runtime smoothing uses g = 128", g); return PQ_ERR_UNSUPPORTED; }
+  return gemm_run(codes_A, token_scales, codes_W, scales_W, T, N, D, g, Y, out_dtype,
                   reinterpret_cast<cudaStream_t>(stream), /*row_scale=*/true);
 }
 
-extern "C" pq_status pq_w4a4_gemm_launch_count(int64_t T, int64_t N, int64_t D, int* launches) {
+extern "C" pq_status pq_w4a4_gemm_launch_count_g(int64_t T, int64_t N, int64_t D, int g, int* launches) {
   clear_error();
   if (!launches) {
     set_error("launches must be non-NULL");
     return PQ_ERR_INVALID_ARG;
   }
+  if (g != 64 && g != 128 && g != 256) { set_error("g=%d: the GEMM supports g = 64, 128, 256", g); return PQ_ERR_UNSUPPORTED; }
   pq_status st = check_gemm_sizes(T, N, D);
   if (st != PQ_OK) return st;
-  const int split = gemm_ksplit(T, N, D, nullptr) > 1 ? 1 : 0;
+  if (D % g != 0) { set_error("D=%lld must be a multiple of g=%d", (long long)D, g); return PQ_ERR_INVALID_ARG; }
+  const int split = gemm_ksplit(T, N, D, g, nullptr) > 1 ? 1 : 0;
   *launches = (T <= kGemmSmallT ? 1 : 2) + split;
   return PQ_OK;
+}
+
+extern "C" pq_status pq_w4a4_gemm_launch_count(int64_t T, int64_t N, int64_t D, int* launches) {
+  return pq_w4a4_gemm_launch_count_g(T, N, D, kGroup, launches);
 }
 
 extern "C" pq_status pq_selftest_wait_timeout(uint64_t limit_ns, void* stream) {

@@ -11,6 +11,13 @@
 // Block Hadamard (Hadamard page §2.1/§6.1): R = H_128 unnormalised (+-1, exact in bf16, one
 // term, the same for every group); the 1/sqrt(128) is folded into the stored scale.
 //
+// Group sizes (ParoQuant page §4.1: g = 64 for layers with many outliers; §6: g = 256 on
+// mobile parts).  A tile always spans 128 channels for g <= 128: g = 64 puts two groups' matrices
+// on the diagonal of the tile's 128 x 128 matrix and takes two maxima per row.  g = 256 (block
+// Hadamard only) spans 256 channels: H_256 = [[H, H], [H, -H]] with H = H_128, so each output
+// half is two accumulating K = 128 products against +H or -H (both resident), into a 256-column
+// accumulator; the row's maximum is taken over both halves before it is quantised.
+//
 // One kernel per call, persistent, one CTA per SM.  Tiles are (128 rows, one group); each CTA
 // takes a contiguous range of tiles in group-major order so the group's matrix stays resident.
 //   warp 0      TMA producer: the X tile (128 rows x 128 channels bf16, two 128-byte swizzled
@@ -35,16 +42,25 @@ namespace {
 constexpr int RT_M = 128;                 // rows per tile (MMA M, TMEM lanes)
 constexpr int RT_N = 128;                 // output channels (MMA N)
 constexpr int RT_KB = 64;                 // bf16 per 128-byte swizzle row (one K-block)
-constexpr int RT_STAGES = 4;
+constexpr int RT_STAGES = 4;              // X stages of two K-blocks (g <= 128)
 constexpr int RT_THREADS = 320;           // warps 0-1 control, 2-5 and 6-9 two epilogue warpgroups
-constexpr uint32_t RT_TMEM_COLS = 256;    // two accumulator buffers of 128 columns
 constexpr uint64_t kRtWaitNs = 2000000000ull;
-constexpr uint32_t kTileBytes = RT_M * 128 * 2;        // one X tile: 32 KB
+constexpr uint32_t kKBlockBytes = RT_M * 128;          // one K-block of an X tile: 16 KB
 constexpr uint32_t kRotBytes = 2 * RT_N * 128 * 2;     // two terms of one matrix: 64 KB
+
+// Per group size: channels per tile, K-blocks per X stage, X stages, accumulator columns.
+template <int GW> struct RtGeom {
+  static constexpr int TW = GW > 128 ? GW : 128;
+  static constexpr int KBS = TW / RT_KB;
+  static constexpr int STAGES = RT_STAGES * 2 / KBS;
+  static constexpr uint32_t BUF = (uint32_t)TW;               // TMEM columns per accumulator buffer
+  static constexpr uint32_t TMEM_COLS = 2 * BUF;
+  static constexpr uint32_t TILE_BYTES = (uint32_t)KBS * kKBlockBytes;
+};
 constexpr float kRoundMagicR = 12582912.0f;            // 1.5 * 2^23
 
 struct __align__(1024) RotSmem {
-  uint8_t x[RT_STAGES][2][RT_M * 128];    // [stage][K-block][128 rows x 128 bytes]
+  uint8_t x[RT_STAGES * 2][RT_M * 128];   // [stage * K-blocks per stage + K-block][128 rows x 128 bytes]
   uint8_t r[2][2][RT_N * 128];            // [term hi/lo][K-block][128 out channels x 128 bytes]
   uint64_t x_full[RT_STAGES];
   uint64_t x_empty[RT_STAGES];
@@ -102,11 +118,16 @@ __device__ __forceinline__ uint32_t rt_pack8(const float* v, float inv) {
 // its maximum over the tile's 128 rows in registers; the result (times scale_mult) is merged
 // into chan_max[channel] with an unsigned atomic maximum on the float's bits (all values are
 // non-negative, for which the bit order is the numeric order).  Rows past the end read as zeros.
-template <bool kColMax>
+// GW: the group size (64, 128 or 256); G counts groups of GW channels; a tile spans
+// RtGeom<GW>::TW channels (one group for 128 and 256, two for 64).
+template <bool kColMax, int GW>
 __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
     const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmR, int64_t rows, int G,
     int row_blocks, int64_t num_tiles, int terms, int r_groups, float scale_mult, uint8_t* __restrict__ codes,
     float* __restrict__ scales, unsigned int* __restrict__ chan_max, unsigned int* status) {
+  static_assert(!kColMax || GW == 128, "column maxima are taken on 128-channel groups");
+  using Geo = RtGeom<GW>;
+  constexpr int KBS = Geo::KBS, STAGES = Geo::STAGES;
   extern __shared__ unsigned char smem_raw[];
   RotSmem& S = *reinterpret_cast<RotSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -115,7 +136,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
   const int64_t end = num_tiles * (blockIdx.x + 1) / gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < RT_STAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(&S.x_full[s], 1);
       ptx::mbar_init(&S.x_empty[s], 1);
     }
@@ -134,7 +155,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
     ptx::prefetch_tmap(&tmR);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(&S.tmem_slot, RT_TMEM_COLS);
+    ptx::tmem_alloc(&S.tmem_slot, Geo::TMEM_COLS);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -162,16 +183,16 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
           cur_r = ri;
           ++loaded;
         }
-        const int s = step % RT_STAGES;
-        const uint32_t ph = (uint32_t)(step / RT_STAGES) & 1u;
+        const int s = step % STAGES;
+        const uint32_t ph = (uint32_t)(step / STAGES) & 1u;
         if (!rt_wait(S, &S.x_empty[s], ph ^ 1u, status)) { ok = false; break; }
-        ptx::mbar_arrive_expect_tx(&S.x_full[s], kTileBytes);
-        for (int kb = 0; kb < 2; ++kb)
-          ptx::tma_load_2d(S.x[s][kb], &tmX, &S.x_full[s], gi * 128 + kb * RT_KB, (int)r0);
+        ptx::mbar_arrive_expect_tx(&S.x_full[s], Geo::TILE_BYTES);
+        for (int kb = 0; kb < KBS; ++kb)
+          ptx::tma_load_2d(S.x[s * KBS + kb], &tmX, &S.x_full[s], gi * Geo::TW + kb * RT_KB, (int)r0);
       }
       // Drain: every load issued lands before the CTA may exit.
-      for (int j = (step > RT_STAGES ? step - RT_STAGES : 0); j < step; ++j)
-        rt_drain(&S.x_full[j % RT_STAGES], (uint32_t)(j / RT_STAGES) & 1u);
+      for (int j = (step > STAGES ? step - STAGES : 0); j < step; ++j)
+        rt_drain(&S.x_full[j % STAGES], (uint32_t)(j / STAGES) & 1u);
       if (loaded > 0) rt_drain(&S.r_full, (uint32_t)(loaded - 1) & 1u);
     }
   } else if (warp == 1) {
@@ -189,27 +210,46 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
           cur_r = ri;
           ++used;
         }
-        const int s = step % RT_STAGES;
-        const uint32_t ph = (uint32_t)(step / RT_STAGES) & 1u;
+        const int s = step % STAGES;
+        const uint32_t ph = (uint32_t)(step / STAGES) & 1u;
         const int b = step & 1;
         const uint32_t u = (uint32_t)(step >> 1);
         if (!rt_wait(S, &S.acc_empty[b], (u & 1u) ^ 1u, status)) { ok = false; break; }
         if (!rt_wait(S, &S.x_full[s], ph, status)) { ok = false; break; }
         ptx::tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)b * RT_N;
-        int n = 0;
-        for (int term = 0; term < terms; ++term)
+        const uint32_t d = tmem + (uint32_t)b * Geo::BUF;
+        if constexpr (GW == 256) {
+          // Output half o = sum over input halves i of X_i (+-H): -H only for (i, o) = (1, 1).
 #pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {
-            const uint32_t a0 = ptx::smem_addr(S.x[s][kb]);
-            const uint32_t b0 = ptx::smem_addr(S.r[term][kb]);
+          for (int o = 0; o < 2; ++o) {
+            int n = 0;
 #pragma unroll
-            for (int k = 0; k < 4; ++k, ++n) {   // K16 per MMA = 32 bytes along the swizzled row
-              const uint64_t da = ptx::smem_desc_sw128(a0 + 32 * k), db = ptx::smem_desc_sw128(b0 + 32 * k);
-              if (kColMax) ptx::umma_f16(d, db, da, kIdescBf16, n > 0 ? 1u : 0u);   // D = R^T X^T
-              else ptx::umma_f16(d, da, db, kIdescBf16, n > 0 ? 1u : 0u);           // D = X R
-            }
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+              for (int kb = 0; kb < 2; ++kb) {
+                const uint32_t a0 = ptx::smem_addr(S.x[s * KBS + 2 * i + kb]);
+                const uint32_t b0 = ptx::smem_addr(S.r[o & i][kb]);
+#pragma unroll
+                for (int k = 0; k < 4; ++k, ++n)
+                  ptx::umma_f16(d + (uint32_t)(o * RT_N), ptx::smem_desc_sw128(a0 + 32 * k),
+                                ptx::smem_desc_sw128(b0 + 32 * k), kIdescBf16, n > 0 ? 1u : 0u);
+              }
           }
+        } else {
+          int n = 0;
+          for (int term = 0; term < terms; ++term)
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb) {
+              const uint32_t a0 = ptx::smem_addr(S.x[s * KBS + kb]);
+              const uint32_t b0 = ptx::smem_addr(S.r[term][kb]);
+#pragma unroll
+              for (int k = 0; k < 4; ++k, ++n) {   // K16 per MMA = 32 bytes along the swizzled row
+                const uint64_t da = ptx::smem_desc_sw128(a0 + 32 * k), db = ptx::smem_desc_sw128(b0 + 32 * k);
+                if (kColMax) ptx::umma_f16(d, db, da, kIdescBf16, n > 0 ? 1u : 0u);   // D = R^T X^T
+                else ptx::umma_f16(d, da, db, kIdescBf16, n > 0 ? 1u : 0u);           // D = X R
+              }
+            }
+        }
         ptx::umma_commit(&S.x_empty[s]);
         ptx::umma_commit(&S.acc_full[b]);
       }
@@ -230,7 +270,37 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
       const uint32_t u = (uint32_t)(step >> 1);
       if (!rt_warp_wait(S, &S.acc_full[b], u & 1u, status)) break;
       ptx::tc_fence_after();
-      const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)b * RT_N;
+      const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)b * Geo::BUF;
+      if constexpr (GW == 256) {
+        // The row's 256 values: the maximum over both halves first, then a second read of the
+        // accumulator to quantise (tcgen05.ld is warp-collective: every lane takes part).
+        float m = 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(ta + 32 * c, r);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(__uint_as_float(r[j])));
+        }
+        const float inv = m > 0.0f ? 7.0f * __frcp_rn(m) : 0.0f;
+        uint4* dst = reinterpret_cast<uint4*>(codes + t * (int64_t)G * 128 + gi * 128);
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(ta + 32 * c, r);
+          ptx::tmem_ld_wait();
+          float y[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(r[j]);
+          if (t < rows) dst[c] = make_uint4(rt_pack8(y, inv), rt_pack8(y + 8, inv), rt_pack8(y + 16, inv),
+                                            rt_pack8(y + 24, inv));
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&S.acc_empty[b]);
+        if (t < rows) scales[t * G + gi] = m * scale_mult;
+      } else {
       float y[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -251,6 +321,24 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
         atomicMax(chan_max + (int64_t)gi * 128 + rl, __float_as_uint(m * scale_mult));
         continue;
       }
+      if constexpr (GW == 64) {
+        // two groups per tile: channels 0..63 and 64..127 of the row, one maximum each
+        float mh[2] = {0.0f, 0.0f};
+#pragma unroll
+        for (int i = 0; i < 128; ++i) mh[i >> 6] = fmaxf(mh[i >> 6], fabsf(y[i]));
+        if (t < rows) {
+          uint4* dst = reinterpret_cast<uint4*>(codes + t * (int64_t)G * 32 + gi * 64);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float inv = mh[k >> 1] > 0.0f ? 7.0f * __frcp_rn(mh[k >> 1]) : 0.0f;
+            dst[k] = make_uint4(rt_pack8(y + 32 * k, inv), rt_pack8(y + 32 * k + 8, inv),
+                                rt_pack8(y + 32 * k + 16, inv), rt_pack8(y + 32 * k + 24, inv));
+          }
+          scales[t * G + 2 * gi] = mh[0] * scale_mult;
+          scales[t * G + 2 * gi + 1] = mh[1] * scale_mult;
+        }
+        continue;
+      }
       const float inv = m > 0.0f ? 7.0f * __frcp_rn(m) : 0.0f;
       if (t < rows) {
         uint4* dst = reinterpret_cast<uint4*>(codes + t * (int64_t)G * 64 + gi * 64);
@@ -260,6 +348,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
                               rt_pack8(y + 32 * k + 16, inv), rt_pack8(y + 32 * k + 24, inv));
         scales[t * G + gi] = m * scale_mult;
       }
+      }   // GW <= 128
     }
   }
 
@@ -268,7 +357,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, RT_TMEM_COLS);
+    ptx::tmem_dealloc(tmem, Geo::TMEM_COLS);
   }
 }
 
@@ -341,42 +430,69 @@ cudaError_t make_bf16_row_lines_map(CUtensorMap* map, const void* base, int64_t 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+namespace {
+
+template <int GW>
+cudaError_t launch_rotate_mma_g(const pq_plan* plan, const CUtensorMap& tmX, const CUtensorMap& tmR, int64_t rows,
+                                int terms, int r_groups, float scale_mult, uint8_t* codes, float* scales,
+                                cudaStream_t stream) {
+  const int row_blocks = (int)((rows + RT_M - 1) / RT_M);
+  const int64_t tiles = (int64_t)row_blocks * (plan->D / RtGeom<GW>::TW);
+  const int sms = device_sm_count();
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  static std::atomic<bool> attr_done[kMaxDevices];
+  cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(rotate_mma_kernel<false, GW>), (int)kRotSmemBytes,
+                                        attr_done);
+  if (e != cudaSuccess) return e;
+  rotate_mma_kernel<false, GW><<<grid, RT_THREADS, kRotSmemBytes, stream>>>(
+      tmX, tmR, rows, plan->G, row_blocks, tiles, terms, r_groups, scale_mult, codes, scales, nullptr, plan->d_status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
                               uint8_t* codes, float* scales, cudaStream_t stream, unsigned int* chan_max) {
   if (rows <= 0) return cudaSuccess;
   const bool givens = plan->kind == PQ_GIVENS;
-  const int terms = givens ? 2 : 1;
-  const int r_groups = givens ? plan->G : 1;
+  const int g = plan->g;
+  // Operand matrices: Givens, one per 128-channel tile (two groups' matrices on the diagonal at
+  // g = 64), two bf16 terms; Hadamard, one exact term (H_128, or diag(H_64, H_64)), or at
+  // g = 256 the two matrices +H_128 and -H_128.
+  const int terms = givens || g == 256 ? 2 : 1;
+  const int r_groups = givens ? plan->D / 128 : 1;
   CUtensorMap tmX, tmR;
   cudaError_t e = make_bf16_tile_map(&tmX, X, rows, plan->D, ldx);
   if (e != cudaSuccess) return e;
   const uint16_t* R = plan->d_rot + (size_t)(weights && givens ? 1 : 0) * r_groups * terms * RT_N * 128;
   e = make_bf16_tile_map(&tmR, R, (int64_t)r_groups * terms * RT_N, 128, 128);
   if (e != cudaSuccess) return e;
-  const int row_blocks = (int)((rows + RT_M - 1) / RT_M);
-  const int64_t tiles = (int64_t)row_blocks * plan->G;
-  const int sms = device_sm_count();
-  const int grid = (int)(tiles < sms ? tiles : sms);
-  // Givens: scale = m / 7.  Hadamard: R = H unnormalised, so y is sqrt(128) times the
-  // orthonormal rotation and scale = m / (7 sqrt(128)).
-  const float scale_mult = givens ? (1.0f / 7.0f) : 0.012626906806902634f;
   if (chan_max) {
     // column maxima of the normalised rotation: max |x R| (Hadamard: R unnormalised, so / sqrt(128))
+    const int row_blocks = (int)((rows + RT_M - 1) / RT_M);
+    const int64_t tiles = (int64_t)row_blocks * plan->G;
+    const int sms = device_sm_count();
+    const int grid = (int)(tiles < sms ? tiles : sms);
     static std::atomic<bool> attr_cm[kMaxDevices];
-    e = set_kernel_attributes(reinterpret_cast<const void*>(rotate_mma_kernel<true>), (int)kRotSmemBytes, attr_cm);
+    e = set_kernel_attributes(reinterpret_cast<const void*>(rotate_mma_kernel<true, 128>), (int)kRotSmemBytes, attr_cm);
     if (e != cudaSuccess) return e;
-    rotate_mma_kernel<true><<<grid, RT_THREADS, kRotSmemBytes, stream>>>(
+    rotate_mma_kernel<true, 128><<<grid, RT_THREADS, kRotSmemBytes, stream>>>(
         tmX, tmR, rows, plan->G, row_blocks, tiles, terms, r_groups, givens ? 1.0f : 0.088388347648318440550f,
         nullptr, nullptr, chan_max, plan->d_status);
     return cudaGetLastError();
   }
-  static std::atomic<bool> attr_done[kMaxDevices];
-  e = set_kernel_attributes(reinterpret_cast<const void*>(rotate_mma_kernel<false>), (int)kRotSmemBytes, attr_done);
-  if (e != cudaSuccess) return e;
-  rotate_mma_kernel<false><<<grid, RT_THREADS, kRotSmemBytes, stream>>>(tmX, tmR, rows, plan->G, row_blocks, tiles,
-                                                                       terms, r_groups, scale_mult, codes, scales,
-                                                                       nullptr, plan->d_status);
-  return cudaGetLastError();
+  // Givens: scale = m / 7.  Hadamard: R = H unnormalised, so y is sqrt(g) times the orthonormal
+  // rotation and scale = m / (7 sqrt(g)).
+  switch (g) {
+    case 64:
+      return launch_rotate_mma_g<64>(plan, tmX, tmR, rows, terms, r_groups, givens ? (1.0f / 7.0f) : (1.0f / 56.0f),
+                                     codes, scales, stream);
+    case 256:
+      return launch_rotate_mma_g<256>(plan, tmX, tmR, rows, terms, r_groups, 1.0f / 112.0f, codes, scales, stream);
+    default:
+      return launch_rotate_mma_g<128>(plan, tmX, tmR, rows, terms, r_groups,
+                                      givens ? (1.0f / 7.0f) : 0.012626906806902634f, codes, scales, stream);
+  }
 }
 
 }  // namespace pq

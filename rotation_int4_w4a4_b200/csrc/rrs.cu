@@ -39,18 +39,33 @@ constexpr int RK_K = 2048;   // other channels per rank block
 
 __global__ void __launch_bounds__(RK_J) rrs_rank_kernel(const unsigned int* __restrict__ chan_max, int D,
                                                        int* __restrict__ inv_perm) {
-  __shared__ unsigned int mk[RK_K];
+  __shared__ __align__(16) unsigned int mk[RK_K];
   const int j = blockIdx.x * RK_J + threadIdx.x;
   const int k0 = blockIdx.y * RK_K;
-  const int nk = min(RK_K, D - k0);
+  const int nk = min(RK_K, D - k0);   // a multiple of 128 (D is)
   for (int i = threadIdx.x; i < nk; i += RK_J) mk[i] = chan_max[k0 + i];
   __syncthreads();
   if (j >= D) return;
   const unsigned int mj = chan_max[j];   // float bits of a non-negative value: bit order = numeric order
+  const uint4* m4 = reinterpret_cast<const uint4*>(mk);
   int cnt = 0;
-  for (int i = 0; i < nk; ++i) {
-    const unsigned int m = mk[i];
-    cnt += (m > mj || (m == mj && k0 + i < j)) ? 1 : 0;
+  if (k0 + nk <= j) {
+    // every channel of the block precedes j: it ranks first when its maximum is at least m_j
+    for (int i = 0; i < nk / 4; ++i) {
+      const uint4 v = m4[i];
+      cnt += (v.x >= mj) + (v.y >= mj) + (v.z >= mj) + (v.w >= mj);
+    }
+  } else if (k0 > j) {
+    // every channel of the block follows j: it ranks first only with a larger maximum
+    for (int i = 0; i < nk / 4; ++i) {
+      const uint4 v = m4[i];
+      cnt += (v.x > mj) + (v.y > mj) + (v.z > mj) + (v.w > mj);
+    }
+  } else {
+    for (int i = 0; i < nk; ++i) {
+      const unsigned int m = mk[i];
+      cnt += (m > mj || (m == mj && k0 + i < j)) ? 1 : 0;
+    }
   }
   if (cnt) atomicAdd(inv_perm + j, cnt);
 }

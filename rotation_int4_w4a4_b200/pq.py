@@ -27,6 +27,7 @@ KINDS = {"hadamard": PQ_HADAMARD, "givens": PQ_GIVENS, "smooth_hadamard": PQ_SMO
 # Every symbol the header declares.
 EXPORTS = ("pq_select_pairs", "pq_make_plan", "pq_destroy_plan", "pq_transform_quant",
            "pq_pack_weights", "pq_w4a4_gemm", "pq_w4a4_gemm_noalloc", "pq_w4a4_gemm_launch_count",
+           "pq_w4a4_gemm_launch_count_g",
            "pq_rrs_prepare", "pq_rrs_transform_quant", "pq_rrs_pack_weights", "pq_rrs_gemm",
            "pq_check_status",
            "pq_selftest_wait_timeout", "pq_status_string", "pq_last_error")
@@ -49,6 +50,8 @@ lib.pq_w4a4_gemm_noalloc.argtypes = lib.pq_w4a4_gemm.argtypes
 lib.pq_w4a4_gemm_noalloc.restype = _i32
 lib.pq_w4a4_gemm_launch_count.argtypes = [_i64, _i64, _i64, _c.POINTER(_i32)]
 lib.pq_w4a4_gemm_launch_count.restype = _i32
+lib.pq_w4a4_gemm_launch_count_g.argtypes = [_i64, _i64, _i64, _i32, _c.POINTER(_i32)]
+lib.pq_w4a4_gemm_launch_count_g.restype = _i32
 lib.pq_rrs_prepare.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]
 lib.pq_rrs_prepare.restype = _i32
 lib.pq_rrs_transform_quant.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]
@@ -292,6 +295,13 @@ def pq_rrs_gemm(codes_A, token_scales, codes_W, scales_W, Y, T=None, N=None, D=N
     T, N, D, out_dtype, ptrs = _gemm_args(codes_A, token_scales, codes_W, scales_W, Y, T, N, D, g, out_dtype,
                                           sa_per_token=True)
     _check(lib.pq_rrs_gemm(*ptrs[:4], T, N, D, g, ptrs[4], out_dtype, _stream(stream)), "pq_rrs_gemm")
+
+
+def pq_w4a4_gemm_launch_count_g(T: int, N: int, D: int, g: int) -> int:
+    """Kernels one pq_w4a4_gemm call of these sizes and group size launches on the current device."""
+    n = _i32(0)
+    _check(lib.pq_w4a4_gemm_launch_count_g(T, N, D, g, _c.byref(n)), "pq_w4a4_gemm_launch_count_g")
+    return n.value
 
 
 def pq_w4a4_gemm_launch_count(T: int, N: int, D: int) -> int:

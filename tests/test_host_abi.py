@@ -39,6 +39,13 @@ def test_select_pairs_matches_oracle(pq, seed, K, N):
     assert np.array_equal(a, b)
 
 
+@pytest.mark.parametrize("seed,K,N", [(3, 4, 32), (11, 8, 20)])
+def test_select_pairs_g64_matches_oracle(pq, seed, K, N):
+    a = pq.pq_select_pairs(seed, 384, 64, K, N)
+    b = oracle.select_pairs(seed, 384, 64, K, N)
+    assert np.array_equal(a, b)
+
+
 def test_status_strings(pq):
     assert pq.lib.pq_status_string(0) == b"PQ_OK"
     assert pq.lib.pq_status_string(5) == b"PQ_ERR_TIMEOUT"
@@ -47,7 +54,8 @@ def test_status_strings(pq):
 
 def test_select_pairs_rejects_bad_arguments(pq):
     out = np.empty(4096, dtype=np.uint8)
-    assert pq.lib.pq_select_pairs(0, 256, 64, 4, 16, out.ctypes.data) == pq.PQ_ERR_UNSUPPORTED
+    assert pq.lib.pq_select_pairs(0, 256, 32, 4, 16, out.ctypes.data) == pq.PQ_ERR_UNSUPPORTED
+    assert pq.lib.pq_select_pairs(0, 512, 256, 4, 16, out.ctypes.data) == pq.PQ_ERR_UNSUPPORTED
     assert pq.lib.pq_select_pairs(0, 200, 128, 4, 16, out.ctypes.data) == pq.PQ_ERR_INVALID_ARG
     assert pq.lib.pq_select_pairs(0, 256, 128, 0, 16, out.ctypes.data) == pq.PQ_ERR_INVALID_ARG
     assert pq.lib.pq_select_pairs(0, 256, 128, 4, 65, out.ctypes.data) == pq.PQ_ERR_INVALID_ARG
@@ -59,9 +67,15 @@ def test_make_plan_validation_before_any_device_call(pq):
     with pytest.raises(pq.PQError) as e:
         pq.Plan("hadamard", 100)
     assert e.value.status == pq.PQ_ERR_INVALID_ARG
+    # group sizes: 64/128/256 for Hadamard, 64/128 for Givens, 128 for smoothing
+    for kind, D, g in (("hadamard", 256, 32), ("givens", 512, 256), ("smooth_hadamard", 256, 64),
+                       ("smooth_hadamard", 512, 256)):
+        with pytest.raises(pq.PQError) as e:
+            pq.Plan(kind, D, g=g, K=2)
+        assert e.value.status == pq.PQ_ERR_UNSUPPORTED, (kind, g)
     with pytest.raises(pq.PQError) as e:
-        pq.Plan("hadamard", 256, g=64)
-    assert e.value.status == pq.PQ_ERR_UNSUPPORTED
+        pq.Plan("hadamard", 384, g=256)                   # D not a multiple of g
+    assert e.value.status == pq.PQ_ERR_INVALID_ARG
     with pytest.raises(pq.PQError) as e:
         pq.Plan("hadamard", 256, flags=pq.PQ_FLAG_SMOOTH_AFTER_ROTATE)
     assert e.value.status == pq.PQ_ERR_INVALID_ARG
@@ -85,7 +99,9 @@ def test_gemm_and_transform_validation(pq):
     L = pq.lib
     p = 16  # any aligned non-null fake address: validation fails before use
     assert L.pq_w4a4_gemm(None, p, p, p, 4, 16, 128, 128, p, 0, None) == pq.PQ_ERR_INVALID_ARG
-    assert L.pq_w4a4_gemm(p, p, p, p, 4, 16, 128, 64, p, 0, None) == pq.PQ_ERR_UNSUPPORTED
+    assert L.pq_w4a4_gemm(p, p, p, p, 4, 16, 128, 32, p, 0, None) == pq.PQ_ERR_UNSUPPORTED
+    assert L.pq_w4a4_gemm(p, p, p, p, 4, 16, 384, 256, p, 0, None) == pq.PQ_ERR_INVALID_ARG   # D % g
+    assert L.pq_rrs_gemm(p, p, p, p, 4, 16, 128, 32, p, 0, None) == pq.PQ_ERR_UNSUPPORTED
     assert L.pq_w4a4_gemm(p, p, p, p, 4, 24, 128, 128, p, 0, None) == pq.PQ_ERR_INVALID_ARG
     assert L.pq_w4a4_gemm(p, p, p, p, 4, 16, 200, 128, p, 0, None) == pq.PQ_ERR_INVALID_ARG
     assert L.pq_w4a4_gemm(p, p, p, p, 0, 16, 128, 128, p, 0, None) == pq.PQ_ERR_INVALID_ARG
