@@ -639,6 +639,52 @@ def measure_rrs(args, dev, stream, peaks, peak_src):
                                                                  f"burst x {INT8_OVER_BF16}"}
 
 
+def measure_decode(args, dev, stream, peaks, peak_src):
+    """Decode-sized linear layers (T <= 64 tokens, D = 4096, block Hadamard, weights packed once
+    beforehand): the activation transform and the GEMM as two calls, and as one pq_w4a4_linear
+    call (the GEMM is the transform's programmatic dependent).  L2 flushed before each step.
+    Bytes: X in, Y out, packed weights and their scales in."""
+    import torch
+
+    from rotation_int4_w4a4_b200 import inputs, pq
+    flush = L2Flush(dev)
+    out = {}
+    for N in (4096, 14336):
+        for T in (1, 16, 64):
+            wl = inputs.workload("sweep", T=T, N=N)
+            D, G = wl.D, wl.D // wl.g
+            plan = pq.Plan("hadamard", D)
+            X, W = dev_bf16(wl.X, dev), dev_bf16(wl.W, dev)
+            cw = torch.empty((N, D // 2), dtype=torch.uint8, device=dev)
+            sw = torch.empty((N, G), dtype=torch.float32, device=dev)
+            pq.pq_pack_weights(plan, W, cw, sw, stream=stream)
+            ca = torch.empty((T, D // 2), dtype=torch.uint8, device=dev)
+            sa = torch.empty((T, G), dtype=torch.float32, device=dev)
+            Y = torch.empty((T, N), dtype=torch.float32, device=dev)
+            two = (lambda: pq.pq_transform_quant(plan, X, ca, sa, stream=stream),
+                   lambda: pq.pq_w4a4_gemm(ca, sa, cw, sw, Y, stream=stream))
+            one = (lambda: pq.pq_w4a4_linear(plan, X, ca, sa, cw, sw, Y, stream=stream),)
+            steps = max(5, min(args.steps, 10))
+            res = {}
+            for name, calls in (("separate", two), ("linear", one)):
+                time_calls(lambda k: calls, flush, max(3, args.warmup), stream)
+                per = time_calls(lambda k: calls, flush, steps, stream)
+                res[name] = 1e3 * statistics.mean(sum(p) for p in per)
+            pq.pq_check_status(plan)
+            nbytes = T * D * 2 + T * N * 4 + N * D / 2 + N * G * 4
+            out[f"T{T}_N{N}"] = {
+                "us_separate": res["separate"], "us_linear": res["linear"],
+                "bytes": nbytes, "GB_s_linear": nbytes / (res["linear"] * 1e-6) / 1e9,
+                "frac_hbm_linear": nbytes / (res["linear"] * 1e-6) / 1e9 / peaks["hbm_gbs"]}
+            plan.close()
+            del X, W, cw, sw, ca, sa, Y
+    del flush
+    torch.cuda.empty_cache()
+    out["note"] = (f"D=4096, block Hadamard, g=128, weights packed beforehand; {peak_src} copy bandwidth; "
+                   "bytes = X + Y + packed W + W scales per call")
+    return out
+
+
 def run_ours(args, wl, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -706,6 +752,7 @@ def run_ours(args, wl, rank, world, local_rank):
         for g in (64, 256):
             also[f"q_proj_g{g}"] = measure_also("q_proj", args, dev, stream, peaks, peak_src, g=g)
         also["rrs_down_proj"] = measure_rrs(args, dev, stream, peaks, peak_src)
+        also["decode"] = measure_decode(args, dev, stream, peaks, peak_src)
     if rank != 0:
         return
     comps = components(wl, per, peaks)

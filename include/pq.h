@@ -191,6 +191,25 @@ pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A, const uint
                        pq_out_dtype out_dtype, void* stream);
 
 /*
+ * pq_w4a4_linear — the activation transform and the GEMM in one call (ParoQuant page §3.2:
+ * rotation, scaling and quantisation fused with the matrix multiply to save memory round trips;
+ * §6, memory tips: transform first, then quantise):
+ *   pq_transform_quant(plan, X, T, ldx, codes_A, scales_A, NULL) followed by
+ *   pq_w4a4_gemm(codes_A, scales_A, codes_W, scales_W, T, N, plan->D, plan->g, Y, out_dtype).
+ *   T <= 128: the GEMM is launched as a programmatic dependent of the transform: its prologue
+ *   and its weight-side loads start while the transform runs, and it reads codes_A and scales_A
+ *   only after the transform has completed.  T > 128: the two run one after the other.
+ *   codes_A [T][D/2] and scales_A [T][D/g] are caller-owned device buffers and are written (the
+ *   activation codes stay available).  codes_W and scales_W must be complete when the call is
+ *   made (written by work enqueued on `stream` before it, or earlier); Y must not overlap X,
+ *   codes_A or scales_A.  Arguments as for the two calls (smoothing plans: no smooth_out).
+ *   Launches: the transform's plus pq_w4a4_gemm_launch_count_g(T, N, D, g).
+ */
+pq_status pq_w4a4_linear(const pq_plan* plan, const void* X, int64_t T, int64_t ldx, uint8_t* codes_A,
+                         float* scales_A, const uint8_t* codes_W, const float* scales_W, int64_t N, void* Y,
+                         pq_out_dtype out_dtype, void* stream);
+
+/*
  * Rotated runtime smoothing with channel reordering: the RRS page's main equation (X_rot = X R,
  * s_j = max |(X_rot)_j|, Quantize(X_rot diag(s)^-1), Y = sum_j (X'_q)_j (W'_q)_j^T s_j) carried
  * out as in its Fig. 4: (1) the channels are reordered by their maxima, (2) the reordered

@@ -198,7 +198,6 @@ __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, 
 struct Work {
   int m_tiles, n_tiles, num_tiles;
   int ksplit, gs, G;
-  int gsl;               // K32 slices per group (g / 32): 2, 4 or 8; a K-block holds 4
   int units;
   int first, stride;     // this CTA pair's first unit and the number of pairs in the grid
   int rank;              // 0 = even CTA (issues the pair's MMAs), 1 = odd CTA
@@ -215,7 +214,7 @@ __device__ __forceinline__ void unit_coords(int u, const Work& wk, int& m0, int&
 // -------------------------------------------------------------------------- control
 // kRow: scales_W holds per-(row, group) factors and scales_A one scale per token (applied in the
 // epilogue after the groups), so the loaders fetch only the weight rows' factors.
-template <bool kRow>
+template <bool kRow, int GSL>
 __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA, const CUtensorMap& tmB,
                                             const float* __restrict__ scales_A, const float* __restrict__ scales_W,
                                             uint32_t tmem, int T, int N, int G, int scales_vec16, const Work& wk,
@@ -233,7 +232,7 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
         int m0, n0, kr, k0, k1;
         unit_coords(u, wk, m0, n0, kr, k0, k1);
         // the unit's K-blocks (its groups start on a K-block boundary: ranges are 4 groups)
-        const int kb0 = k0 * wk.gsl / 4, kb1 = k1 * wk.gsl / 4;
+        const int kb0 = k0 * GSL / 4, kb1 = k1 * GSL / 4;
         for (int kb = kb0; kb < kb1; ++kb, ++step) {
           const int s = step % OP_STAGES;
           const uint32_t ph = (uint32_t)(step / OP_STAGES) & 1u;
@@ -271,10 +270,14 @@ __device__ __forceinline__ void cta_control(GemmSmem& S, const CUtensorMap& tmA,
           if (!wait_or_abort(S, &S.acc_empty[b], (u & 1u) ^ 1u, status)) { ok = false; break; }
           ptx::tc_fence_after();
           const uint32_t d = tmem + (uint32_t)b * BN;
-          // The group's K32 slices (2, 4 or 8): a K-block's stage is awaited at its first slice
-          // and released after its fourth; slice 0 of the group overwrites the buffer.
-          for (int sl = 0; sl < wk.gsl; ++sl) {
-            const int sub = ((kg - k0) * wk.gsl + sl) & 3;
+          // The group's GSL K32 slices (compile-time, so the MMAs issue back to back): a K-block's
+          // stage is awaited at its first slice and released after its fourth; slice 0 of the
+          // group overwrites the buffer.  GSL = 2: the group is the first or second half of a
+          // K-block (by its parity within the unit).
+          const int h = GSL == 2 ? ((kg - k0) & 1) : 0;
+#pragma unroll
+          for (int sl = 0; sl < GSL; ++sl) {
+            const int sub = GSL == 2 ? 2 * h + sl : (sl & 3);
             const int s = kstep % OP_STAGES;
             if (sub == 0) {
               if (!wait_or_abort(S, &S.op_full[s], (uint32_t)(kstep / OP_STAGES) & 1u, status)) { ok = false; break; }
@@ -466,11 +469,12 @@ __device__ __forceinline__ void cta_epilogue(GemmSmem& S, uint32_t tmem, void* _
   }
 }
 
-template <bool kRow>
+// GSL: K32 tensor-core slices per group (g / 32 = 2, 4 or 8; a 128-code K-block holds 4).
+template <bool kRow, int GSL>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1) w4a4_gemm_kernel(
     const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
     const float* __restrict__ scales_A, const float* __restrict__ scales_W, void* __restrict__ Y,
-    int T, int N, int G, int gsl, int scales_vec16, int out_bf16, int m_tiles, int n_tiles, int ksplit, int gs,
+    int T, int N, int G, int scales_vec16, int out_bf16, int m_tiles, int n_tiles, int ksplit, int gs,
     float* __restrict__ ws, unsigned int* status) {
   extern __shared__ unsigned char smem_raw[];
   GemmSmem& S = *reinterpret_cast<GemmSmem*>(
@@ -483,7 +487,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1) w4a4
   wk.ksplit = ksplit;
   wk.gs = gs;
   wk.G = G;
-  wk.gsl = gsl;
   wk.units = wk.num_tiles * ksplit;
   wk.rank = (int)ptx::cluster_ctarank();
   wk.first = (int)(blockIdx.x >> 1);
@@ -522,7 +525,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1) w4a4
 
   if (warp < EPI_WARP0) {
     ptx::setmaxnreg_dec<REG_CTRL>();
-    cta_control<kRow>(S, tmA, tmB, scales_A, scales_W, tmem, T, N, G, scales_vec16, wk, status);
+    cta_control<kRow, GSL>(S, tmA, tmB, scales_A, scales_W, tmem, T, N, G, scales_vec16, wk, status);
   } else {
     ptx::setmaxnreg_inc<REG_EPI>();
     cta_epilogue<kRow>(S, tmem, Y, T, N, G, out_bf16, wk, ws, scales_A, status);
@@ -672,7 +675,7 @@ pq_status gemm_max_pairs(int sms, int* out) {
     attr.val.clusterDim.z = 1;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    e = cudaOccupancyMaxActiveClusters(&n, w4a4_gemm_kernel<false>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, w4a4_gemm_kernel<false, 4>, &cfg);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveClusters(gemm)");
     if (n < 1) {
       set_error("w4a4_gemm_kernel: no CTA pair fits on this device");
@@ -681,6 +684,31 @@ pq_status gemm_max_pairs(int sms, int* out) {
     if (slot) cache[dev].store(n, std::memory_order_relaxed);
   }
   *out = n;
+  return PQ_OK;
+}
+
+// Shared-memory attribute of one contraction instantiation, and the register guard: the warp
+// roles re-divide the launch's registers with setmaxnreg, which only works when the kernel was
+// compiled with exactly the budgeted count (otherwise an increase would never be granted).
+template <bool kRow, int GSL>
+pq_status pair_gemm_prepare() {
+  static std::atomic<bool> attr_done[kMaxDevices];
+  cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_kernel<kRow, GSL>), (int)kSmemBytes,
+                                        attr_done);
+  if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel attributes");
+  static std::atomic<int> num_regs_cache{-1};   // a property of the kernel binary
+  int num_regs = num_regs_cache.load(std::memory_order_relaxed);
+  if (num_regs < 0) {
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, w4a4_gemm_kernel<kRow, GSL>);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(gemm)");
+    num_regs = fa.numRegs;
+    num_regs_cache.store(num_regs, std::memory_order_relaxed);
+  }
+  if (num_regs != (int)REG_LAUNCH) {
+    set_error("w4a4_gemm_kernel compiled with %d registers per thread, %u expected", num_regs, REG_LAUNCH);
+    return PQ_ERR_CUDA;
+  }
   return PQ_OK;
 }
 
@@ -748,15 +776,15 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   const int64_t chunksA = T * (D / 32), chunksW = N * (D / 32);   // 16 packed bytes each
   const int64_t want = (chunksA + chunksW + 255) / 256;
   const int egrid = (int)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
-  static std::atomic<bool> attr_expand[kMaxDevices], attr_gemm[kMaxDevices], attr_gemm_row[kMaxDevices];
+  static std::atomic<bool> attr_expand[kMaxDevices];
   cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(expand_codes_kernel), 0, attr_expand);
   if (e != cudaSuccess) return cuda_fail(e, "expand_codes_kernel attributes");
-  e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_kernel<false>), (int)kSmemBytes, attr_gemm);
-  if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel attributes");
-  if (row_scale) {
-    e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_kernel<true>), (int)kSmemBytes, attr_gemm_row);
-    if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel attributes");
-  }
+  // The contraction's attributes are set before the expansion is launched, so that a failure
+  // leaves nothing enqueued.
+  st = g == 64 ? (row_scale ? pair_gemm_prepare<true, 2>() : pair_gemm_prepare<false, 2>())
+       : g == 256 ? (row_scale ? pair_gemm_prepare<true, 8>() : pair_gemm_prepare<false, 8>())
+                  : (row_scale ? pair_gemm_prepare<true, 4>() : pair_gemm_prepare<false, 4>());
+  if (st != PQ_OK) return st;
   expand_codes_kernel<<<egrid, 256, 0, stream>>>(codes_A, chunksA, codes_W, chunksW, A8, W8, g == 64 ? 1 : 0);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "expand_codes_kernel launch");
@@ -768,32 +796,21 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
   if (st != PQ_OK) return st;
   const int64_t pairs = max_pairs;
   const int grid = 2 * (int)(units < pairs ? units : pairs);
-  // The warp roles re-divide the launch's registers with setmaxnreg; that only works when the
-  // kernel was compiled with exactly the budgeted count (otherwise an increase would never be
-  // granted), so refuse to launch anything else.
-  static std::atomic<int> num_regs_cache[2] = {-1, -1};   // a property of each kernel binary
-  int num_regs = num_regs_cache[row_scale].load(std::memory_order_relaxed);
-  if (num_regs < 0) {
-    cudaFuncAttributes fa;
-    e = row_scale ? cudaFuncGetAttributes(&fa, w4a4_gemm_kernel<true>) : cudaFuncGetAttributes(&fa, w4a4_gemm_kernel<false>);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(gemm)");
-    num_regs = fa.numRegs;
-    num_regs_cache[row_scale].store(num_regs, std::memory_order_relaxed);
-  }
-  if (num_regs != (int)REG_LAUNCH) {
-    set_error("w4a4_gemm_kernel compiled with %d registers per thread, %u expected", num_regs, REG_LAUNCH);
-    return PQ_ERR_CUDA;
-  }
-  const int G = (int)(D / g), gsl = g / 32;
+  const int G = (int)(D / g);
   const int scales_vec16 = (G % SC_GROUPS == 0) ? 1 : 0;   // rows of 16-byte multiples
-  if (row_scale)
-    w4a4_gemm_kernel<true><<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB, scales_A, scales_W, Y, (int)T, (int)N,
-                                                                      G, gsl, scales_vec16, out_dtype == PQ_OUT_BF16 ? 1 : 0,
-                                                                      m_tiles, n_tiles, ksplit, gs, ws, status);
-  else
-    w4a4_gemm_kernel<false><<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB, scales_A, scales_W, Y, (int)T, (int)N,
-                                                                       G, gsl, scales_vec16, out_dtype == PQ_OUT_BF16 ? 1 : 0,
-                                                                       m_tiles, n_tiles, ksplit, gs, ws, status);
+  const int bf16 = out_dtype == PQ_OUT_BF16 ? 1 : 0;
+#define PQ_PAIR_CASE(ROW, GSL)                                                                                  \
+  w4a4_gemm_kernel<ROW, GSL><<<grid, NUM_THREADS, kSmemBytes, stream>>>(tmA, tmB, scales_A, scales_W, Y, (int)T, \
+                                                                         (int)N, G, scales_vec16, bf16, m_tiles, \
+                                                                         n_tiles, ksplit, gs, ws, status)
+  if (g == 64) {
+    if (row_scale) PQ_PAIR_CASE(true, 2); else PQ_PAIR_CASE(false, 2);
+  } else if (g == 256) {
+    if (row_scale) PQ_PAIR_CASE(true, 8); else PQ_PAIR_CASE(false, 8);
+  } else {
+    if (row_scale) PQ_PAIR_CASE(true, 4); else PQ_PAIR_CASE(false, 4);
+  }
+#undef PQ_PAIR_CASE
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel launch");
   if (ksplit > 1) return launch_splitk_reduce(ws, ksplit, T, N, Y, out_dtype == PQ_OUT_BF16 ? 1 : 0, stream);
@@ -828,6 +845,42 @@ pq_status gemm_run(const uint8_t* codes_A, const float* scales_A, const uint8_t*
                              static_cast<uint8_t*>(scratch), ws, status, stream, row_scale);
   e = cudaFreeAsync(scratch, stream);
   if (st == PQ_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(gemm scratch)");
+  return st;
+}
+
+pq_status gemm_run_linear(transform_launcher transform, const void* ctx, const uint8_t* codes_A, const float* scales_A,
+                          const uint8_t* codes_W, const float* scales_W, int64_t T, int64_t N, int64_t D, int g,
+                          void* Y, pq_out_dtype out_dtype, cudaStream_t stream) {
+  if (T > kGemmSmallT) {
+    pq_status st = cuda_fail(transform(ctx), "pq_w4a4_linear transform launch");
+    if (st != PQ_OK) return st;
+    return gemm_run(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype, stream, false);
+  }
+  unsigned int* status = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&status), g_gemm_status);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(gemm status)");
+  // The split workspace is taken before the transform, so that the GEMM directly follows it on
+  // the stream and can be its programmatic dependent.
+  const size_t ws_bytes = gemm_workspace_bytes(T, N, D, g);
+  void* scratch = nullptr;
+  if (ws_bytes) {
+    cudaMemPool_t pool = nullptr;
+    e = scratch_pool(&pool);
+    if (e != cudaSuccess) return cuda_fail(e, "scratch memory pool");
+    e = cudaMallocFromPoolAsync(&scratch, ws_bytes, pool, stream);
+    if (e != cudaSuccess) {
+      set_error("cudaMallocFromPoolAsync(%zu bytes of GEMM scratch): %s", ws_bytes, cudaGetErrorString(e));
+      return PQ_ERR_ALLOC;
+    }
+  }
+  pq_status st = cuda_fail(transform(ctx), "pq_w4a4_linear transform launch");
+  if (st == PQ_OK)
+    st = gemm_small_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype, static_cast<float*>(scratch),
+                           status, stream, false, /*pdl=*/true);
+  if (scratch) {
+    e = cudaFreeAsync(scratch, stream);
+    if (st == PQ_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(gemm scratch)");
+  }
   return st;
 }
 

@@ -163,16 +163,21 @@ __device__ __forceinline__ Unit unit_of(int u, int ranges, int gs, int G) {
 
 // kRow: scales_W holds per-(row, group) factors and scales_A one scale per token: per group
 // acc += float(256 d) * (F / 256), and the token's scale multiplies the sum at the end.
-template <int NT, bool kRow>
+template <int NT, bool kRow, int GSL>
 __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
     const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA,
     const float* __restrict__ scales_A, const float* __restrict__ scales_W, void* __restrict__ Y,
-    float* __restrict__ ws, int T, int N, int G, int gsl, int ranges, int gs, int units, int out_bf16,
+    float* __restrict__ ws, int T, int N, int G, int ranges, int gs, int units, int out_bf16, int pdl,
     unsigned int* status) {
-  // gsl: K32 slices per group (g / 32 = 2, 4 or 8); a K-block of 128 codes holds 4, an operand
+  // pdl: launched as the programmatic dependent of the kernel that writes codes_A and scales_A
+  // (pq_w4a4_linear).  The weights were written before that kernel started, so the first ring
+  // of weight tiles is requested at once; activation codes and scales are read only after
+  // griddepcontrol.wait (every role that reads them waits first).
+  // GSL: K32 slices per group (g / 32 = 2, 4 or 8); a K-block of 128 codes holds 4, an operand
   // stage is one K-block and a packed-code stage four.  Group ranges start on K-block boundaries.
   using Smem = SmallSmem<NT>;
-  const int g64 = gsl == 2 ? 1 : 0;
+  constexpr int gsl = GSL;
+  const int g64 = GSL == 2 ? 1 : 0;
   constexpr int RAW = Smem::RAW, GS_OPS = Smem::OPS, GS_NACC = Smem::NACC;
   constexpr uint32_t kTmemCols = GS_NACC * NT < 32 ? 32 : GS_NACC * NT;
   constexpr uint32_t kRawBytes = 2 * GS_M * 128 + 2 * NT * 128;
@@ -219,19 +224,35 @@ __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
     if (lane == 0) {
       int ss = 0;   // stages issued
       bool ok = true;
+      // Activation boxes of the first ring fill are deferred (pdl): their stages' weight boxes go
+      // out first, then griddepcontrol.wait, then these.
+      int pend_kq[RAW];
+      int npend = 0;
+      bool waited = pdl == 0;
+      auto release_pending = [&]() {
+        ptx::griddep_wait();
+        for (int i = 0; i < npend; ++i)
+          for (int b = 0; b < 2; ++b)
+            ptx::tma_load_2d(S.rawA[i][b], &tmA, &S.raw_full[i], (pend_kq[i] + 2 * b) * 64, 0);
+        npend = 0;
+        waited = true;
+      };
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const Unit w = unit_of(u, ranges, gs, G);
         const int kb1 = w.k1 * gsl / 4;
         for (int kq = w.k0 * gsl / 4; kq < kb1; kq += GS_KPS, ++ss) {
           const int s = ss % RAW;
+          if (!waited && ss == RAW) release_pending();
           if (!gs_wait(S, &S.raw_empty[s], ((uint32_t)(ss / RAW) & 1u) ^ 1u, status)) { ok = false; break; }
           ptx::mbar_arrive_expect_tx(&S.raw_full[s], kRawBytes);
           for (int b = 0; b < 2; ++b) {   // K-blocks kq + 2b, kq + 2b + 1 (bytes past a row read as zeros)
             ptx::tma_load_2d(S.rawW[s][b], &tmW, &S.raw_full[s], (kq + 2 * b) * 64, w.m0);
-            ptx::tma_load_2d(S.rawA[s][b], &tmA, &S.raw_full[s], (kq + 2 * b) * 64, 0);
+            if (waited) ptx::tma_load_2d(S.rawA[s][b], &tmA, &S.raw_full[s], (kq + 2 * b) * 64, 0);
           }
+          if (!waited) pend_kq[npend++] = kq;   // ss < RAW: stage s == ss
         }
       }
+      if (!waited) release_pending();   // fewer stages than the ring (or an abort): still land them
       // Every load issued lands before the CTA may exit.
       for (int j = ss > RAW ? ss - RAW : 0; j < ss; ++j)
         gs_drain(&S.raw_full[j % RAW], (uint32_t)(j / RAW) & 1u);
@@ -251,9 +272,12 @@ __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
           ptx::tc_fence_after();
           const uint32_t d = tmem + (uint32_t)(b * NT);
           // K32 per MMA = 32 bytes along the swizzled row; a stage is awaited at its first slice
-          // and released after its fourth; slice 0 of the group overwrites the buffer.
-          for (int sl = 0; sl < gsl; ++sl) {
-            const int sub = ((kg - w.k0) * gsl + sl) & 3;
+          // and released after its fourth; slice 0 of the group overwrites the buffer.  The
+          // slices are unrolled (GSL is a template parameter) so the MMAs issue back to back.
+          const int h = GSL == 2 ? ((kg - w.k0) & 1) : 0;
+#pragma unroll
+          for (int sl = 0; sl < GSL; ++sl) {
+            const int sub = GSL == 2 ? 2 * h + sl : (sl & 3);
             const int o = kstep % GS_OPS;
             if (sub == 0) {
               if (!gs_wait(S, &S.op_full[o], (uint32_t)(kstep / GS_OPS) & 1u, status)) { ok = false; break; }
@@ -304,6 +328,7 @@ __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
     }
   } else {
     ptx::setmaxnreg_inc<GS_REG_EPI>();
+    if (pdl) ptx::griddep_wait();   // token scales come from the preceding grid
     // -------------------------------------------------------------------------- epilogue
     const int ew = warp - GS_EPI0;              // 0..3
     const int quarter = warp & 3;               // TMEM lane quarter this warp may access
@@ -410,12 +435,12 @@ __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
   }
 }
 
-template <int NT, bool kRow>
+template <int NT, bool kRow, int GSL>
 pq_status launch_small(const CUtensorMap& tmW, const CUtensorMap& tmA, const float* scales_A, const float* scales_W,
-                       void* Y, float* ws, int T, int N, int G, int gsl, int ranges, int gs, int units, int out_bf16,
-                       unsigned int* status, cudaStream_t stream) {
+                       void* Y, float* ws, int T, int N, int G, int ranges, int gs, int units, int out_bf16,
+                       bool pdl, unsigned int* status, cudaStream_t stream) {
   static std::atomic<bool> attr_done[kMaxDevices];
-  cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_small_kernel<NT, kRow>),
+  cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_small_kernel<NT, kRow, GSL>),
                                         (int)small_smem_bytes<NT>(), attr_done);
   if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_small_kernel attributes");
   // The warpgroups' setmaxnreg shares are drawn from the launch allocation (compiled registers x
@@ -424,7 +449,7 @@ pq_status launch_small(const CUtensorMap& tmW, const CUtensorMap& tmA, const flo
   int regs = regs_cache.load(std::memory_order_relaxed);
   if (regs < 0) {
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, w4a4_gemm_small_kernel<NT, kRow>);
+    e = cudaFuncGetAttributes(&fa, w4a4_gemm_small_kernel<NT, kRow, GSL>);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes(w4a4_gemm_small_kernel)");
     regs = fa.numRegs;
     regs_cache.store(regs, std::memory_order_relaxed);
@@ -435,9 +460,25 @@ pq_status launch_small(const CUtensorMap& tmW, const CUtensorMap& tmA, const flo
     return PQ_ERR_CUDA;
   }
   const int grid = std::min(units, device_sm_count());
-  w4a4_gemm_small_kernel<NT, kRow><<<grid, GS_THREADS, small_smem_bytes<NT>(), stream>>>(
-      tmW, tmA, scales_A, scales_W, Y, ws, T, N, G, gsl, ranges, gs, units, out_bf16, status);
-  return cuda_fail(cudaGetLastError(), "w4a4_gemm_small_kernel launch");
+  if (!pdl) {
+    w4a4_gemm_small_kernel<NT, kRow, GSL><<<grid, GS_THREADS, small_smem_bytes<NT>(), stream>>>(
+        tmW, tmA, scales_A, scales_W, Y, ws, T, N, G, ranges, gs, units, out_bf16, 0, status);
+    return cuda_fail(cudaGetLastError(), "w4a4_gemm_small_kernel launch");
+  }
+  // Programmatic dependent of the preceding kernel on `stream` (the activation transform).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(GS_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = small_smem_bytes<NT>();
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cuda_fail(cudaLaunchKernelEx(&cfg, w4a4_gemm_small_kernel<NT, kRow, GSL>, tmW, tmA, scales_A, scales_W, Y, ws, T,
+                                      N, G, ranges, gs, units, out_bf16, 1, status),
+                   "w4a4_gemm_small_kernel launch (programmatic dependent)");
 }
 
 static_assert(small_smem_bytes<16>() <= 232448 && small_smem_bytes<32>() <= 232448 &&
@@ -467,7 +508,7 @@ int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int g, int* gs_out) {
 pq_status gemm_small_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                             const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
                             pq_out_dtype out_dtype, float* ws, unsigned int* status, cudaStream_t stream,
-                            bool row_scale) {
+                            bool row_scale, bool pdl) {
   const int NT = T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128;
   const int G = (int)(D / g), gsl = g / 32;
   int gs = G;
@@ -488,17 +529,22 @@ pq_status gemm_small_launch(const uint8_t* codes_A, const float* scales_A, const
   if (e != cudaSuccess) return cuda_fail(e, "tensor map (packed activations)");
   const int bf16 = out_dtype == PQ_OUT_BF16 ? 1 : 0;
   pq_status st;
-#define PQ_SMALL_CASE(W)                                                                                      \
-  st = row_scale ? launch_small<W, true>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, gsl, ranges,  \
-                                         gs, (int)units, bf16, status, stream)                                    \
-                 : launch_small<W, false>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, gsl, ranges, \
-                                          gs, (int)units, bf16, status, stream)
+#define PQ_SMALL_CASE3(W, GSL)                                                                                  \
+  st = row_scale ? launch_small<W, true, GSL>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, ranges, gs, \
+                                              (int)units, bf16, pdl, status, stream)                              \
+                 : launch_small<W, false, GSL>(tmW, tmA, scales_A, scales_W, Y, ws, (int)T, (int)N, G, ranges, gs, \
+                                               (int)units, bf16, pdl, status, stream)
+#define PQ_SMALL_CASE(W)                          \
+  if (gsl == 2) PQ_SMALL_CASE3(W, 2);             \
+  else if (gsl == 8) PQ_SMALL_CASE3(W, 8);        \
+  else PQ_SMALL_CASE3(W, 4)
   switch (NT) {
     case 16: PQ_SMALL_CASE(16); break;
     case 32: PQ_SMALL_CASE(32); break;
     case 64: PQ_SMALL_CASE(64); break;
     default: PQ_SMALL_CASE(128); break;
   }
+#undef PQ_SMALL_CASE3
 #undef PQ_SMALL_CASE
   if (st != PQ_OK || ranges == 1) return st;
   return launch_splitk_reduce(ws, ranges, T, N, Y, bf16, stream);

@@ -147,10 +147,13 @@ constexpr int64_t kGemmSmallT = 128;
 // Group ranges per 128-row weight tile of the few-token kernel (1 = no split); g = group size.
 int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int g, int* gs_out);
 // The few-token GEMM (+ the split reduction when ws != nullptr and the sizes call for it).
+// pdl: launch it as the programmatic dependent of the preceding kernel on `stream`, which must be
+// the one writing codes_A and scales_A, itself started after everything codes_W and scales_W
+// depend on.
 pq_status gemm_small_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                             const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
                             pq_out_dtype out_dtype, float* ws, unsigned int* status, cudaStream_t stream,
-                            bool row_scale);
+                            bool row_scale, bool pdl = false);
 // Y = sum over ksplit float32 partial [T][N] tiles in ws, ascending (gemm.cu).
 pq_status launch_splitk_reduce(const float* ws, int ksplit, int64_t T, int64_t N, void* Y, int out_bf16,
                                cudaStream_t stream);
@@ -172,6 +175,14 @@ pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8
                       const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
                       pq_out_dtype out_dtype, uint8_t* scratch, float* ws, unsigned int* status,
                       cudaStream_t stream, bool row_scale);
+// pq_w4a4_linear: `transform(ctx)` launches the activation transform (writing codes_A and
+// scales_A) on `stream`; the GEMM follows.  T <= 128: the few-token GEMM is launched as the
+// transform's programmatic dependent (its weight loads overlap the transform; the split
+// workspace, if any, is allocated before the transform).  T > 128: as pq_w4a4_gemm.
+typedef cudaError_t (*transform_launcher)(const void* ctx);
+pq_status gemm_run_linear(transform_launcher transform, const void* ctx, const uint8_t* codes_A, const float* scales_A,
+                          const uint8_t* codes_W, const float* scales_W, int64_t T, int64_t N, int64_t D, int g,
+                          void* Y, pq_out_dtype out_dtype, cudaStream_t stream);
 pq_status gemm_read_and_clear_status(unsigned int* bits);
 // Launches the bounded-wait diagnostic (a wait that cannot complete, limited to limit_ns).
 pq_status gemm_wait_timeout_selftest(uint64_t limit_ns, cudaStream_t stream);

@@ -302,10 +302,11 @@ static pq_status check_plan(const pq_plan* plan) {
   return PQ_OK;
 }
 
-extern "C" pq_status pq_transform_quant(const pq_plan* plan, const void* X, int64_t T,
-                                        int64_t ldx, uint8_t* codes, float* scales,
-                                        float* smooth_out, void* stream) {
-  clear_error();
+namespace {
+
+// Argument checks of the activation transform; nothing here touches the device.
+pq_status check_transform_args(const pq_plan* plan, const void* X, int64_t T, int64_t ldx, const uint8_t* codes,
+                               const float* scales, const float* smooth_out) {
   if (!plan) { set_error("plan is NULL"); return PQ_ERR_INVALID_ARG; }
   if (!X || !codes || !scales) { set_error("X, codes and scales must be non-NULL"); return PQ_ERR_INVALID_ARG; }
   if (T < 1) { set_error("T=%lld must be >= 1", (long long)T); return PQ_ERR_INVALID_ARG; }
@@ -323,25 +324,49 @@ extern "C" pq_status pq_transform_quant(const pq_plan* plan, const void* X, int6
     return PQ_ERR_INVALID_ARG;
   }
   if (T >= ((int64_t)1 << 31)) { set_error("T=%lld must be < 2^31", (long long)T); return PQ_ERR_INVALID_ARG; }
-  pq_status st = check_plan(plan);
-  if (st != PQ_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaSuccess;
+  return PQ_OK;
+}
+
+cudaError_t launch_transform(const pq_plan* plan, const void* X, int64_t T, int64_t ldx, uint8_t* codes,
+                             float* scales, float* smooth_out, cudaStream_t s) {
   switch (plan->kind) {
     case PQ_HADAMARD:
-      e = launch_rotate_mma(plan, X, T, ldx, 0, codes, scales, s);
-      break;
     case PQ_GIVENS:
-      e = launch_rotate_mma(plan, X, T, ldx, 0, codes, scales, s);
-      break;
+      return launch_rotate_mma(plan, X, T, ldx, 0, codes, scales, s);
     case PQ_SMOOTH_HADAMARD:
       if (plan->flags & PQ_FLAG_SMOOTH_AFTER_ROTATE)
-        e = launch_smooth_hadamard(plan, X, T, ldx, codes, scales, smooth_out, s);
-      else
-        e = launch_smooth_rows(plan, X, T, ldx, PQ_SR_COLMAX, nullptr, codes, scales, smooth_out, s);
-      break;
+        return launch_smooth_hadamard(plan, X, T, ldx, codes, scales, smooth_out, s);
+      return launch_smooth_rows(plan, X, T, ldx, PQ_SR_COLMAX, nullptr, codes, scales, smooth_out, s);
   }
-  return cuda_fail(e, "pq_transform_quant launch");
+  return cudaErrorInvalidValue;
+}
+
+struct TransformCall {
+  const pq_plan* plan;
+  const void* X;
+  int64_t T, ldx;
+  uint8_t* codes;
+  float* scales;
+  cudaStream_t stream;
+};
+
+cudaError_t transform_thunk(const void* ctx) {
+  const TransformCall& c = *static_cast<const TransformCall*>(ctx);
+  return launch_transform(c.plan, c.X, c.T, c.ldx, c.codes, c.scales, nullptr, c.stream);
+}
+
+}  // namespace
+
+extern "C" pq_status pq_transform_quant(const pq_plan* plan, const void* X, int64_t T,
+                                        int64_t ldx, uint8_t* codes, float* scales,
+                                        float* smooth_out, void* stream) {
+  clear_error();
+  pq_status st = check_transform_args(plan, X, T, ldx, codes, scales, smooth_out);
+  if (st != PQ_OK) return st;
+  st = check_plan(plan);
+  if (st != PQ_OK) return st;
+  return cuda_fail(launch_transform(plan, X, T, ldx, codes, scales, smooth_out, reinterpret_cast<cudaStream_t>(stream)),
+                   "pq_transform_quant launch");
 }
 
 extern "C" pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t N,
@@ -440,6 +465,22 @@ extern "C" pq_status pq_w4a4_gemm_noalloc(const uint8_t* codes_A, const float* s
   if (st != PQ_OK) return st;
   return gemm_run_static_scratch(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype,
                                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+
+extern "C" pq_status pq_w4a4_linear(const pq_plan* plan, const void* X, int64_t T, int64_t ldx, uint8_t* codes_A,
+                                    float* scales_A, const uint8_t* codes_W, const float* scales_W, int64_t N,
+                                    void* Y, pq_out_dtype out_dtype, void* stream) {
+  clear_error();
+  pq_status st = check_transform_args(plan, X, T, ldx, codes_A, scales_A, nullptr);
+  if (st != PQ_OK) return st;
+  st = check_gemm_args(codes_A, scales_A, codes_W, scales_W, T, N, plan->D, plan->g, Y, out_dtype);
+  if (st != PQ_OK) return st;
+  st = check_plan(plan);
+  if (st != PQ_OK) return st;
+  const TransformCall call{plan, X, T, ldx, codes_A, scales_A, reinterpret_cast<cudaStream_t>(stream)};
+  return gemm_run_linear(&transform_thunk, &call, codes_A, scales_A, codes_W, scales_W, T, N, plan->D, plan->g, Y,
+                         out_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // --------------------------------------- rotated runtime smoothing (RRS page, Fig. 4)

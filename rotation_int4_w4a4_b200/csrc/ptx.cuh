@@ -399,6 +399,13 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 
+// ------------------------------------------------------ programmatic dependent launch
+// In a kernel launched with programmatic stream serialization: wait until the preceding grid
+// has completed and its memory operations are visible (returns at once otherwise).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next grid in the stream, if launched as a programmatic dependent, to start now.
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // ------------------------------------------------------------------ packed float32 pairs
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;

@@ -132,6 +132,9 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
   RotSmem& S = *reinterpret_cast<RotSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // A GEMM launched as this grid's programmatic dependent may start its prologue and weight
+  // loads now; it waits for this grid's completion before it reads the codes.
+  ptx::griddep_launch_dependents();
   const int64_t begin = num_tiles * blockIdx.x / gridDim.x;
   const int64_t end = num_tiles * (blockIdx.x + 1) / gridDim.x;
 

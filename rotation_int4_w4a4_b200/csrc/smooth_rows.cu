@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
   const int t = threadIdx.x, lane = t & 31;
   const int64_t first = blockIdx.x, stride = gridDim.x;
   const int64_t D = (int64_t)G * 128;
+  ptx::griddep_launch_dependents();   // a programmatic dependent may start (it waits before reading)
 
   if (t == 0) {
     for (int s = 0; s < SR_STAGES; ++s) ptx::mbar_init(&S.full[s], 1);

@@ -27,7 +27,7 @@ KINDS = {"hadamard": PQ_HADAMARD, "givens": PQ_GIVENS, "smooth_hadamard": PQ_SMO
 # Every symbol the header declares.
 EXPORTS = ("pq_select_pairs", "pq_make_plan", "pq_destroy_plan", "pq_transform_quant",
            "pq_pack_weights", "pq_w4a4_gemm", "pq_w4a4_gemm_noalloc", "pq_w4a4_gemm_launch_count",
-           "pq_w4a4_gemm_launch_count_g",
+           "pq_w4a4_gemm_launch_count_g", "pq_w4a4_linear",
            "pq_rrs_prepare", "pq_rrs_transform_quant", "pq_rrs_pack_weights", "pq_rrs_gemm",
            "pq_check_status",
            "pq_selftest_wait_timeout", "pq_status_string", "pq_last_error")
@@ -52,6 +52,8 @@ lib.pq_w4a4_gemm_launch_count.argtypes = [_i64, _i64, _i64, _c.POINTER(_i32)]
 lib.pq_w4a4_gemm_launch_count.restype = _i32
 lib.pq_w4a4_gemm_launch_count_g.argtypes = [_i64, _i64, _i64, _i32, _c.POINTER(_i32)]
 lib.pq_w4a4_gemm_launch_count_g.restype = _i32
+lib.pq_w4a4_linear.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _i32, _vp]
+lib.pq_w4a4_linear.restype = _i32
 lib.pq_rrs_prepare.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]
 lib.pq_rrs_prepare.restype = _i32
 lib.pq_rrs_transform_quant.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]
@@ -247,6 +249,20 @@ def pq_w4a4_gemm_noalloc(codes_A, scales_A, codes_W, scales_W, Y, T=None, N=None
     T, N, D, out_dtype, ptrs = _gemm_args(codes_A, scales_A, codes_W, scales_W, Y, T, N, D, g, out_dtype)
     _check(lib.pq_w4a4_gemm_noalloc(*ptrs[:4], T, N, D, g, ptrs[4], out_dtype, _stream(stream)),
            "pq_w4a4_gemm_noalloc")
+
+
+def pq_w4a4_linear(plan: Plan, X, codes_A, scales_A, codes_W, scales_W, Y, T=None, ldx=None, N=None,
+                   out_dtype=None, stream=None) -> None:
+    """Transform X into codes_A / scales_A and multiply with the packed weights into Y, one call
+    (for T <= 128 the GEMM overlaps the transform as its programmatic dependent)."""
+    T = X.shape[0] if T is None else T
+    ldx = X.stride(0) if ldx is None else ldx
+    N = codes_W.shape[0] if N is None else N
+    D, g = plan.D, plan.g
+    xp = _arg(X, "X", "bf16", (T - 1) * ldx + D if T > 0 else 0, rows_strided=True)
+    T, N, D, out_dtype, ptrs = _gemm_args(codes_A, scales_A, codes_W, scales_W, Y, T, N, D, g, out_dtype)
+    _check(lib.pq_w4a4_linear(plan.handle, xp, T, ldx, ptrs[0], ptrs[1], ptrs[2], ptrs[3], N, ptrs[4], out_dtype,
+                              _stream(stream)), "pq_w4a4_linear")
 
 
 def pq_rrs_prepare(plan: Plan, X, chan_max, perm, inv_perm, group_scale, T=None, ldx=None, stream=None) -> None:

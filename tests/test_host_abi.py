@@ -108,6 +108,8 @@ def test_gemm_and_transform_validation(pq):
     assert L.pq_w4a4_gemm(p + 4, p, p, p, 4, 16, 128, 128, p, 0, None) == pq.PQ_ERR_INVALID_ARG
     assert L.pq_w4a4_gemm(p, p, p, p, 4, 16, 128, 128, p, 7, None) == pq.PQ_ERR_INVALID_ARG
     assert L.pq_transform_quant(None, p, 4, 128, p, p, None, None) == pq.PQ_ERR_INVALID_ARG
+    assert L.pq_w4a4_linear(None, p, 4, 128, p, p, p, p, 16, p, 0, None) == pq.PQ_ERR_INVALID_ARG
+    assert L.pq_w4a4_gemm_launch_count_g(4, 16, 384, 256, None) == pq.PQ_ERR_INVALID_ARG
     assert L.pq_pack_weights(None, p, 4, None, p, p, None) == pq.PQ_ERR_INVALID_ARG
     L.pq_destroy_plan(None)                              # no-op
 
@@ -142,6 +144,13 @@ def test_gemm_launch_count_query(pq):
     # 64 and 128 tokens: partial tiles would outweigh the weights, so one launch writes Y
     assert pq.pq_w4a4_gemm_launch_count(64, 4096, 4096) == 1
     assert pq.pq_w4a4_gemm_launch_count(128, 14336, 4096) == 1
+    # other group sizes: the same kernels, split by groups of g (ranges of 4 groups)
+    for g in (64, 128, 256):
+        assert pq.pq_w4a4_gemm_launch_count_g(4096, 14336, 4096, g) == 2
+        assert pq.pq_w4a4_gemm_launch_count_g(1, 14336, 4096, g) == 1
+    assert pq.pq_w4a4_gemm_launch_count_g(1, 4096, 4096, 128) == pq.pq_w4a4_gemm_launch_count(1, 4096, 4096)
+    assert pq.pq_w4a4_gemm_launch_count_g(1, 4096, 512, 64) == 2      # 8 groups of 64: two ranges
+    assert pq.pq_w4a4_gemm_launch_count_g(1, 4096, 512, 256) == 1     # 2 groups: one range
 
 
 def test_binding_rejects_host_and_strided_tensors(pq):
