@@ -17,4 +17,5 @@ from .oracle import (NONE, Plan, SplitMix64, TQResult, GemmResult, Quantized,  #
                      select_pairs_group, hadamard_matrix, fwht, hadamard_rotate,
                      hadamard_rotate_explicit, givens_rotate, givens_matrix, smooth_scales,
                      apply_smoothing, bf16_to_f64, bf16_round, RRSPrep, rrs_prepare,
-                     rrs_transform_quant, rrs_pack_weights, rrs_gemm)
+                     rrs_transform_quant, rrs_pack_weights, rrs_gemm, LEVELS8, quantize_mixed,
+                     transform_quant_mixed, pack_weights_mixed, gemm_mixed)

@@ -496,3 +496,69 @@ def rrs_gemm(codes_a, token_scales, codes_w, F, g: int = 128) -> GemmResult:
         acc = (acc + (Fw[:, gi][None, :] * d[gi].astype(np.float32)).astype(np.float32)).astype(np.float32)
         acc64 += Fw[:, gi].astype(np.float64)[None, :] * d[gi].astype(np.float64)
     return GemmResult((acc * sa[:, None]).astype(np.float32), acc64 * sa.astype(np.float64)[:, None])
+
+
+# ------------------------------------ 8-bit outlier groups ([ParoQuant page] §4.1, third remedy)
+LEVELS8 = 119   # symmetric range of an 8-bit code made of two signed 4-bit digits (reading below)
+
+
+def quantize_mixed(y: np.ndarray, g: int, groups8, tie_band: float = 1e-3) -> Quantized:
+    """Mixed precision ([ParoQuant page] §4.1: extreme outliers keep an 8-bit representation):
+    the listed groups are quantised with an 8-bit code, the others as :func:`quantize` (INT4).
+    Per group: L = 119 for an 8-bit group, 7 otherwise; scale = max|y| / L (float32),
+    codes = clamp(round_half_even(L y / max|y|), -L, L) (INT4: -8..7).
+
+    Reading: the page does not fix the 8-bit format.  An 8-bit code here is one byte made of two
+    signed 4-bit digits, q = 16 q_hi + q_lo with q_hi, q_lo in -8..7 (so that an 8-bit group can
+    be multiplied as four 4-bit groups); the largest symmetric range of such bytes is +-119.
+    Returns int16 codes [rows, D] (not packed)."""
+    rows, D = y.shape
+    G = D // g
+    L = np.full(G, 7.0)
+    L[np.asarray(list(groups8), dtype=np.int64)] = float(LEVELS8)
+    yg = y.reshape(rows, G, g)
+    if not np.all(np.isfinite(yg)):
+        raise ValueError("non-finite input is outside the contract")
+    m = np.max(np.abs(yg), axis=2, keepdims=True)
+    safe = np.where(m > 0.0, m, 1.0)
+    ratio = np.where(m > 0.0, L[None, :, None] * yg / safe, 0.0)
+    low = np.where(L == 7.0, -8.0, -float(LEVELS8))[None, :, None]
+    codes = np.clip(np.rint(ratio), low, L[None, :, None]).astype(np.int16)
+    scales = (m[..., 0] / L[None, :]).astype(np.float32)
+    frac = ratio - np.floor(ratio)
+    near = np.abs(frac - 0.5) < tie_band
+    return Quantized(codes.reshape(rows, D), scales, ratio.reshape(rows, D), near.reshape(rows, D))
+
+
+def transform_quant_mixed(x_bits: np.ndarray, plan: Plan, groups8) -> TQResult:
+    """The activation path with 8-bit outlier groups (codes unpacked, int16 [rows, D])."""
+    y, s = activation_transform(bf16_to_f64(x_bits), plan)
+    q = quantize_mixed(y, plan.g, groups8)
+    return TQResult(q.codes, q.scales, None if s is None else s.astype(np.float32), q, y)
+
+
+def pack_weights_mixed(w_bits: np.ndarray, plan: Plan, groups8, smooth_w: np.ndarray | None = None) -> TQResult:
+    """The weight path with the same 8-bit groups (codes unpacked, int16 [rows, D])."""
+    y = weight_transform(bf16_to_f64(w_bits), plan, smooth_w)
+    q = quantize_mixed(y, plan.g, groups8)
+    return TQResult(q.codes, q.scales, None, q, y)
+
+
+def gemm_mixed(qa: np.ndarray, scales_a, qw: np.ndarray, scales_w, g: int = 128) -> GemmResult:
+    """The W4A4 GEMM of :func:`gemm` on integer codes of either width (unpacked):
+    Y[t,n] = sum_G fl32(fl32(sa sw) d_G), d_G the exact integer dot (|d| <= 128 * 119^2 < 2^21,
+    exact in float32), float32 accumulation over G ascending; float64 shadow of the exact sum."""
+    qa = np.asarray(qa, dtype=np.float64)
+    qw = np.asarray(qw, dtype=np.float64)
+    T, D = qa.shape
+    N = qw.shape[0]
+    sa = np.asarray(scales_a, dtype=np.float32)
+    sw = np.asarray(scales_w, dtype=np.float32)
+    acc = np.zeros((T, N), dtype=np.float32)
+    acc64 = np.zeros((T, N), dtype=np.float64)
+    for gi in range(D // g):
+        d = qa[:, gi * g:(gi + 1) * g] @ qw[:, gi * g:(gi + 1) * g].T
+        s = sa[:, gi][:, None] * sw[:, gi][None, :]
+        acc = (acc + (s * d.astype(np.float32)).astype(np.float32)).astype(np.float32)
+        acc64 += sa[:, gi].astype(np.float64)[:, None] * sw[:, gi].astype(np.float64)[None, :] * d
+    return GemmResult(acc, acc64)
