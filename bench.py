@@ -399,9 +399,10 @@ def dev_bf16(bits, dev):
 
 
 class Setup:
-    """A workload's plan and device buffers (one or several complete sets)."""
+    """A workload's plan and device buffers (one or several complete sets); groups8: 8-bit
+    outlier groups of the plan (codes and scales then hold the plan's Gx groups per row)."""
 
-    def __init__(self, wl, dev, l2):
+    def __init__(self, wl, dev, l2, groups8=None):
         import torch
 
         from rotation_int4_w4a4_b200 import pq
@@ -410,16 +411,17 @@ class Setup:
             pairs = pq.pq_select_pairs(wl.pair_seed, wl.D, wl.g, wl.K, wl.g // 2)
             self.plan = pq.Plan("givens", wl.D, K=wl.K, pairs=pairs, angles=wl.angles, beta=wl.beta)
         else:
-            self.plan = pq.Plan(wl.kind, wl.D, g=wl.g)
-        T, D, N, G = wl.T, wl.D, wl.N, wl.D // wl.g
+            self.plan = pq.Plan(wl.kind, wl.D, g=wl.g, groups8=groups8)
+        T, D, N = wl.T, wl.D, wl.N
+        G, Dx = getattr(self.plan, "Gx", D // wl.g), getattr(self.plan, "Dx", D)
         self.X0, self.W0 = dev_bf16(wl.X, dev), dev_bf16(wl.W, dev)
         self.smooth_w = torch.ones(D, dtype=torch.float32, device=dev) if wl.kind == "smooth_hadamard" else None
 
         def buffer_set(first):
             return {"X": self.X0 if first else self.X0.clone(), "W": self.W0 if first else self.W0.clone(),
-                    "ca": torch.empty((T, D // 2), dtype=torch.uint8, device=dev),
+                    "ca": torch.empty((T, Dx // 2), dtype=torch.uint8, device=dev),
                     "sa": torch.empty((T, G), dtype=torch.float32, device=dev),
-                    "cw": torch.empty((N, D // 2), dtype=torch.uint8, device=dev),
+                    "cw": torch.empty((N, Dx // 2), dtype=torch.uint8, device=dev),
                     "sw": torch.empty((N, G), dtype=torch.float32, device=dev),
                     "Y": torch.empty((T, N), dtype=torch.float32, device=dev),
                     "sm": torch.empty(((T + 127) // 128, D), dtype=torch.float32, device=dev)
@@ -549,9 +551,10 @@ def e2e_run(args, setup, stream):
     return total / n, hX.numel() * 2 + hW.numel() * 2, hY.numel() * 4
 
 
-def measure_also(name, args, dev, stream, peaks, peak_src, g=None):
+def measure_also(name, args, dev, stream, peaks, peak_src, g=None, outliers8=False):
     """Components of another workload (fewer steps, same method), for the extra keys; g: the same
-    workload at another group size (block-Hadamard workloads)."""
+    workload at another group size (block-Hadamard workloads); outliers8: the groups holding the
+    activations' 8 largest channels kept as 8-bit groups."""
     import dataclasses
 
     import torch
@@ -560,7 +563,13 @@ def measure_also(name, args, dev, stream, peaks, peak_src, g=None):
     wl = inputs.workload(name)
     if g is not None:
         wl = dataclasses.replace(wl, g=g, name=f"{name}_g{g}")
-    setup = Setup(wl, dev, "flush")
+    groups8 = None
+    if outliers8:
+        import numpy as np
+        x = np.abs(inputs.bf16_bits_to_f32(wl.X)).max(axis=0)
+        groups8 = sorted(set(int(c) // wl.g for c in np.argsort(-x)[:8]))
+        wl = dataclasses.replace(wl, name=f"{name}_outliers8")
+    setup = Setup(wl, dev, "flush", groups8)
     for i in range(max(3, args.warmup)):
         setup.flush()
         setup.run_step(i, stream)
@@ -751,6 +760,7 @@ def run_ours(args, wl, rank, world, local_rank):
             also[name] = measure_also(name, args, dev, stream, peaks, peak_src)
         for g in (64, 256):
             also[f"q_proj_g{g}"] = measure_also("q_proj", args, dev, stream, peaks, peak_src, g=g)
+        also["q_proj_outliers8"] = measure_also("q_proj", args, dev, stream, peaks, peak_src, outliers8=True)
         also["rrs_down_proj"] = measure_rrs(args, dev, stream, peaks, peak_src)
         also["decode"] = measure_decode(args, dev, stream, peaks, peak_src)
     if rank != 0:

@@ -121,6 +121,30 @@ pq_status pq_select_pairs(uint64_t seed, int D, int g, int K, int N, uint8_t* pa
 pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int K, const uint8_t* pairs,
                        const float* angles, const float* beta, uint32_t flags);
 
+/*
+ * pq_make_plan_outliers — pq_make_plan with 8-bit outlier groups (ParoQuant page §4.1: extreme
+ * outliers keep an 8-bit representation).  PQ_HADAMARD or PQ_GIVENS with g = 128 only
+ * (PQ_ERR_UNSUPPORTED otherwise).
+ *   n8       number of 8-bit groups, 0 <= n8 <= D/g (0: the same plan as pq_make_plan).
+ *   groups8  host int32 [n8]: distinct group indices.
+ *   In those groups a row's codes are q = RNE(119 y / m) (|q| <= 119), scale s = m / 119 (with the
+ *   Hadamard's 1/sqrt(g) folded in as for 4-bit groups).  Each 8-bit code is written as two signed
+ *   4-bit digits, q = 16 q_hi + q_lo with q_hi, q_lo in -8..7 (119 is the largest symmetric range
+ *   that splits so), and the group as four 4-bit groups of the ordinary layout, so that
+ *   pq_w4a4_gemm computes the 8-bit product exactly from 4-bit codes:
+ *     codes and scales hold Gx = D/g + 3 n8 groups per row ([T][Gx*g/2] bytes, [T][Gx] floats);
+ *     8-bit group gi, the j-th listed, uses its own slot gi and the appended slots G + 3j,
+ *     G + 3j + 1, G + 3j + 2 (G = D/g);
+ *     activations: digits (hi, hi, lo, lo), scales (16 s, 16 s, s, s);
+ *     weights:     digits (hi, lo, hi, lo), scales (16 s, s, 16 s, s);
+ *   so the four digit-group products add up to s_a s_w sum(q_a q_w).  Multiply with
+ *   pq_w4a4_gemm(..., D = Gx * g, g) (pq_w4a4_linear does this itself).  The plan is otherwise
+ *   as from pq_make_plan; rotated runtime smoothing rejects it.
+ */
+pq_status pq_make_plan_outliers(pq_plan** out, pq_kind kind, int D, int g, int K, const uint8_t* pairs,
+                                const float* angles, const float* beta, uint32_t flags, int n8,
+                                const int32_t* groups8);
+
 /* pq_destroy_plan — frees the plan's device tables (synchronous).  NULL is a no-op. */
 void pq_destroy_plan(pq_plan* plan);
 
@@ -200,7 +224,8 @@ pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A, const uint
  *   and its weight-side loads start while the transform runs, and it reads codes_A and scales_A
  *   only after the transform has completed.  T > 128: the two run one after the other.
  *   codes_A [T][D/2] and scales_A [T][D/g] are caller-owned device buffers and are written (the
- *   activation codes stay available).  codes_W and scales_W must be complete when the call is
+ *   activation codes stay available; with 8-bit outlier groups D is the plan's Gx * g and D/g its
+ *   Gx, for codes_W and scales_W too).  codes_W and scales_W must be complete when the call is
  *   made (written by work enqueued on `stream` before it, or earlier); Y must not overlap X,
  *   codes_A or scales_A.  Arguments as for the two calls (smoothing plans: no smooth_out).
  *   Launches: the transform's plus pq_w4a4_gemm_launch_count_g(T, N, D, g).

@@ -29,12 +29,18 @@ struct pq_plan {
   int K;
   uint32_t flags;
   int device;
-  // Tensor-core rotation operands (bf16, [n][k] = R[k][n]):
-  //   Givens:   [2 (activations, weights)][G][2 (hi, lo)][128][128] for R = G_0 ... G_{K-1}
-  //             diag(exp(-+beta)) per group (y = x R);
-  //   Hadamard: [128][128] unnormalised H_128 (also used by the smooth kinds' plans, unused there).
+  // Tensor-core rotation operands (bf16, [n][k] = R[k][n]), one 128 x 128 matrix per tile:
+  //   Givens:   [2 (activations, weights)][D/128][2 (hi, lo)][128][128] for R = G_0 ... G_{K-1}
+  //             diag(exp(-+beta)) per group (y = x R; two groups on the diagonal at g = 64);
+  //   Hadamard: unnormalised H_128, diag(H_64, H_64) (g = 64) or +H_128 and -H_128 (g = 256).
   uint16_t* d_rot;
   unsigned int* d_status;   // device status word (PQ_DEV_* bits)
+  // 8-bit outlier groups (g = 128): n8 groups, d_slot8[G] = the group's index among them or -1.
+  // Codes and scales then have Gx = G + 3 n8 groups per row (four 4-bit digit groups per 8-bit
+  // group: its own slot and three appended at G + 3 j).
+  int n8;
+  int Gx;
+  int16_t* d_slot8;
 };
 
 namespace pq {

@@ -108,6 +108,7 @@ static void free_plan_tables(pq_plan* p) {
   if (!p) return;
   if (p->d_rot) cudaFree(p->d_rot);
   if (p->d_status) cudaFree(p->d_status);
+  if (p->d_slot8) cudaFree(p->d_slot8);
 }
 
 template <class T>
@@ -186,10 +187,8 @@ static void build_rotation_operands(int D, int g, int K, const uint8_t* pairs, c
   }
 }
 
-extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int K,
-                                  const uint8_t* pairs, const float* angles, const float* beta,
-                                  uint32_t flags) {
-  clear_error();
+static pq_status make_plan(pq_plan** out, pq_kind kind, int D, int g, int K, const uint8_t* pairs,
+                           const float* angles, const float* beta, uint32_t flags, int n8, const int32_t* groups8) {
   if (!out) { set_error("out is NULL"); return PQ_ERR_INVALID_ARG; }
   if (kind != PQ_HADAMARD && kind != PQ_GIVENS && kind != PQ_SMOOTH_HADAMARD) {
     set_error("unknown kind %d", (int)kind);
@@ -212,6 +211,24 @@ extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int
     return PQ_ERR_INVALID_ARG;
   }
   const int G = D / g, half = g / 2;
+  // 8-bit outlier groups (ParoQuant page §4.1): distinct group indices, rotation plans at g = 128.
+  std::vector<int16_t> slot8;
+  if (n8 != 0) {
+    if (n8 < 0 || n8 > G || !groups8) { set_error("n8=%d: 0..G groups and a group list are needed", n8); return PQ_ERR_INVALID_ARG; }
+    if ((kind != PQ_HADAMARD && kind != PQ_GIVENS) || g != kGroup) {
+      set_error("8-bit outlier groups need a PQ_HADAMARD or PQ_GIVENS plan with g = 128");
+      return PQ_ERR_UNSUPPORTED;
+    }
+    slot8.assign(G, -1);
+    for (int j = 0; j < n8; ++j) {
+      const int32_t gi = groups8[j];
+      if (gi < 0 || gi >= G || slot8[gi] >= 0) {
+        set_error("groups8[%d]=%d must be distinct group indices below G=%d", j, gi, G);
+        return PQ_ERR_INVALID_ARG;
+      }
+      slot8[gi] = (int16_t)j;
+    }
+  }
   if (kind == PQ_GIVENS) {
     if (K < 1 || K > 64) { set_error("K=%d out of range 1..64", K); return PQ_ERR_INVALID_ARG; }
     if (!pairs || !angles) { set_error("Givens plan needs pairs and angles"); return PQ_ERR_INVALID_ARG; }
@@ -277,6 +294,9 @@ extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int
     st = upload(&p->d_rot, h.data(), h.size(), "hadamard tensor-core operand");
   }
   if (st == PQ_OK) st = upload<unsigned int>(&p->d_status, nullptr, 1, "status word");
+  p->n8 = n8;
+  p->Gx = G + 3 * n8;
+  if (st == PQ_OK && n8 > 0) st = upload(&p->d_slot8, slot8.data(), slot8.size(), "8-bit group slots");
   if (st != PQ_OK) {
     free_plan_tables(p);
     delete p;
@@ -284,6 +304,20 @@ extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int
   }
   *out = p;
   return PQ_OK;
+}
+
+extern "C" pq_status pq_make_plan(pq_plan** out, pq_kind kind, int D, int g, int K,
+                                  const uint8_t* pairs, const float* angles, const float* beta,
+                                  uint32_t flags) {
+  clear_error();
+  return make_plan(out, kind, D, g, K, pairs, angles, beta, flags, 0, nullptr);
+}
+
+extern "C" pq_status pq_make_plan_outliers(pq_plan** out, pq_kind kind, int D, int g, int K,
+                                           const uint8_t* pairs, const float* angles, const float* beta,
+                                           uint32_t flags, int n8, const int32_t* groups8) {
+  clear_error();
+  return make_plan(out, kind, D, g, K, pairs, angles, beta, flags, n8, groups8);
 }
 
 extern "C" void pq_destroy_plan(pq_plan* plan) {
@@ -474,12 +508,14 @@ extern "C" pq_status pq_w4a4_linear(const pq_plan* plan, const void* X, int64_t 
   clear_error();
   pq_status st = check_transform_args(plan, X, T, ldx, codes_A, scales_A, nullptr);
   if (st != PQ_OK) return st;
-  st = check_gemm_args(codes_A, scales_A, codes_W, scales_W, T, N, plan->D, plan->g, Y, out_dtype);
+  // The GEMM's reduction length: D, or with 8-bit groups the Gx groups of their digit layout.
+  const int64_t Dk = (int64_t)plan->Gx * plan->g;
+  st = check_gemm_args(codes_A, scales_A, codes_W, scales_W, T, N, Dk, plan->g, Y, out_dtype);
   if (st != PQ_OK) return st;
   st = check_plan(plan);
   if (st != PQ_OK) return st;
   const TransformCall call{plan, X, T, ldx, codes_A, scales_A, reinterpret_cast<cudaStream_t>(stream)};
-  return gemm_run_linear(&transform_thunk, &call, codes_A, scales_A, codes_W, scales_W, T, N, plan->D, plan->g, Y,
+  return gemm_run_linear(&transform_thunk, &call, codes_A, scales_A, codes_W, scales_W, T, N, Dk, plan->g, Y,
                          out_dtype, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -488,8 +524,8 @@ namespace {
 
 pq_status check_rrs_plan(const pq_plan* plan) {
   if (!plan) { set_error("plan is NULL"); return PQ_ERR_INVALID_ARG; }
-  if (plan->kind != PQ_HADAMARD || plan->g != kGroup) {
-    set_error("rotated runtime smoothing needs a PQ_HADAMARD plan with g = 128");
+  if (plan->kind != PQ_HADAMARD || plan->g != kGroup || plan->n8 != 0) {
+    set_error("rotated runtime smoothing needs a PQ_HADAMARD plan with g = 128 (no 8-bit groups)");
     return PQ_ERR_UNSUPPORTED;
   }
   if (plan->D > 16384 || rrs_rows_smem_bytes(plan->D) > 232448) {

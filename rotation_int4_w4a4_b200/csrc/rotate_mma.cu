@@ -109,6 +109,18 @@ __device__ __forceinline__ uint32_t rt_pack8(const float* v, float inv) {
   return (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
 }
 
+// 8 values -> 8 high digits of 8-bit codes: with q = RNE(v * inv) (|q| <= 119), the high digit
+// floor((q + 8) / 16) is bits 4..7 of q + 8, which the FMA with 1.5 * 2^23 + 8 leaves there (the
+// low digit, q - 16 q_hi, has the nibble of q itself: rt_pack8).
+__device__ __forceinline__ uint32_t rt_pack8_hi(const float* v, float inv) {
+  uint32_t b[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) b[k] = __float_as_uint(fmaf(v[k], inv, kRoundMagicR + 8.0f)) >> 4;
+  const uint32_t even = __byte_perm(__byte_perm(b[0], b[2], 0x0040), __byte_perm(b[4], b[6], 0x0040), 0x5410);
+  const uint32_t odd = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
+  return (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);
+}
+
 // Tiles are numbered group-major: tile = gi * row_blocks + rb.  CTA c owns [begin, end).
 // terms: 1 (R exact in bf16) or 2 (R_hi + R_lo).  r_groups: number of distinct matrices (G, or 1
 // when every group uses the same one).  scale_mult: stored scale = max|y| * scale_mult.
@@ -120,11 +132,18 @@ __device__ __forceinline__ uint32_t rt_pack8(const float* v, float inv) {
 // non-negative, for which the bit order is the numeric order).  Rows past the end read as zeros.
 // GW: the group size (64, 128 or 256); G counts groups of GW channels; a tile spans
 // RtGeom<GW>::TW channels (one group for 128 and 256, two for 64).
+// Gx, slot8, scale_mult8, weights (g = 128): 8-bit outlier groups (ParoQuant page §4.1).  Rows
+// of codes and scales hold Gx = G + 3 n8 groups; slot8[gi] >= 0 marks an 8-bit group j: its
+// codes q = RNE(119 y / m) split into digits q = 16 q_hi + q_lo (both -8..7), written as four
+// 4-bit groups with power-of-two scale factors so that the W4A4 GEMM forms the 8-bit product:
+// activations (hi, hi, lo, lo) with (16 s, 16 s, s, s), weights (hi, lo, hi, lo) with
+// (16 s, s, 16 s, s), at slots gi, G + 3j, G + 3j + 1, G + 3j + 2; s = m * scale_mult8.
 template <bool kColMax, int GW>
 __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
     const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmR, int64_t rows, int G,
     int row_blocks, int64_t num_tiles, int terms, int r_groups, float scale_mult, uint8_t* __restrict__ codes,
-    float* __restrict__ scales, unsigned int* __restrict__ chan_max, unsigned int* status) {
+    float* __restrict__ scales, unsigned int* __restrict__ chan_max, unsigned int* status, int Gx,
+    const int16_t* __restrict__ slot8, float scale_mult8, int weights) {
   static_assert(!kColMax || GW == 128, "column maxima are taken on 128-channel groups");
   using Geo = RtGeom<GW>;
   constexpr int KBS = Geo::KBS, STAGES = Geo::STAGES;
@@ -342,14 +361,43 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
         }
         continue;
       }
+      const int j8 = slot8 != nullptr ? (int)__ldg(slot8 + gi) : -1;   // the same for the whole tile
+      if (j8 >= 0) {
+        if (t < rows) {
+          const float inv8 = m > 0.0f ? 119.0f * __frcp_rn(m) : 0.0f;
+          uint8_t* crow = codes + t * (int64_t)Gx * 64;
+          uint4* hi_a = reinterpret_cast<uint4*>(crow + gi * 64);
+          uint4* hi_b = reinterpret_cast<uint4*>(crow + (G + 3 * j8 + (weights ? 1 : 0)) * 64);
+          uint4* lo_a = reinterpret_cast<uint4*>(crow + (G + 3 * j8 + (weights ? 0 : 1)) * 64);
+          uint4* lo_b = reinterpret_cast<uint4*>(crow + (G + 3 * j8 + 2) * 64);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint4 hi = make_uint4(rt_pack8_hi(y + 32 * k, inv8), rt_pack8_hi(y + 32 * k + 8, inv8),
+                                        rt_pack8_hi(y + 32 * k + 16, inv8), rt_pack8_hi(y + 32 * k + 24, inv8));
+            const uint4 lo = make_uint4(rt_pack8(y + 32 * k, inv8), rt_pack8(y + 32 * k + 8, inv8),
+                                        rt_pack8(y + 32 * k + 16, inv8), rt_pack8(y + 32 * k + 24, inv8));
+            hi_a[k] = hi;
+            hi_b[k] = hi;
+            lo_a[k] = lo;
+            lo_b[k] = lo;
+          }
+          const float s8 = m * scale_mult8;
+          float* srow = scales + t * Gx;
+          srow[gi] = 16.0f * s8;
+          srow[G + 3 * j8] = weights ? s8 : 16.0f * s8;
+          srow[G + 3 * j8 + 1] = weights ? 16.0f * s8 : s8;
+          srow[G + 3 * j8 + 2] = s8;
+        }
+        continue;
+      }
       const float inv = m > 0.0f ? 7.0f * __frcp_rn(m) : 0.0f;
       if (t < rows) {
-        uint4* dst = reinterpret_cast<uint4*>(codes + t * (int64_t)G * 64 + gi * 64);
+        uint4* dst = reinterpret_cast<uint4*>(codes + t * (int64_t)Gx * 64 + gi * 64);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           dst[k] = make_uint4(rt_pack8(y + 32 * k, inv), rt_pack8(y + 32 * k + 8, inv),
                               rt_pack8(y + 32 * k + 16, inv), rt_pack8(y + 32 * k + 24, inv));
-        scales[t * G + gi] = m * scale_mult;
+        scales[t * Gx + gi] = m * scale_mult;
       }
       }   // GW <= 128
     }
@@ -438,7 +486,7 @@ namespace {
 template <int GW>
 cudaError_t launch_rotate_mma_g(const pq_plan* plan, const CUtensorMap& tmX, const CUtensorMap& tmR, int64_t rows,
                                 int terms, int r_groups, float scale_mult, uint8_t* codes, float* scales,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, float scale_mult8 = 0.0f, int weights = 0) {
   const int row_blocks = (int)((rows + RT_M - 1) / RT_M);
   const int64_t tiles = (int64_t)row_blocks * (plan->D / RtGeom<GW>::TW);
   const int sms = device_sm_count();
@@ -448,7 +496,8 @@ cudaError_t launch_rotate_mma_g(const pq_plan* plan, const CUtensorMap& tmX, con
                                         attr_done);
   if (e != cudaSuccess) return e;
   rotate_mma_kernel<false, GW><<<grid, RT_THREADS, kRotSmemBytes, stream>>>(
-      tmX, tmR, rows, plan->G, row_blocks, tiles, terms, r_groups, scale_mult, codes, scales, nullptr, plan->d_status);
+      tmX, tmR, rows, plan->G, row_blocks, tiles, terms, r_groups, scale_mult, codes, scales, nullptr, plan->d_status,
+      plan->Gx, plan->n8 > 0 ? plan->d_slot8 : nullptr, scale_mult8, weights);
   return cudaGetLastError();
 }
 
@@ -481,7 +530,7 @@ cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, 
     if (e != cudaSuccess) return e;
     rotate_mma_kernel<true, 128><<<grid, RT_THREADS, kRotSmemBytes, stream>>>(
         tmX, tmR, rows, plan->G, row_blocks, tiles, terms, r_groups, givens ? 1.0f : 0.088388347648318440550f,
-        nullptr, nullptr, chan_max, plan->d_status);
+        nullptr, nullptr, chan_max, plan->d_status, plan->G, nullptr, 0.0f, 0);
     return cudaGetLastError();
   }
   // Givens: scale = m / 7.  Hadamard: R = H unnormalised, so y is sqrt(g) times the orthonormal
@@ -493,8 +542,10 @@ cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, 
     case 256:
       return launch_rotate_mma_g<256>(plan, tmX, tmR, rows, terms, r_groups, 1.0f / 112.0f, codes, scales, stream);
     default:
+      // 8-bit groups: scale = m / 119 (Givens) or m / (119 sqrt(128)) (Hadamard).
       return launch_rotate_mma_g<128>(plan, tmX, tmR, rows, terms, r_groups,
-                                      givens ? (1.0f / 7.0f) : 0.012626906806902634f, codes, scales, stream);
+                                      givens ? (1.0f / 7.0f) : 0.012626906806902634f, codes, scales, stream,
+                                      givens ? (1.0f / 119.0f) : 0.00074275922393545f, weights);
   }
 }
 

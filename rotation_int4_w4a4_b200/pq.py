@@ -27,7 +27,7 @@ KINDS = {"hadamard": PQ_HADAMARD, "givens": PQ_GIVENS, "smooth_hadamard": PQ_SMO
 # Every symbol the header declares.
 EXPORTS = ("pq_select_pairs", "pq_make_plan", "pq_destroy_plan", "pq_transform_quant",
            "pq_pack_weights", "pq_w4a4_gemm", "pq_w4a4_gemm_noalloc", "pq_w4a4_gemm_launch_count",
-           "pq_w4a4_gemm_launch_count_g", "pq_w4a4_linear",
+           "pq_w4a4_gemm_launch_count_g", "pq_w4a4_linear", "pq_make_plan_outliers",
            "pq_rrs_prepare", "pq_rrs_transform_quant", "pq_rrs_pack_weights", "pq_rrs_gemm",
            "pq_check_status",
            "pq_selftest_wait_timeout", "pq_status_string", "pq_last_error")
@@ -38,6 +38,8 @@ lib.pq_select_pairs.argtypes = [_u64, _i32, _i32, _i32, _i32, _vp]
 lib.pq_select_pairs.restype = _i32
 lib.pq_make_plan.argtypes = [_c.POINTER(_vp), _i32, _i32, _i32, _i32, _vp, _vp, _vp, _u32]
 lib.pq_make_plan.restype = _i32
+lib.pq_make_plan_outliers.argtypes = [_c.POINTER(_vp), _i32, _i32, _i32, _i32, _vp, _vp, _vp, _u32, _i32, _vp]
+lib.pq_make_plan_outliers.restype = _i32
 lib.pq_destroy_plan.argtypes = [_vp]
 lib.pq_destroy_plan.restype = None
 lib.pq_transform_quant.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp]
@@ -146,9 +148,14 @@ class Plan:
     """Owns a ``pq_plan`` (device tables); freed by :meth:`close` or garbage collection."""
 
     def __init__(self, kind, D: int, g: int = 128, K: int = 0, pairs=None, angles=None,
-                 beta=None, flags: int = 0):
+                 beta=None, flags: int = 0, groups8=None):
+        """groups8: group indices kept as 8-bit outlier groups (codes and scales then hold
+        Gx = D/g + 3 len(groups8) groups per row; see ``Dx``)."""
         kind = KINDS.get(kind, kind)
         self.kind, self.D, self.g, self.K, self.flags = kind, D, g, K, flags
+        self.groups8 = [] if groups8 is None else [int(v) for v in groups8]
+        self.Gx = D // g + 3 * len(self.groups8)
+        self.Dx = self.Gx * g            # the GEMM's reduction length for this plan's codes
         keep = []
 
         def host(a, dt):
@@ -159,9 +166,15 @@ class Plan:
             return a.ctypes.data
 
         h = _vp()
-        _check(lib.pq_make_plan(_c.byref(h), kind, D, g, K, host(pairs, np.uint8),
-                                host(angles, np.float32), host(beta, np.float32), flags),
-               "pq_make_plan")
+        if self.groups8:
+            _check(lib.pq_make_plan_outliers(_c.byref(h), kind, D, g, K, host(pairs, np.uint8),
+                                             host(angles, np.float32), host(beta, np.float32), flags,
+                                             len(self.groups8), host(self.groups8, np.int32)),
+                   "pq_make_plan_outliers")
+        else:
+            _check(lib.pq_make_plan(_c.byref(h), kind, D, g, K, host(pairs, np.uint8),
+                                    host(angles, np.float32), host(beta, np.float32), flags),
+                   "pq_make_plan")
         self._h = h
 
     @property
@@ -190,26 +203,27 @@ def pq_destroy_plan(plan: Plan) -> None:
 
 def pq_transform_quant(plan: Plan, X, codes, scales, smooth_out=None, T=None, ldx=None,
                        stream=None) -> None:
-    """X bf16 [T, ldx] -> codes uint8 [T, D/2], scales float32 [T, D/g] (device tensors)."""
+    """X bf16 [T, ldx] -> codes uint8 [T, Dx/2], scales float32 [T, Gx] (device tensors;
+    Dx = D and Gx = D/g unless the plan has 8-bit groups)."""
     T = X.shape[0] if T is None else T
     ldx = X.stride(0) if ldx is None else ldx
-    D, G = plan.D, plan.D // plan.g
+    D, G = plan.D, plan.Gx
     if not isinstance(X, int) and X.dim() == 2 and X.stride(0) != ldx:
         raise ValueError(f"X: row stride {X.stride(0)} differs from ldx={ldx}")
     xp = _arg(X, "X", "bf16", (T - 1) * ldx + D if T > 0 else 0, rows_strided=True)
-    _check(lib.pq_transform_quant(plan.handle, xp, T, ldx, _arg(codes, "codes", "u8", T * D // 2),
+    _check(lib.pq_transform_quant(plan.handle, xp, T, ldx, _arg(codes, "codes", "u8", T * plan.Dx // 2),
                                   _arg(scales, "scales", "f32", T * G),
                                   _arg(smooth_out, "smooth_out", "f32", -(-T // 128) * D),
                                   _stream(stream)), "pq_transform_quant")
 
 
 def pq_pack_weights(plan: Plan, W, codes_W, scales_W, smooth_w=None, N=None, stream=None) -> None:
-    """W bf16 [N, D] -> codes_W uint8 [N, D/2], scales_W float32 [N, D/g] (device tensors)."""
+    """W bf16 [N, D] -> codes_W uint8 [N, Dx/2], scales_W float32 [N, Gx] (device tensors)."""
     N = W.shape[0] if N is None else N
-    D, G = plan.D, plan.D // plan.g
+    D, G = plan.D, plan.Gx
     _check(lib.pq_pack_weights(plan.handle, _arg(W, "W", "bf16", N * D), N,
                                _arg(smooth_w, "smooth_w", "f32", D),
-                               _arg(codes_W, "codes_W", "u8", N * D // 2),
+                               _arg(codes_W, "codes_W", "u8", N * plan.Dx // 2),
                                _arg(scales_W, "scales_W", "f32", N * G), _stream(stream)),
            "pq_pack_weights")
 
@@ -260,7 +274,7 @@ def pq_w4a4_linear(plan: Plan, X, codes_A, scales_A, codes_W, scales_W, Y, T=Non
     N = codes_W.shape[0] if N is None else N
     D, g = plan.D, plan.g
     xp = _arg(X, "X", "bf16", (T - 1) * ldx + D if T > 0 else 0, rows_strided=True)
-    T, N, D, out_dtype, ptrs = _gemm_args(codes_A, scales_A, codes_W, scales_W, Y, T, N, D, g, out_dtype)
+    T, N, _, out_dtype, ptrs = _gemm_args(codes_A, scales_A, codes_W, scales_W, Y, T, N, plan.Dx, g, out_dtype)
     _check(lib.pq_w4a4_linear(plan.handle, xp, T, ldx, ptrs[0], ptrs[1], ptrs[2], ptrs[3], N, ptrs[4], out_dtype,
                               _stream(stream)), "pq_w4a4_linear")
 

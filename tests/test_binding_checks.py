@@ -82,7 +82,7 @@ def test_gemm_out_dtype_must_match_y(pq):
 
 
 class FakePlan:
-    D, g = 256, 128
+    D, g, Gx, Dx = 256, 128, 2, 256
     handle = None
 
 

@@ -76,6 +76,15 @@ def test_make_plan_validation_before_any_device_call(pq):
     with pytest.raises(pq.PQError) as e:
         pq.Plan("hadamard", 384, g=256)                   # D not a multiple of g
     assert e.value.status == pq.PQ_ERR_INVALID_ARG
+    # 8-bit outlier groups: rotation plans at g = 128, distinct groups below D/g
+    for kind, g, groups, status in (("smooth_hadamard", 128, [0], pq.PQ_ERR_UNSUPPORTED),
+                                    ("hadamard", 64, [0], pq.PQ_ERR_UNSUPPORTED),
+                                    ("hadamard", 128, [1, 1], pq.PQ_ERR_INVALID_ARG),
+                                    ("hadamard", 128, [2], pq.PQ_ERR_INVALID_ARG),
+                                    ("hadamard", 128, [-1], pq.PQ_ERR_INVALID_ARG)):
+        with pytest.raises(pq.PQError) as e:
+            pq.Plan(kind, 256, g=g, groups8=groups)
+        assert e.value.status == status, (kind, g, groups)
     with pytest.raises(pq.PQError) as e:
         pq.Plan("hadamard", 256, flags=pq.PQ_FLAG_SMOOTH_AFTER_ROTATE)
     assert e.value.status == pq.PQ_ERR_INVALID_ARG
