@@ -53,8 +53,10 @@ constexpr size_t kSrSmemBytes = sizeof(SrSmem) + 1024;
 // loaded with the 128-byte swizzle: chunk index XOR (row mod 8).
 __device__ __forceinline__ uint32_t sr_chunk(int r, int j) { return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4)); }
 
+// The mode is a template parameter so that each mode's code is allocated registers on its own.
+template <int mode>
 __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
-    const __grid_constant__ CUtensorMap tmX, int64_t rows, int G, int64_t num_tiles, int mode,
+    const __grid_constant__ CUtensorMap tmX, int64_t rows, int G, int64_t num_tiles,
     const float* __restrict__ vec, uint8_t* __restrict__ codes, float* __restrict__ scales,
     float* __restrict__ smooth_out, unsigned int* status) {
   extern __shared__ unsigned char smem_raw[];
@@ -101,7 +103,7 @@ __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!__syncthreads_and(ok)) break;
 
-    if (mode == SR_COLMAX) {
+    if constexpr (mode == SR_COLMAX) {
       // Thread (slot r0, chunk c) takes the maximum of |x| over rows 16 r0 .. 16 r0 + 15 for the
       // 8 channels of chunk c; |bf16| is compared as an unsigned 16-bit integer (exact).
       const int r0 = t >> 4, c = t & 15, kb = c >> 3, j = c & 7;
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
         if (smooth_out)
           *reinterpret_cast<float2*>(smooth_out + (int64_t)rb * D + gi * 128 + 2 * t) = make_float2(sa, sb);
       }
-    } else if (mode != SR_NONE) {
+    } else if constexpr (mode != SR_NONE) {
       S.mul[t] = __ldg(vec + (int64_t)gi * 128 + t);
     }
 
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
     __syncthreads();   // every row (and column) of stage s is read; S.mul is complete
     if (t == 0 && tile + 2 * stride < num_tiles) issue(tile + 2 * stride, s);
 
-    if (mode == SR_COLMAX || mode == SR_PRE) {
+    if constexpr (mode == SR_COLMAX || mode == SR_PRE) {
 #pragma unroll
       for (int i = 0; i < 128; i += 4) {
         const float4 f = *reinterpret_cast<const float4*>(&S.mul[i]);
@@ -155,7 +157,7 @@ __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
       }
     }
     row_fwht128(v);
-    if (mode == SR_POST) {
+    if constexpr (mode == SR_POST) {
 #pragma unroll
       for (int i = 0; i < 128; i += 4) {
         const float4 f = *reinterpret_cast<const float4*>(&S.mul[i]);
@@ -191,20 +193,19 @@ __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
 
 }  // namespace
 
-cudaError_t launch_smooth_rows(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int mode,
-                               const float* vec, uint8_t* codes, float* scales, float* smooth_out,
-                               cudaStream_t stream) {
-  if (rows <= 0) return cudaSuccess;
-  CUtensorMap tmX;
-  cudaError_t e = make_bf16_tile_map(&tmX, X, rows, plan->D, ldx);
-  if (e != cudaSuccess) return e;
+namespace {
+
+template <int mode>
+cudaError_t launch_smooth_rows_mode(const pq_plan* plan, const CUtensorMap& tmX, int64_t rows, const float* vec,
+                                    uint8_t* codes, float* scales, float* smooth_out, cudaStream_t stream) {
   static std::atomic<bool> attr_done[kMaxDevices];
-  e = set_kernel_attributes(reinterpret_cast<const void*>(smooth_rows_kernel), (int)kSrSmemBytes, attr_done);
+  cudaError_t e = set_kernel_attributes(reinterpret_cast<const void*>(smooth_rows_kernel<mode>), (int)kSrSmemBytes,
+                                        attr_done);
   if (e != cudaSuccess) return e;
   static std::atomic<int> per_sm_cache{0};
   int per_sm = per_sm_cache.load(std::memory_order_relaxed);
   if (per_sm < 1) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, smooth_rows_kernel, SR_ROWS, kSrSmemBytes) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, smooth_rows_kernel<mode>, SR_ROWS, kSrSmemBytes) !=
             cudaSuccess || per_sm < 1)
       per_sm = 1;
     per_sm_cache.store(per_sm, std::memory_order_relaxed);
@@ -213,9 +214,26 @@ cudaError_t launch_smooth_rows(const pq_plan* plan, const void* X, int64_t rows,
   const int64_t tiles = row_blocks * plan->G;
   const int64_t cap = (int64_t)device_sm_count() * per_sm;
   const int grid = (int)(tiles < cap ? tiles : cap);
-  smooth_rows_kernel<<<grid, SR_ROWS, kSrSmemBytes, stream>>>(tmX, rows, plan->G, tiles, mode, vec, codes, scales,
-                                                              smooth_out, plan->d_status);
+  smooth_rows_kernel<mode><<<grid, SR_ROWS, kSrSmemBytes, stream>>>(tmX, rows, plan->G, tiles, vec, codes, scales,
+                                                                    smooth_out, plan->d_status);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_smooth_rows(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int mode,
+                               const float* vec, uint8_t* codes, float* scales, float* smooth_out,
+                               cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  CUtensorMap tmX;
+  cudaError_t e = make_bf16_tile_map(&tmX, X, rows, plan->D, ldx);
+  if (e != cudaSuccess) return e;
+  switch (mode) {
+    case SR_COLMAX: return launch_smooth_rows_mode<SR_COLMAX>(plan, tmX, rows, vec, codes, scales, smooth_out, stream);
+    case SR_PRE: return launch_smooth_rows_mode<SR_PRE>(plan, tmX, rows, vec, codes, scales, smooth_out, stream);
+    case SR_POST: return launch_smooth_rows_mode<SR_POST>(plan, tmX, rows, vec, codes, scales, smooth_out, stream);
+    default: return launch_smooth_rows_mode<SR_NONE>(plan, tmX, rows, vec, codes, scales, smooth_out, stream);
+  }
 }
 
 }  // namespace pq
