@@ -655,7 +655,7 @@ cudaError_t scratch_pool(cudaMemPool_t* out) {
 }
 
 // CTA pairs (clusters of 2) of w4a4_gemm_kernel resident at once on the current device: one
-// per SM pair when every pair can host one.  Needs the kernel's shared-memory attribute set.
+// per SM pair when every pair can host one.
 pq_status gemm_max_pairs(int sms, int* out) {
   static std::atomic<int> cache[kMaxDevices];
   int dev = 0;
@@ -664,6 +664,12 @@ pq_status gemm_max_pairs(int sms, int* out) {
   const bool slot = dev >= 0 && dev < kMaxDevices;
   int n = slot ? cache[dev].load(std::memory_order_relaxed) : 0;
   if (n < 1) {
+    // Every instantiation has the same block and shared memory, so one stands for all; its
+    // shared-memory limit must be raised before the occupancy is asked (whichever instantiation
+    // the caller is about to launch).
+    static std::atomic<bool> attr_done[kMaxDevices];
+    e = set_kernel_attributes(reinterpret_cast<const void*>(w4a4_gemm_kernel<false, 4>), (int)kSmemBytes, attr_done);
+    if (e != cudaSuccess) return cuda_fail(e, "w4a4_gemm_kernel attributes");
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);

@@ -35,6 +35,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "rows.cuh"
 
 namespace pq {
 namespace {
@@ -302,8 +303,10 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
           uint32_t r[32];
           ptx::tmem_ld32(ta + 32 * c, r);
           ptx::tmem_ld_wait();
+          float f[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(__uint_as_float(r[j])));
+          for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(r[j]);
+          m = fmaxf(m, row_absmax<32>(f));
         }
         const float inv = m > 0.0f ? 7.0f * __frcp_rn(m) : 0.0f;
         uint4* dst = reinterpret_cast<uint4*>(codes + t * (int64_t)G * 128 + gi * 128);
@@ -335,9 +338,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&S.acc_empty[b]);
-      float m = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 128; ++i) m = fmaxf(m, fabsf(y[i]));
+      const float m = row_absmax<128>(y);
       if constexpr (kColMax) {
         // this thread's lane is output channel rl of group gi; its columns are the tile's rows
         atomicMax(chan_max + (int64_t)gi * 128 + rl, __float_as_uint(m * scale_mult));
@@ -345,9 +346,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1) rotate_mma_kernel(
       }
       if constexpr (GW == 64) {
         // two groups per tile: channels 0..63 and 64..127 of the row, one maximum each
-        float mh[2] = {0.0f, 0.0f};
-#pragma unroll
-        for (int i = 0; i < 128; ++i) mh[i >> 6] = fmaxf(mh[i >> 6], fabsf(y[i]));
+        const float mh[2] = {row_absmax<64>(y), row_absmax<64>(y + 64)};
         if (t < rows) {
           uint4* dst = reinterpret_cast<uint4*>(codes + t * (int64_t)G * 32 + gi * 64);
 #pragma unroll

@@ -66,6 +66,23 @@ __device__ __forceinline__ void row_fwht32(float (&v)[32]) {
   }
 }
 
+// max |v[i]| over N register values (N a multiple of 8) with eight independent partial maxima,
+// so the dependency chain is N/8 + 3 long instead of N; the maximum is exact in any order.
+template <int N>
+__device__ __forceinline__ float row_absmax(const float* v) {
+  static_assert(N % 8 == 0 && N >= 8, "N must be a positive multiple of 8");
+  float m[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = fabsf(v[k]);
+#pragma unroll
+  for (int i = 8; i < N; ++i) m[i & 7] = fmaxf(m[i & 7], fabsf(v[i]));
+#pragma unroll
+  for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+    for (int k = 0; k < w; ++k) m[k] = fmaxf(m[k], m[k + w]);
+  return m[0];
+}
+
 // 8 values -> 8 nibbles: byte k = q[2k] | q[2k+1] << 4, q = RNE(v * inv) (|q| <= 7); the FMA with
 // 1.5 * 2^23 leaves q's two's-complement low bits in the low byte.
 __device__ __forceinline__ uint32_t row_pack8(const float* v, float inv) {

@@ -228,17 +228,14 @@ __global__ void __launch_bounds__(RR_MAX_THREADS, 1) rrs_rows_kernel(
     }
     uint8_t* crow = codes + row * (int64_t)(D / 2);
     if (MODE == 0) {
-      float m = 0.0f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int c = p + i * RT;
         const float is = c < chunks8 ? inv_s[c >> 4] : 0.0f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          v[8 * i + e] *= is;
-          m = fmaxf(m, fabsf(v[8 * i + e]));
-        }
+        for (int e = 0; e < 8; ++e) v[8 * i + e] *= is;
       }
+      float m = row_absmax<32>(v);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       const int wr = RT / 32;                      // warps per row
@@ -260,9 +257,7 @@ __global__ void __launch_bounds__(RR_MAX_THREADS, 1) rrs_rows_kernel(
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int c = p + i * RT;
-        float m = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[8 * i + e]));
+        float m = row_absmax<8>(v + 8 * i);
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         const float inv = m > 0.0f ? 7.0f * __frcp_rn(m) : 0.0f;

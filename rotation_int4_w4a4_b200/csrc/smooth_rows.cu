@@ -167,9 +167,7 @@ __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
         v[i + 3] *= f.w;
       }
     }
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 128; ++i) m = fmaxf(m, fabsf(v[i]));
+    const float m = row_absmax<128>(v);
     const float inv = m > 0.0f ? 7.0f * __frcp_rn(m) : 0.0f;
     const int64_t row = (int64_t)rb * SR_ROWS + t;
     if (row < rows) {

@@ -17,6 +17,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "rows.cuh"
 
 namespace pq {
 namespace {
@@ -85,12 +86,7 @@ __device__ __forceinline__ void fwht_across4(float (&v)[32], int lane) {
   }
 }
 
-__device__ __forceinline__ float absmax32(const float (&v)[32]) {
-  float m = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
-  return m;
-}
+__device__ __forceinline__ float absmax32(const float (&v)[32]) { return row_absmax<32>(v); }
 
 __device__ __forceinline__ float group_max4(float m) {
   m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));

@@ -183,3 +183,31 @@ def test_chain_matches_oracle_chain(pq, kind, g, T):
     own = oracle.gemm(ca.cpu().numpy(), sa.cpu().numpy(), cw.cpu().numpy(), sw.cpu().numpy(), g).y64
     assert rel_fro(got, own) < 1e-5
     assert rel_fro(got, ref) < 1e-2
+
+
+@pytest.mark.parametrize("first", ["g64", "g256", "rrs"])
+def test_first_pair_gemm_of_a_process(first):
+    """The CTA-pair GEMM's occupancy query must hold whichever instantiation a process launches
+    first (g = 64 or 256, or the row-scale variant): run each alone in a fresh process."""
+    import subprocess
+    import sys
+    code = f"""
+import numpy as np, torch
+from rotation_int4_w4a4_b200 import pq, inputs
+g = {{'g64': 64, 'g256': 256, 'rrs': 128}}['{first}']
+T, N, D = 200, 256, 512
+ca, sa = inputs.random_codes(1, T, D, g)
+cw, sw = inputs.random_codes(2, N, D, g)
+Y = torch.empty((T, N), dtype=torch.float32, device='cuda')
+dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+if '{first}' == 'rrs':
+    pq.pq_rrs_gemm(dev(ca), dev(sa[:, 0].copy()), dev(cw), dev(sw), Y)
+else:
+    pq.pq_w4a4_gemm(dev(ca), dev(sa), dev(cw), dev(sw), Y, g=g)
+pq.pq_check_status()
+print('ok')
+"""
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=root, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stderr[-2000:]
