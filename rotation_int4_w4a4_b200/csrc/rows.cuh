@@ -84,11 +84,18 @@ __device__ __forceinline__ float row_absmax(const float* v) {
 }
 
 // 8 values -> 8 nibbles: byte k = q[2k] | q[2k+1] << 4, q = RNE(v * inv) (|q| <= 7); the FMA with
-// 1.5 * 2^23 leaves q's two's-complement low bits in the low byte.
+// 1.5 * 2^23 leaves q's two's-complement low bits in the low byte (packed-pair FMAs, the same
+// float32 operation on each value).
 __device__ __forceinline__ uint32_t row_pack8(const float* v, float inv) {
   uint32_t b[8];
+  const uint64_t inv2 = ptx::f2_pack(inv, inv), magic2 = ptx::f2_pack(kRowRoundMagic, kRowRoundMagic);
 #pragma unroll
-  for (int k = 0; k < 8; ++k) b[k] = __float_as_uint(fmaf(v[k], inv, kRowRoundMagic));
+  for (int k = 0; k < 8; k += 2) {
+    float lo, hi;
+    ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(v[k], v[k + 1]), inv2, magic2), lo, hi);
+    b[k] = __float_as_uint(lo);
+    b[k + 1] = __float_as_uint(hi);
+  }
   const uint32_t even = __byte_perm(__byte_perm(b[0], b[2], 0x0040), __byte_perm(b[4], b[6], 0x0040), 0x5410);
   const uint32_t odd = __byte_perm(__byte_perm(b[1], b[3], 0x0040), __byte_perm(b[5], b[7], 0x0040), 0x5410);
   return (even & 0x0F0F0F0Fu) | ((odd << 4) & 0xF0F0F0F0u);

@@ -150,10 +150,8 @@ __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
 #pragma unroll
       for (int i = 0; i < 128; i += 4) {
         const float4 f = *reinterpret_cast<const float4*>(&S.mul[i]);
-        v[i] *= f.x;
-        v[i + 1] *= f.y;
-        v[i + 2] *= f.z;
-        v[i + 3] *= f.w;
+        ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(v[i], v[i + 1]), ptx::f2_pack(f.x, f.y)), v[i], v[i + 1]);
+        ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(v[i + 2], v[i + 3]), ptx::f2_pack(f.z, f.w)), v[i + 2], v[i + 3]);
       }
     }
     row_fwht128(v);
