@@ -679,10 +679,14 @@ def measure_decode(args, dev, stream, peaks, peak_src):
                 time_calls(lambda k: calls, flush, max(3, args.warmup), stream)
                 per = time_calls(lambda k: calls, flush, steps, stream)
                 res[name] = 1e3 * statistics.mean(sum(p) for p in per)
+                if name == "separate":
+                    res["transform"] = 1e3 * statistics.mean(p[0] for p in per)
+                    res["gemm"] = 1e3 * statistics.mean(p[1] for p in per)
             pq.pq_check_status(plan)
             nbytes = T * D * 2 + T * N * 4 + N * D / 2 + N * G * 4
             out[f"T{T}_N{N}"] = {
                 "us_separate": res["separate"], "us_linear": res["linear"],
+                "us_transform": res["transform"], "us_gemm": res["gemm"],
                 "bytes": nbytes, "GB_s_linear": nbytes / (res["linear"] * 1e-6) / 1e9,
                 "frac_hbm_linear": nbytes / (res["linear"] * 1e-6) / 1e9 / peaks["hbm_gbs"]}
             plan.close()

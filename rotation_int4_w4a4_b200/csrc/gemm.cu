@@ -480,6 +480,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1) w4a4
   GemmSmem& S = *reinterpret_cast<GemmSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // The split-K reduction, launched as this grid's programmatic dependent, may start now (it
+  // waits for this grid before reading).
+  ptx::griddep_launch_dependents();
   Work wk;
   wk.m_tiles = m_tiles;
   wk.n_tiles = n_tiles;
@@ -548,8 +551,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1) w4a4
 }
 
 // Split-K reduction: Y = sum over kr of ws[kr] (ascending), float32 or bf16 (RNE) out.
+// Launched as the programmatic dependent of the kernel that writes the partial tiles: it may start
+// while that kernel runs and waits for its completion before reading them.
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __restrict__ ws, int ksplit, int64_t n4,
                                                             void* __restrict__ Y, int out_bf16) {
+  ptx::griddep_wait();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
     float4 a = ws[i];
@@ -753,8 +759,20 @@ pq_status launch_splitk_reduce(const float* ws, int ksplit, int64_t T, int64_t N
   const int64_t rwant = (n4 + 255) / 256;
   const int64_t cap = (int64_t)device_sm_count() * 8;
   const int rgrid = (int)(rwant < cap ? rwant : cap);
-  splitk_reduce_kernel<<<rgrid, 256, 0, stream>>>(reinterpret_cast<const float4*>(ws), ksplit, n4, Y, out_bf16);
-  return cuda_fail(cudaGetLastError(), "splitk_reduce_kernel launch");
+  // Programmatic dependent of the GEMM kernel just launched on `stream` (which releases its
+  // dependents at its start), so the launch overlaps the GEMM; the kernel waits before reading.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)rgrid, 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cuda_fail(cudaLaunchKernelEx(&cfg, splitk_reduce_kernel, reinterpret_cast<const float4*>(ws), ksplit, n4, Y,
+                                      out_bf16),
+                   "splitk_reduce_kernel launch");
 }
 
 pq_status gemm_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W, const float* scales_W,

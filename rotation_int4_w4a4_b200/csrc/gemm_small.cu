@@ -177,6 +177,7 @@ __global__ void __launch_bounds__(GS_THREADS, 1) w4a4_gemm_small_kernel(
   // stage is one K-block and a packed-code stage four.  Group ranges start on K-block boundaries.
   using Smem = SmallSmem<NT>;
   constexpr int gsl = GSL;
+  ptx::griddep_launch_dependents();   // the range reduction may launch now; it waits for this grid
   const int g64 = GSL == 2 ? 1 : 0;
   constexpr int RAW = Smem::RAW, GS_OPS = Smem::OPS, GS_NACC = Smem::NACC;
   constexpr uint32_t kTmemCols = GS_NACC * NT < 32 ? 32 : GS_NACC * NT;
@@ -489,13 +490,13 @@ static_assert(small_smem_bytes<16>() <= 232448 && small_smem_bytes<32>() <= 2324
 
 // Group ranges per 128-row weight tile: as many as keep every unit in one wave over the SMs (a
 // second, partial wave would double the time of the CTAs that run it), and only while the
-// float32 partial tiles (written and read back, 8 T N bytes per range) stay within a quarter of
-// the packed weight bytes (N D / 2).  A range is a multiple of 4 groups (one packed-code stage).
+// float32 partial tiles of the ranges (written and read back, 8 T N bytes per range, mostly in
+// L2) stay within the packed weight bytes (N D / 2).  A range is a multiple of 4 groups.
 int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int g, int* gs_out) {
   const int G = (int)(D / g);
   const int64_t m_tiles = (N + GS_M - 1) / GS_M;
   const int64_t fill = device_sm_count() / m_tiles;
-  const int64_t traffic = std::max<int64_t>(1, D / (64 * T));
+  const int64_t traffic = std::max<int64_t>(1, D / (16 * T));
   int r = (int)std::max<int64_t>(1, std::min<int64_t>({fill, traffic, (int64_t)((G + GS_GPS - 1) / GS_GPS)}));
   int gs = (G + r - 1) / r;
   gs = (gs + GS_GPS - 1) / GS_GPS * GS_GPS;

@@ -83,5 +83,5 @@ def test_job_value_is_weak_scaling():
     assert bench.launches_per_step(256, 4096, 4096) == 5       # 16 pair tiles: split-K + reduce
     assert bench.launches_per_step(1, 4096, 4096) == 4         # few tokens: group ranges + reduce
     assert bench.launches_per_step(16, 14336, 4096) == 3       # few tokens, 112 tiles: one launch
-    assert bench.launches_per_step(64, 4096, 4096) == 3        # few tokens, one launch
+    assert bench.launches_per_step(64, 4096, 4096) == 4        # few tokens: ranges + reduce
     assert bench.launches_per_step(1, 272, 4096) == 4          # ragged N: ranges + reduce

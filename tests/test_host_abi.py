@@ -150,9 +150,11 @@ def test_gemm_launch_count_query(pq):
     assert pq.pq_w4a4_gemm_launch_count(1, 4096, 4096) == 2
     assert pq.pq_w4a4_gemm_launch_count(1, 4096, 512) == 1        # 4 groups: one range (one stage)
     assert pq.pq_w4a4_gemm_launch_count(1, 14336, 4096) == 1      # 112 tiles: one wave unsplit
-    # 64 and 128 tokens: partial tiles would outweigh the weights, so one launch writes Y
-    assert pq.pq_w4a4_gemm_launch_count(64, 4096, 4096) == 1
+    # 64 tokens: four ranges (the partial tiles stay below the weight bytes); 128 tokens at
+    # N = 14336: 112 weight tiles fill one wave, one launch writes Y
+    assert pq.pq_w4a4_gemm_launch_count(64, 4096, 4096) == 2
     assert pq.pq_w4a4_gemm_launch_count(128, 14336, 4096) == 1
+    assert pq.pq_w4a4_gemm_launch_count(128, 4096, 4096) == 2
     # other group sizes: the same kernels, split by groups of g (ranges of 4 groups)
     for g in (64, 128, 256):
         assert pq.pq_w4a4_gemm_launch_count_g(4096, 14336, 4096, g) == 2
