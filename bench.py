@@ -49,7 +49,8 @@ DECODE_T_MAX = 128
 # Kernel sources whose DRAM counters profiles/traffic.json records; a change to any of them
 # makes the recorded traffic stale (reported as null).
 KERNEL_SOURCES = tuple("rotation_int4_w4a4_b200/csrc/" + f for f in (
-    "gemm.cu", "gemm_small.cu", "ptx.cuh", "rotate_mma.cu", "transform.cu", "smooth_rows.cu", "rows.cuh", "rrs.cu"))
+    "gemm.cu", "gemm_small.cu", "ptx.cuh", "rotate_mma.cu", "transform.cu", "smooth_rows.cu", "rows.cuh", "rrs.cu",
+    "rows_small.cu"))
 
 
 def load_peaks():

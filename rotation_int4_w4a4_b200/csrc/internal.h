@@ -147,6 +147,12 @@ cudaError_t launch_smooth_hadamard(const pq_plan* plan, const void* X, int64_t T
 // nothing is quantised: chan_max[j] becomes max over the rows of |y[:, j]| (normalised rotation).
 cudaError_t launch_rotate_mma(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, int weights,
                               uint8_t* codes, float* scales, cudaStream_t stream, unsigned int* chan_max = nullptr);
+// Activation transforms of at most this many rows (Hadamard or Givens, g = 64 or 128, no 8-bit
+// groups) run one warp per (row, 128-channel tile) on the CUDA cores (rows_small.cu).
+constexpr int64_t kRowsSmallT = 16;
+bool rows_small_applies(const pq_plan* plan, int64_t rows);
+cudaError_t launch_rows_small(const pq_plan* plan, const void* X, int64_t rows, int64_t ldx, uint8_t* codes,
+                              float* scales, cudaStream_t stream);
 // Calls with at most this many tokens take the few-token kernel (gemm_small.cu): packed codes
 // read directly, int8 tensor-core products, no operand scratch.
 constexpr int64_t kGemmSmallT = 128;

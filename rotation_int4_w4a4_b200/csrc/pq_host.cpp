@@ -366,6 +366,7 @@ cudaError_t launch_transform(const pq_plan* plan, const void* X, int64_t T, int6
   switch (plan->kind) {
     case PQ_HADAMARD:
     case PQ_GIVENS:
+      if (rows_small_applies(plan, T)) return launch_rows_small(plan, X, T, ldx, codes, scales, s);
       return launch_rotate_mma(plan, X, T, ldx, 0, codes, scales, s);
     case PQ_SMOOTH_HADAMARD:
       if (plan->flags & PQ_FLAG_SMOOTH_AFTER_ROTATE)

@@ -240,3 +240,27 @@ def test_pack_weights_full_size_sampled(pq, name):
     assert_codes_match(codes[rt].cpu().numpy(), ref)
     assert_scales_close(scales[rt].cpu().numpy(), ref.scales,
                         RTOL_G if wl.kind == "givens" else 2 * RTOL_H)
+
+
+# ------------------------------------------------------------ few rows (CUDA-core path)
+@pytest.mark.parametrize("kind", ["hadamard", "givens"])
+@pytest.mark.parametrize("T", [1, 2, 7, 16, 17])
+def test_few_rows(pq, kind, T):
+    """Up to 16 rows take the warp-per-tile kernel (shuffle butterflies for Hadamard, the composed
+    matrix from L2 for Givens); 17 rows the tensor-core kernel.  Both against the oracle, with the
+    up_proj Givens plan (K = 16) and the q_proj Hadamard plan."""
+    name = "up_proj" if kind == "givens" else "q_proj"
+    wl = inputs.workload(name, T=T)
+    if kind == "givens":
+        pairs, angles, beta = givens_inputs(wl)
+        plan = pq.Plan("givens", wl.D, K=wl.K, pairs=pairs, angles=angles, beta=beta)
+        oplan = oracle_plan("givens", wl.D, wl.K, pairs, angles, beta)
+        rtol = RTOL_G
+    else:
+        plan = pq.Plan("hadamard", wl.D)
+        oplan = oracle_plan("hadamard", wl.D)
+        rtol = RTOL_H
+    codes, scales, _ = run_tq(pq, plan, wl.X, wl.D, ldx=wl.D + 64)
+    ref = oracle.transform_quant(wl.X, oplan)
+    assert_codes_match(codes, ref)
+    assert_scales_close(scales, ref.scales, rtol)
