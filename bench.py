@@ -50,7 +50,7 @@ DECODE_T_MAX = 128
 # makes the recorded traffic stale (reported as null).
 KERNEL_SOURCES = tuple("rotation_int4_w4a4_b200/csrc/" + f for f in (
     "gemm.cu", "gemm_small.cu", "ptx.cuh", "rotate_mma.cu", "transform.cu", "smooth_rows.cu", "rows.cuh", "rrs.cu",
-    "rows_small.cu"))
+    "rows_small.cu", "gemv.cu"))
 
 
 def load_peaks():
@@ -660,7 +660,7 @@ def measure_decode(args, dev, stream, peaks, peak_src):
     flush = L2Flush(dev)
     out = {}
     for N in (4096, 14336):
-        for T in (1, 16, 64):
+        for T in (1, 4, 8, 16, 64):
             wl = inputs.workload("sweep", T=T, N=N)
             D, G = wl.D, wl.D // wl.g
             plan = pq.Plan("hadamard", D)

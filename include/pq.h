@@ -202,13 +202,17 @@ pq_status pq_pack_weights(const pq_plan* plan, const void* W, int64_t N, const f
  *   pairs): the groups are split into ranges of a multiple of 4 handled by different SM pairs,
  *   and the float32 partial results are added in ascending range order (4 * ranges * T * N
  *   extra scratch bytes).
- *   T <= 128 (decode): the packed codes are read directly (no operand scratch) and widened to
- *   int8 q * 16 inside the kernel; tcgen05.mma kind::i8 forms 256 d_G exactly in int32 and the
- *   epilogue applies sw / 256 (exact) and sa, giving the same per-group float32 values.  One
- *   kernel writes Y, unless the 128-row weight tiles are too few to fill the device: then the
- *   groups are split into ranges and their float32 partial tiles (4 * ranges * T * N scratch
- *   bytes) are added in ascending range order by a second kernel.
- *   A split result differs from the unsplit order only by float32 rounding.
+ *   4 < T <= 128 (decode batches): the packed codes are read directly (no operand scratch) and
+ *   widened to int8 q * 16 inside the kernel; tcgen05.mma kind::i8 forms 256 d_G exactly in
+ *   int32 and the epilogue applies sw / 256 (exact) and sa, giving the same per-group float32
+ *   values.  One kernel writes Y, unless the 128-row weight tiles are too few to fill the
+ *   device: then the groups are split into ranges and their float32 partial tiles
+ *   (4 * ranges * T * N scratch bytes) are added in ascending range order by a second kernel.
+ *   T <= 4 (single-token decode): one kernel on the CUDA cores, no scratch: the weights stream
+ *   through registers, __dp4a on q * 16 operands forms 256 d_G exactly in int32, the same
+ *   per-group term fl(d_G * sw) * sa is accumulated, and the groups' terms are added in an
+ *   order of the kernel's own (ascending per lane, then a tree over lanes).
+ *   A split or reordered sum differs from the ascending order only by float32 rounding.
  */
 pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W,
                        const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
@@ -221,8 +225,9 @@ pq_status pq_w4a4_gemm(const uint8_t* codes_A, const float* scales_A, const uint
  *   pq_transform_quant(plan, X, T, ldx, codes_A, scales_A, NULL) followed by
  *   pq_w4a4_gemm(codes_A, scales_A, codes_W, scales_W, T, N, plan->D, plan->g, Y, out_dtype).
  *   T <= 128: the GEMM is launched as a programmatic dependent of the transform: its prologue
- *   and its weight-side loads start while the transform runs, and it reads codes_A and scales_A
- *   only after the transform has completed.  T > 128: the two run one after the other.
+ *   and its weight-side loads start while the transform runs (T <= 4: the first 2 KB of each
+ *   weight row), and it reads codes_A and scales_A only after the transform has completed.
+ *   T > 128: the two run one after the other.
  *   codes_A [T][D/2] and scales_A [T][D/g] are caller-owned device buffers and are written (the
  *   activation codes stay available; with 8-bit outlier groups D is the plan's Gx * g and D/g its
  *   Gx, for codes_W and scales_W too).  codes_W and scales_W must be complete when the call is
@@ -322,7 +327,7 @@ pq_status pq_w4a4_gemm_noalloc(const uint8_t* codes_A, const float* scales_A,
  * *launches the number of kernels one pq_w4a4_gemm call with these sizes and g = 128 launches
  * on the current device (pq_w4a4_gemm_launch_count_g: the same for group size g).  T > 128: 2 (operand expansion, contraction) or 3 (plus the split-K
  * reduction, chosen when the 256 x 256 output tiles fill at most half of the device's SM
- * pairs).  T <= 128: 1, or 2 with the group-range reduction.  pq_w4a4_gemm_noalloc never
+ * pairs).  4 < T <= 128: 1, or 2 with the group-range reduction.  T <= 4: 1.  pq_w4a4_gemm_noalloc never
  * splits: it launches 2 for T > 128 and 1 otherwise.  Sizes are validated as for
  * pq_w4a4_gemm (PQ_ERR_INVALID_ARG otherwise).  Without a usable device the count assumes 148 SMs.
  */

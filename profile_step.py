@@ -1,6 +1,6 @@
 """Run one workload's hot-path step a few times through the library, for profilers.
 
-    python profile_step.py [--workload q_proj] [--repeat 3] [--rrs]
+    python profile_step.py [--workload q_proj] [--T tokens] [--N rows] [--repeat 3] [--rrs]
 
 Each repetition launches, in order, the activation transform (pq_transform_quant), the weight
 transform (pq_pack_weights) and the W4A4 GEMM (pq_w4a4_gemm) on the named synthetic workload,
@@ -31,10 +31,11 @@ def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="q_proj")
     ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--N", type=int, default=None)
     ap.add_argument("--repeat", type=int, default=3)
     ap.add_argument("--rrs", action="store_true")
     args = ap.parse_args()
-    wl = inputs.workload(args.workload, T=args.T)
+    wl = inputs.workload(args.workload, T=args.T, N=args.N)
     dev = torch.device("cuda")
 
     def bf16(bits):

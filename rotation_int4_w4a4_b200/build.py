@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libpq.so")
 OBJDIR = os.path.join(ROOT, "_build")
-SOURCES = ["pq_host.cpp", "transform.cu", "smooth_rows.cu", "rotate_mma.cu", "gemm.cu", "gemm_small.cu", "rrs.cu", "rows_small.cu", "gemm_static_scratch.cu"]
+SOURCES = ["pq_host.cpp", "transform.cu", "smooth_rows.cu", "rotate_mma.cu", "gemm.cu", "gemm_small.cu", "gemv.cu", "rrs.cu", "rows_small.cu", "gemm_static_scratch.cu"]
 HEADERS = ["internal.h", "ptx.cuh", "rows.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-O2,-Wall",

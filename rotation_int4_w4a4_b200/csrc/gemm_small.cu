@@ -1,4 +1,5 @@
-// W4A4 GEMM for few tokens (T <= 128, the decode regime) on tcgen05 tensor cores (sm_100a).
+// W4A4 GEMM for few tokens (4 < T <= 128; at most 4 tokens take the CUDA-core kernel of gemv.cu) on
+// tcgen05 tensor cores (sm_100a).
 //
 // Y[t][n] = sum_G sa[t][G] * sw[n][G] * d_G[t][n] (RRS page, main equation, last line; Fig. 4
 // step (3) with block size = group size), as in gemm.cu, for calls whose cost is streaming the
@@ -494,6 +495,10 @@ static_assert(small_smem_bytes<16>() <= 232448 && small_smem_bytes<32>() <= 2324
 // L2) stay within the packed weight bytes (N D / 2).  A range is a multiple of 4 groups.
 int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int g, int* gs_out) {
   const int G = (int)(D / g);
+  if (T <= kGemvT) {            // the CUDA-core kernel: one launch over all groups
+    if (gs_out) *gs_out = G;
+    return 1;
+  }
   const int64_t m_tiles = (N + GS_M - 1) / GS_M;
   const int64_t fill = device_sm_count() / m_tiles;
   const int64_t traffic = std::max<int64_t>(1, D / (16 * T));
@@ -510,6 +515,8 @@ pq_status gemm_small_launch(const uint8_t* codes_A, const float* scales_A, const
                             const float* scales_W, int64_t T, int64_t N, int64_t D, int g, void* Y,
                             pq_out_dtype out_dtype, float* ws, unsigned int* status, cudaStream_t stream,
                             bool row_scale, bool pdl) {
+  if (T <= kGemvT)
+    return gemv_launch(codes_A, scales_A, codes_W, scales_W, T, N, D, g, Y, out_dtype, stream, row_scale, pdl);
   const int NT = T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128;
   const int G = (int)(D / g), gsl = g / 32;
   int gs = G;

@@ -156,6 +156,12 @@ cudaError_t launch_rows_small(const pq_plan* plan, const void* X, int64_t rows, 
 // Calls with at most this many tokens take the few-token kernel (gemm_small.cu): packed codes
 // read directly, int8 tensor-core products, no operand scratch.
 constexpr int64_t kGemmSmallT = 128;
+// Calls with at most this many tokens take the CUDA-core kernel (gemv.cu) instead: weights
+// streamed into registers, __dp4a products, one launch, no workspace.
+constexpr int64_t kGemvT = 4;
+pq_status gemv_launch(const uint8_t* codes_A, const float* scales_A, const uint8_t* codes_W, const float* scales_W,
+                      int64_t T, int64_t N, int64_t D, int g, void* Y, pq_out_dtype out_dtype, cudaStream_t stream,
+                      bool row_scale, bool pdl);
 // Group ranges per 128-row weight tile of the few-token kernel (1 = no split); g = group size.
 int gemm_small_ranges(int64_t T, int64_t N, int64_t D, int g, int* gs_out);
 // The few-token GEMM (+ the split reduction when ws != nullptr and the sizes call for it).

@@ -81,7 +81,9 @@ def test_job_value_is_weak_scaling():
     # No GPU here: the library counts with B200's 148 SMs (74 SM pairs).
     assert bench.launches_per_step(2048, 4096, 4096) == 4      # 128 pair tiles: no split
     assert bench.launches_per_step(256, 4096, 4096) == 5       # 16 pair tiles: split-K + reduce
-    assert bench.launches_per_step(1, 4096, 4096) == 4         # few tokens: group ranges + reduce
-    assert bench.launches_per_step(16, 14336, 4096) == 3       # few tokens, 112 tiles: one launch
+    assert bench.launches_per_step(1, 4096, 4096) == 3         # at most 4 tokens: CUDA-core kernel
+    assert bench.launches_per_step(4, 14336, 4096) == 3
+    assert bench.launches_per_step(16, 4096, 4096) == 4        # few tokens: group ranges + reduce
+    assert bench.launches_per_step(17, 14336, 4096) == 3       # few tokens, 112 tiles: one launch
     assert bench.launches_per_step(64, 4096, 4096) == 4        # few tokens: ranges + reduce
-    assert bench.launches_per_step(1, 272, 4096) == 4          # ragged N: ranges + reduce
+    assert bench.launches_per_step(17, 272, 4096) == 4         # ragged N: ranges + reduce

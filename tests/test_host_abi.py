@@ -134,7 +134,8 @@ def test_selftest_wait_timeout_validation(pq):
 def test_gemm_launch_count_query(pq):
     """Host-only query (no GPU here, so 148 SMs are assumed): sizes are validated as for the
     GEMM.  More than 128 tokens: 2 or 3 launches (operand expansion, contraction, split-K
-    reduction).  At most 128 tokens: 1, or 2 with the group-range reduction."""
+    reduction).  5 to 128 tokens: 1, or 2 with the group-range reduction.  At most 4 tokens:
+    the CUDA-core kernel, 1."""
     import ctypes
     L = pq.lib
     n = ctypes.c_int(-1)
@@ -146,10 +147,16 @@ def test_gemm_launch_count_query(pq):
     assert pq.pq_w4a4_gemm_launch_count(4096, 14336, 4096) == 2   # 896 pair tiles
     assert pq.pq_w4a4_gemm_launch_count(256, 4096, 4096) == 3     # 16 pair tiles, 32 groups
     assert pq.pq_w4a4_gemm_launch_count(129, 4096, 4096) == 3     # 129 tokens: CTA-pair kernel
-    # few tokens: 32 weight tiles of 128 rows -> 4 group ranges in one wave over 148 SMs
-    assert pq.pq_w4a4_gemm_launch_count(1, 4096, 4096) == 2
-    assert pq.pq_w4a4_gemm_launch_count(1, 4096, 512) == 1        # 4 groups: one range (one stage)
-    assert pq.pq_w4a4_gemm_launch_count(1, 14336, 4096) == 1      # 112 tiles: one wave unsplit
+    # at most 4 tokens: one CUDA-core launch whatever the shape
+    for T in (1, 2, 3, 4):
+        assert pq.pq_w4a4_gemm_launch_count(T, 4096, 4096) == 1
+        assert pq.pq_w4a4_gemm_launch_count(T, 14336, 4096) == 1
+        assert pq.pq_w4a4_gemm_launch_count(T, 16, 128) == 1
+    # 5 to 128 tokens: 32 weight tiles of 128 rows -> group ranges in one wave over 148 SMs
+    assert pq.pq_w4a4_gemm_launch_count(5, 4096, 4096) == 2
+    assert pq.pq_w4a4_gemm_launch_count(17, 4096, 4096) == 2
+    assert pq.pq_w4a4_gemm_launch_count(17, 4096, 512) == 1       # 4 groups: one range (one stage)
+    assert pq.pq_w4a4_gemm_launch_count(17, 14336, 4096) == 1     # 112 tiles: one wave unsplit
     # 64 tokens: four ranges (the partial tiles stay below the weight bytes); 128 tokens at
     # N = 14336: 112 weight tiles fill one wave, one launch writes Y
     assert pq.pq_w4a4_gemm_launch_count(64, 4096, 4096) == 2
@@ -158,10 +165,12 @@ def test_gemm_launch_count_query(pq):
     # other group sizes: the same kernels, split by groups of g (ranges of 4 groups)
     for g in (64, 128, 256):
         assert pq.pq_w4a4_gemm_launch_count_g(4096, 14336, 4096, g) == 2
-        assert pq.pq_w4a4_gemm_launch_count_g(1, 14336, 4096, g) == 1
-    assert pq.pq_w4a4_gemm_launch_count_g(1, 4096, 4096, 128) == pq.pq_w4a4_gemm_launch_count(1, 4096, 4096)
-    assert pq.pq_w4a4_gemm_launch_count_g(1, 4096, 512, 64) == 2      # 8 groups of 64: two ranges
-    assert pq.pq_w4a4_gemm_launch_count_g(1, 4096, 512, 256) == 1     # 2 groups: one range
+        assert pq.pq_w4a4_gemm_launch_count_g(17, 14336, 4096, g) == 1
+        assert pq.pq_w4a4_gemm_launch_count_g(1, 4096, 4096, g) == 1
+    assert pq.pq_w4a4_gemm_launch_count_g(17, 4096, 4096, 128) == pq.pq_w4a4_gemm_launch_count(17, 4096, 4096)
+    assert pq.pq_w4a4_gemm_launch_count_g(17, 4096, 4096, 64) == 2    # 64 groups of 64: ranges
+    assert pq.pq_w4a4_gemm_launch_count_g(17, 4096, 512, 64) == 1     # partial tiles would pass the weights
+    assert pq.pq_w4a4_gemm_launch_count_g(17, 4096, 512, 256) == 1    # 2 groups: one range
 
 
 def test_binding_rejects_host_and_strided_tensors(pq):
