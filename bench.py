@@ -8,8 +8,10 @@ quantise the activations), pq_pack_weights(W) (rotate + quantise the weights), p
 (codes -> Y float32).  Default workload: the largest configuration, the runtime-smoothing +
 block-Hadamard FFN down-projection, X bf16 [8192, 14336] Laplace(0, 1) with 16 outlier channels,
 W bf16 [4096, 14336], g = 128 (synthetic, seeded).  The same run also measures, under "also",
-the Givens K=16 up-projection (the 4096 x 14336 x 4096 W4A4 GEMM) and the block-Hadamard q_proj
-shape.  L2 is flushed (256 MiB write, then a 256 MiB read) before every timed step; each call is
+the Givens K=16 up-projection (the 4096 x 14336 x 4096 W4A4 GEMM), the block-Hadamard q_proj
+shape (also at g = 64 and 256, and with 8 outlier groups kept at 8 bits), rotated runtime
+smoothing on the down_proj shapes, and decode-sized layers (T in {1, 4, 8, 16, 64} at N = 4096
+and 14336: transform and GEMM as two calls and as one pq_w4a4_linear call).  L2 is flushed (256 MiB write, then a 256 MiB read) before every timed step; each call is
 timed with CUDA events on the launching stream, and the sum over K steps is reduced with MAX over
 ranks.  N > 1 runs independent replicas (no data-path collective): ``scaling`` is weak and
 ``value`` is the total over ranks.
