@@ -522,35 +522,79 @@ def roofline_of(wl, comps, peaks, peak_src):
             "algorithmic": f"{per_unit:.4g} bytes per call"}
 
 
+def e2e_chunks(T, N, D):
+    """Token chunks of the end-to-end step: four, in whole 256-token tiles, when each chunk's GEMM
+    takes the same kernels (the same launches, no split that the whole call would not make) as
+    the whole call, so that every output element is computed exactly as unchunked; else one."""
+    from rotation_int4_w4a4_b200 import pq
+    rows = -(-(-(-T // 4)) // 256) * 256
+    chunks = [(t0, min(T, t0 + rows)) for t0 in range(0, T, rows)]
+    whole = pq.pq_w4a4_gemm_launch_count(T, N, D)
+    if T < 1024 or any(pq.pq_w4a4_gemm_launch_count(t1 - t0, N, D) != whole for t0, t1 in chunks):
+        return [(0, T)]
+    return chunks
+
+
 def e2e_run(args, setup, stream):
     """Same step through the public API from pinned host buffers: H2D of X and W, the three
-    calls, D2H of Y, all inside the CUDA-event-timed region."""
+    calls, D2H of Y, all inside the CUDA-event-timed region.  The copies overlap the work, as a
+    caller streaming its inputs would arrange it: W and then X (in token chunks) go over a copy
+    stream; the weight pack starts when W has landed and each chunk's transform and GEMM as soon
+    as its rows have; each chunk of Y goes back over a third stream.  The result must equal the
+    unchunked step's Y bit for bit."""
     import numpy as np
     import torch
     wl, pq, dev = setup.wl, setup.pq, setup.dev
-    T, D, N, G = wl.T, wl.D, wl.N, wl.D // wl.g
+    T, N = wl.T, wl.N
     hX = torch.from_numpy(np.ascontiguousarray(wl.X).view(np.int16)).view(torch.bfloat16).pin_memory()
     hW = torch.from_numpy(np.ascontiguousarray(wl.W).view(np.int16)).view(torch.bfloat16).pin_memory()
     hY = torch.empty((T, N), dtype=torch.float32).pin_memory()
     bs = setup.sets[0]
-    dX, dW = bs["X"], bs["W"]
+    dX, dW, Y, sm = bs["X"], bs["W"], bs["Y"], bs["sm"]
+    # Y of the unchunked step on the same inputs (the timed steps ran on set 0's X and W).
+    pq.pq_transform_quant(setup.plan, dX, bs["ca"], bs["sa"], sm, stream=stream)
+    pq.pq_pack_weights(setup.plan, dW, bs["cw"], bs["sw"], setup.smooth_w, stream=stream)
+    pq.pq_w4a4_gemm(bs["ca"], bs["sa"], bs["cw"], bs["sw"], Y, stream=stream)
+    y_ref = Y.cpu()
+    chunks = e2e_chunks(T, N, wl.D)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     total = 0.0
     n = max(3, min(args.steps, 10))
     for i in range(args.warmup + n):
         setup.flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev_w = torch.cuda.Event()
+        ev_x = [torch.cuda.Event() for _ in chunks]
+        ev_y = [torch.cuda.Event() for _ in chunks]
+        ev_o = torch.cuda.Event()
         e0.record(stream)
-        dX.copy_(hX, non_blocking=True)
-        dW.copy_(hW, non_blocking=True)
-        pq.pq_transform_quant(setup.plan, dX, bs["ca"], bs["sa"], bs["sm"], stream=stream)
+        s_in.wait_event(e0)
+        with torch.cuda.stream(s_in):
+            dW.copy_(hW, non_blocking=True)
+            ev_w.record(s_in)
+            for (t0, t1), ev in zip(chunks, ev_x):
+                dX[t0:t1].copy_(hX[t0:t1], non_blocking=True)
+                ev.record(s_in)
+        stream.wait_event(ev_w)
         pq.pq_pack_weights(setup.plan, dW, bs["cw"], bs["sw"], setup.smooth_w, stream=stream)
-        pq.pq_w4a4_gemm(bs["ca"], bs["sa"], bs["cw"], bs["sw"], bs["Y"], stream=stream)
-        hY.copy_(bs["Y"], non_blocking=True)
+        for (t0, t1), ex, ey in zip(chunks, ev_x, ev_y):
+            stream.wait_event(ex)
+            smk = sm[t0 // 128:(t1 + 127) // 128] if sm is not None else None
+            pq.pq_transform_quant(setup.plan, dX[t0:t1], bs["ca"][t0:t1], bs["sa"][t0:t1], smk, stream=stream)
+            pq.pq_w4a4_gemm(bs["ca"][t0:t1], bs["sa"][t0:t1], bs["cw"], bs["sw"], Y[t0:t1], stream=stream)
+            ey.record(stream)
+            s_out.wait_event(ey)
+            with torch.cuda.stream(s_out):
+                hY[t0:t1].copy_(Y[t0:t1], non_blocking=True)
+        ev_o.record(s_out)
+        stream.wait_event(ev_o)
         e1.record(stream)
         torch.cuda.synchronize()
         if i >= args.warmup:
             total += e0.elapsed_time(e1)
     pq.pq_check_status(setup.plan)
+    if not torch.equal(hY, y_ref):
+        raise RuntimeError("end-to-end step: the chunked result differs from the unchunked step's Y")
     return total / n, hX.numel() * 2 + hW.numel() * 2, hY.numel() * 4
 
 
