@@ -203,6 +203,9 @@ __global__ void __launch_bounds__(RR_MAX_THREADS, 1) rrs_rows_kernel(
         *reinterpret_cast<float4*>(yrow + rr_y_chunk((uint32_t)p * 8 + k)) =
             make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
     }
+    // The next load into buffer b is an async-proxy write: order this thread's generic-proxy
+    // reads of the buffer before it.
+    ptx::fence_proxy_async_smem();
     __syncthreads();   // rotated rows complete; TMA buffer b is free
     if (t == 0 && tile + 2 * stride < num_tiles) issue(tile + 2 * stride, b);
 

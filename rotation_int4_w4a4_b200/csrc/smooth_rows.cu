@@ -143,6 +143,9 @@ __global__ void __launch_bounds__(SR_ROWS, 3) smooth_rows_kernel(
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         row_bf16x8(*reinterpret_cast<const uint4*>(S.x[s][kb] + sr_chunk(t, j)), v + 64 * kb + 8 * j);
+    // The next load into stage s is an async-proxy write: order this thread's generic-proxy reads
+    // of the stage before it (without the fence the copy can overwrite bytes not yet read).
+    ptx::fence_proxy_async_smem();
     __syncthreads();   // every row (and column) of stage s is read; S.mul is complete
     if (t == 0 && tile + 2 * stride < num_tiles) issue(tile + 2 * stride, s);
 
