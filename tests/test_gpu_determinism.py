@@ -110,3 +110,53 @@ def test_hadamard_transform_and_gemm(env, name):
 
     assert repeat_identical(flush, run, (ca, sa, cw, sw, Y)) == 0
     pq.pq_check_status(plan)
+
+
+def test_givens_transform_and_gemm(env):
+    """up_proj: the Givens K = 16 rotation on the tensor cores (two bf16 terms), its weight pack
+    and the 4096 x 14336 x 4096 GEMM."""
+    import torch
+    pq, dev, flush = env
+    wl = inputs.workload("up_proj")
+    T, D, N, G = wl.T, wl.D, wl.N, wl.D // 128
+    X, W = bf16(wl.X, dev), bf16(wl.W, dev)
+    pairs = pq.pq_select_pairs(wl.pair_seed, wl.D, wl.g, wl.K, wl.g // 2)
+    plan = pq.Plan("givens", D, K=wl.K, pairs=pairs, angles=wl.angles, beta=wl.beta)
+    ca = torch.empty((T, D // 2), dtype=torch.uint8, device=dev)
+    sa = torch.empty((T, G), dtype=torch.float32, device=dev)
+    cw = torch.empty((N, D // 2), dtype=torch.uint8, device=dev)
+    sw = torch.empty((N, G), dtype=torch.float32, device=dev)
+    Y = torch.empty((T, N), dtype=torch.float32, device=dev)
+
+    def run():
+        pq.pq_transform_quant(plan, X, ca, sa)
+        pq.pq_pack_weights(plan, W, cw, sw)
+        pq.pq_w4a4_gemm(ca, sa, cw, sw, Y)
+
+    assert repeat_identical(flush, run, (ca, sa, cw, sw, Y)) == 0
+    pq.pq_check_status(plan)
+
+
+@pytest.mark.parametrize("T,N", [(1, 14336), (3, 4096), (16, 4096), (64, 14336)])
+def test_decode_fused_call(env, T, N):
+    """pq_w4a4_linear at decode sizes: the few-row transform, then the CUDA-core (T <= 4) or the
+    few-token tensor-core GEMM (with its range reduction at N = 4096) as a programmatic
+    dependent launch."""
+    import torch
+    pq, dev, flush = env
+    wl = inputs.workload("sweep", T=T, N=N)
+    D, G = wl.D, wl.D // 128
+    X, W = bf16(wl.X, dev), bf16(wl.W, dev)
+    plan = pq.Plan("hadamard", D)
+    cw = torch.empty((N, D // 2), dtype=torch.uint8, device=dev)
+    sw = torch.empty((N, G), dtype=torch.float32, device=dev)
+    pq.pq_pack_weights(plan, W, cw, sw)
+    ca = torch.empty((T, D // 2), dtype=torch.uint8, device=dev)
+    sa = torch.empty((T, G), dtype=torch.float32, device=dev)
+    Y = torch.empty((T, N), dtype=torch.float32, device=dev)
+
+    def run():
+        pq.pq_w4a4_linear(plan, X, ca, sa, cw, sw, Y)
+
+    assert repeat_identical(flush, run, (ca, sa, Y)) == 0
+    pq.pq_check_status(plan)
