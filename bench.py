@@ -523,16 +523,18 @@ def roofline_of(wl, comps, peaks, peak_src):
 
 
 def e2e_chunks(T, N, D):
-    """Token chunks of the end-to-end step: four, in whole 256-token tiles, when each chunk's GEMM
-    takes the same kernels (the same launches, no split that the whole call would not make) as
-    the whole call, so that every output element is computed exactly as unchunked; else one."""
+    """Token chunks of the end-to-end step: eight or else four, in whole 256-token tiles, when
+    each chunk's GEMM takes the same kernels (the same launches, no split that the whole call
+    would not make) as the whole call, so that every output element is computed exactly as
+    unchunked; else one."""
     from rotation_int4_w4a4_b200 import pq
-    rows = -(-(-(-T // 4)) // 256) * 256
-    chunks = [(t0, min(T, t0 + rows)) for t0 in range(0, T, rows)]
     whole = pq.pq_w4a4_gemm_launch_count(T, N, D)
-    if T < 1024 or any(pq.pq_w4a4_gemm_launch_count(t1 - t0, N, D) != whole for t0, t1 in chunks):
-        return [(0, T)]
-    return chunks
+    for n in (8, 4):
+        rows = -(-(-(-T // n)) // 256) * 256
+        chunks = [(t0, min(T, t0 + rows)) for t0 in range(0, T, rows)]
+        if T >= 256 * n and all(pq.pq_w4a4_gemm_launch_count(t1 - t0, N, D) == whole for t0, t1 in chunks):
+            return chunks
+    return [(0, T)]
 
 
 def e2e_run(args, setup, stream):
@@ -540,8 +542,8 @@ def e2e_run(args, setup, stream):
     calls, D2H of Y, all inside the CUDA-event-timed region.  The copies overlap the work, as a
     caller streaming its inputs would arrange it: W and then X (in token chunks) go over a copy
     stream; the weight pack starts when W has landed and each chunk's transform and GEMM as soon
-    as its rows have; each chunk of Y goes back over a third stream.  The result must equal the
-    unchunked step's Y bit for bit."""
+    as its rows have (eight or four chunks, see e2e_chunks); each chunk of Y goes back over a
+    third stream.  The result must equal the unchunked step's Y bit for bit."""
     import numpy as np
     import torch
     wl, pq, dev = setup.wl, setup.pq, setup.dev
