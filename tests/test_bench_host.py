@@ -87,3 +87,21 @@ def test_job_value_is_weak_scaling():
     assert bench.launches_per_step(17, 14336, 4096) == 3       # few tokens, 112 tiles: one launch
     assert bench.launches_per_step(64, 4096, 4096) == 4        # few tokens: ranges + reduce
     assert bench.launches_per_step(17, 272, 4096) == 4         # ragged N: ranges + reduce
+
+
+def test_e2e_chunks_keep_the_whole_calls_kernels():
+    """The end-to-end step splits the tokens only where every chunk's GEMM takes the same kernels
+    as the whole call (no split-K the whole call would not make), in whole 256-token tiles."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from rotation_int4_w4a4_b200 import pq
+    for T, N, D in ((8192, 4096, 14336), (4096, 14336, 4096), (2048, 4096, 4096), (16384, 4096, 4096),
+                    (1000, 4096, 4096), (1, 4096, 4096), (8200, 4096, 14336)):
+        chunks = bench.e2e_chunks(T, N, D)
+        assert chunks[0][0] == 0 and chunks[-1][1] == T
+        assert all(a[1] == b[0] for a, b in zip(chunks, chunks[1:]))
+        assert all(t0 % 256 == 0 for t0, _ in chunks)
+        whole = pq.pq_w4a4_gemm_launch_count(T, N, D)
+        assert all(pq.pq_w4a4_gemm_launch_count(t1 - t0, N, D) == whole for t0, t1 in chunks)
+    assert len(bench.e2e_chunks(8192, 4096, 14336)) == 8          # the default workload
+    assert bench.e2e_chunks(2048, 4096, 4096) == [(0, 2048)]      # 512-token chunks would split K
